@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark one decode step of one attention layer: copy-on-write block
+copies, KV append and paged decode, on the Llama-2-7B-shaped layer (32 query
+heads = 32 KV heads, head_dim 128, fp16, block size 16, batch 64 per GPU,
+context lengths uniform in [512, 4096], random block placement).
+
+Prints one JSON line (rank 0). `value` is KV-path throughput in GB/s: the
+algorithmic bytes of a step (unique KV bytes read by decode, query, output,
+block-table entries and lengths, plus the append's and copies' bytes) over
+the device-timed step; `roofline` relates the decode call's own bytes and
+time to the measured HBM copy bandwidth; `e2e` repeats the measurement with
+the step's inputs copied from pinned host memory and the output read back
+inside the timed region; `cpu_baseline` times the float64 CPU oracle on the
+host's cores on the same inputs.
+
+Multi-GPU (torchrun): every rank runs its own independent batch of the same
+shape (sequences are independent; no data-path collective), so per-GPU work
+is fixed ("weak" scaling); the step time is the max over ranks.
+
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged-decode KV GB/s and % of B200 HBM peak; decode attn tokens/s per layer"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama2_7b.md")
+KERNEL_SOURCES = ["paged_kv_cache_410_b200/csrc/pa_api.cu",
+                  "paged_kv_cache_410_b200/csrc/pa_common.cuh",
+                  "paged_kv_cache_410_b200/csrc/pa_decode.cuh",
+                  "paged_kv_cache_410_b200/csrc/pa_append_copy.cuh"]
+
+
+# ---------------------------------------------------------------- helpers ---
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch: the family's seed plus 1000 * rank."""
+    return 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def make_workload(name: str, rank: int, batch: int | None):
+    from paged_kv_cache_410_b200 import workloads as W
+    fam = W.FAMILIES[name]
+    import inspect
+    kw = {}
+    params = inspect.signature(fam).parameters
+    if batch is not None:
+        kw["batch"] = batch
+    seed = params["seed"].default
+    if seed is None:  # fp8 family derives its seed from the block size
+        seed = W.SEED_BASE + 5 + params["block_size"].default
+    kw["seed"] = seed + rank_seed_offset(rank)
+    return W.make(name, **kw)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources for this workload; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    def field(k):
+        m = re.search(rf"^{k}:\s*(\S+)", text, re.M)
+        return m.group(1) if m else None
+    if field("workload") != workload_name or field("kernel_source_sha256") != kernel_source_hash():
+        return None
+    v = field("dram_bytes_per_full_launch")
+    return float(v) if v else None
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line.strip())
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------ CPU oracle ---
+
+def oracle_step_time(w, seqs, reps=1):
+    """Seconds for `reps` oracle passes (append of the sample's tokens +
+    decode of the sample) over the sampled sequences."""
+    import oracle
+    from paged_kv_cache_410_b200 import workloads as W
+    s = W.subset(w, seqs)
+    if w.cache_dtype == "e4m3":
+        raise NotImplementedError("the CPU baseline is timed on 16-bit caches")
+    kc, vc = w.k_pool, w.v_pool  # the oracle append rewrites the same slots each pass
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.append_kv(s.k_new, s.v_new, s.io_dtype, s.slot_mapping, kc, vc, s.cache_dtype,
+                         s.block_size)
+        oracle.decode(s.q, s.io_dtype, kc, vc, s.cache_dtype, s.block_tables, s.context_lens,
+                      s.scale)
+    return time.perf_counter() - t0, s
+
+
+def cpu_baseline(w, target_s=12.0):
+    """Oracle throughput on a bounded sample: whole passes over the batch (or
+    the first sequences of it) repeated until about `target_s` seconds."""
+    import oracle
+    from paged_kv_cache_410_b200 import accounting as A
+    t1, s1 = oracle_step_time(w, np.arange(1))
+    per_seq = max(t1, 1e-4)
+    n = int(min(w.batch, max(1, target_s / per_seq)))
+    seqs = np.arange(n)
+    t, s = oracle_step_time(w, seqs)
+    reps = max(1, int(target_s / max(t, 1e-6)))
+    if reps > 1:
+        t, s = oracle_step_time(w, seqs, reps)
+    nbytes = A.step_bytes(s)["total"] * reps
+    return {"value": nbytes / t / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of {w.batch} sequences x {reps} passes (append + decode), "
+                      f"{t:.1f} s, float64 C oracle, OpenMP over (sequence, head)",
+            "seconds": t, "tokens_per_s_per_layer": n * reps / t}
+
+
+# ----------------------------------------------------------------- main ----
+
+def base_line(args, w, n_gpus):
+    return {"metric": METRIC, "unit": UNIT, "n_gpus": n_gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.cache_dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch,
+                       "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+                       "head_dim": w.head_dim, "block_size": w.block_size,
+                       "context_lens": f"{int(w.context_lens.min())}..{int(w.context_lens.max())}"
+                                       f" (mean {float(w.context_lens.mean()):.0f})",
+                       "kv_cache_dtype": w.cache_dtype, "io_dtype": w.io_dtype,
+                       "parallelism": f"independent batch per GPU x{n_gpus}",
+                       "l2": "not flushed: the step reads more than the 126 MB L2 "
+                             f"(pool {2 * w.num_blocks * w.block_size * w.num_kv_heads * w.head_dim * (1 if w.cache_dtype == 'e4m3' else 2) / 1e9:.2f} GB)"}}
+
+
+def run_reference(args):
+    rank, local_rank, world = dist_env()
+    if rank != 0:
+        return 0
+    w = make_workload(args.workload, 0, args.batch)
+    from paged_kv_cache_410_b200 import accounting as A
+    import oracle
+    oracle.build()
+    # per-step sample sized so warmup + steps fit in about two minutes
+    budget = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    t1, _ = oracle_step_time(w, np.arange(1))
+    n = int(min(w.batch, max(1, budget / max(t1, 1e-4))))
+    seqs = np.arange(n)
+    for _ in range(args.warmup):
+        oracle_step_time(w, seqs)
+    times = []
+    s = None
+    for _ in range(args.steps):
+        t, s = oracle_step_time(w, seqs)
+        times.append(t)
+    total = sum(times)
+    nbytes = A.step_bytes(s)["total"] * args.steps
+    value = nbytes / total / 1e9
+    line = base_line(args, w, world)
+    line["dtype"] = "f64"
+    line.update({"impl": "reference", "value": value, "ms_per_step": 1e3 * total / args.steps,
+                 "tokens_per_s_per_layer": n * args.steps / total,
+                 "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"{n} of {w.batch} sequences per step "
+                                            "(append + decode), float64 C oracle"},
+                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                         "d2h_bytes_per_step": 0},
+                 "gpu_launches": 0})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    from paged_kv_cache_410_b200 import accounting as A
+    from paged_kv_cache_410_b200 import binding as B
+    from paged_kv_cache_410_b200 import build as libbuild
+    from paged_kv_cache_410_b200.session import DecodeStep
+    if not os.path.exists(libbuild.LIB):
+        raise RuntimeError("libpagedattn.so is not built; run __graft_entry__.build()")
+
+    w = make_workload(args.workload, rank, args.batch)
+    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens)
+    stream = torch.cuda.current_stream(dev)
+    sb = A.step_bytes(w)
+    plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context,
+                                                                     step.cache)
+    n_parts = max(1, math.ceil(w.max_context / plan_pt))
+    launches_per_step = (1 + 1 + (1 if n_parts > 1 else 0) +
+                         math.ceil(len(w.copy_pairs) / 256))
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize(dev)
+    if step.device_errors():
+        raise RuntimeError("device bounds error during warm-up")
+
+    # ---- device-timed steps, per-call events for the decode roofline ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.25)  # let the sampler start before the timed region
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step.copy()
+        step.append()
+        ev[i][0].record(stream)
+        step.decode()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_local = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_total = max_over_ranks(ms_local, dev)
+    ms_per_step = ms_total / args.steps
+    total_bytes = sum_over_ranks(sb["total"], dev) * args.steps
+    value = total_bytes / (ms_total * 1e-3) / 1e9
+    tokens_per_s = sum_over_ranks(w.batch, dev) * args.steps / (ms_total * 1e-3)
+
+    # ---- end to end: host inputs -> device -> host output, every step ----
+    pinned = {k: getattr(step, k).cpu().pin_memory()
+              for k in ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")}
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        for k, t in pinned.items():
+            getattr(step, k).copy_(t, non_blocking=True)
+        step.run()
+        out_host.copy_(step.out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k, t in pinned.items():
+            getattr(step, k).copy_(t, non_blocking=True)
+        step.run()
+        out_host.copy_(step.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = sum_over_ranks(sb["total"], dev) * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    errs = step.device_errors()
+
+    # ---- roofline of the decode call ----
+    peaks = measured_peaks()
+    if peaks and peaks.get("hbm_gbs"):
+        peak, peak_src = float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    else:
+        peak, peak_src = FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+    dec_ms = statistics.mean(decode_ms)
+    achieved = sb["decode"] / (dec_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name)
+
+    line = base_line(args, w, world)
+    line.update({
+        "value": value, "ms_per_step": ms_per_step,
+        "tokens_per_s_per_layer": tokens_per_s,
+        "frac_of_hbm_peak": value / peak,
+        "frac_of_hbm_spec_8tbs": value / SPEC_HBM_GBS,
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": sb["decode"],
+                     "decode_ms_mean": dec_ms, "decode_ms_median": statistics.median(decode_ms),
+                     "partition_tokens": plan_pt, "partitions": n_parts},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "bytes_per_step": sb,
+        "clocks": clk,
+        "device_errors": errs,
+    })
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        line["cpu_baseline"] = cpu_baseline(w)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2_7b")
+    ap.add_argument("--batch", type=int, default=None, help="sequences per GPU (default: the family's)")
+    ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

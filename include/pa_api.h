@@ -1,0 +1,167 @@
+/*
+ * pa_api.h -- C ABI of the B200 (sm_100a) paged-attention decode library
+ * (libpagedattn.so).
+ *
+ * Three operations make up one decode step of one attention layer:
+ *
+ *   pa_append_kv    store each new token's K and V in its cache slot;
+ *   pa_decode       one query token per sequence attends to that sequence's
+ *                   whole cached history, gathered through its block table;
+ *   pa_copy_blocks  duplicate whole blocks (copy-on-write at a fork).
+ *
+ * Sources of the definitions (page titles and sections):
+ *  - "AI 陪读顶会论文（三）：KV Cache 显存占用计算与 PagedAttention 原理拆解",
+ *    section "为什么自回归解码必须使用 KV Cache？": the attention equation
+ *    o = softmax(q_t K_{1:t}^T / sqrt(d)) V_{1:t}, and the rule that each
+ *    step computes only the new token's k_t, v_t and appends them;
+ *    section "PagedAttention 的破局哲学": fixed-size blocks (16 tokens by
+ *    default) in arbitrary physical places, a block table per sequence,
+ *    copy-on-write for branches that share prompt blocks.
+ *  - KV cache article (ainews.alishangtian.com), section
+ *    "PagedAttention：把操作系统的老智慧搬进推理引擎": block table, shared
+ *    prefix blocks stored once and reference-counted, copy-on-write at the
+ *    fork point; section "显存账本：长上下文时代，KV cache 反超权重": grouped-
+ *    query attention (several query heads share one KV head); section
+ *    "再往后：压 KV 的三条路线": FP8 K/V with per-channel scaling factors.
+ *
+ * Conventions shared by every entry point
+ *  - Every tensor argument is a DEVICE pointer to caller-owned memory (for
+ *    example a torch tensor's data_ptr()), dense and row-major in the layout
+ *    stated, and 16-byte aligned. The library allocates no device memory;
+ *    pa_decode's split-K workspace is supplied by the caller.
+ *  - KV cache layout: [num_blocks][block_size][num_kv_heads][head_dim]. The
+ *    token at logical position j of sequence b lives in physical block
+ *    block_tables[b * max_blocks_per_seq + j / block_size], row
+ *    j % block_size; slot s names block s / block_size, row s % block_size.
+ *  - Query head i reads KV head i / (num_q_heads / num_kv_heads).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream); every
+ *    call is asynchronous on it and returns after enqueueing its kernels.
+ *  - Arguments are checked on the host before anything is enqueued; a
+ *    failed check returns PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED and leaves
+ *    all memory untouched. Values that live in device memory (slots, block
+ *    ids, context lengths) are checked by the kernels: an out-of-range value
+ *    sets a bit in a per-device error word and the access it would have made
+ *    is skipped (reads yield zeros, writes are dropped); pa_get_device_error
+ *    reports and clears that word.
+ *  - Supported: block_size a power of two in [1, 256]; head_dim 64 or 128;
+ *    16-bit caches (PA_F16, PA_BF16) whose dtype equals the input's, or an
+ *    E4M3 cache with fp16 or bf16 inputs; num_q_heads a multiple of
+ *    num_kv_heads.
+ */
+#ifndef PA_API_H
+#define PA_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,   /* a host-side argument check failed */
+  PA_ERR_UNSUPPORTED = 2,   /* valid, but a dtype/shape this build has no kernel for */
+  PA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  PA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+  PA_ERR_DEVICE_BOUNDS = 5  /* pa_get_device_error: a kernel saw an out-of-range value */
+} pa_status;
+
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
+
+/* Bits of the device error word (pa_get_device_error). */
+#define PA_DEVERR_BLOCK_ID 0x1u    /* a block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2u /* context_len < 0, > max_context, or beyond the table */
+#define PA_DEVERR_SLOT 0x4u        /* append slot >= num_blocks * block_size */
+
+/* Describes one paged KV cache (one layer's K cache and V cache). */
+typedef struct pa_cache_desc {
+  int64_t num_blocks;    /* physical blocks in each of the K and V caches */
+  int32_t block_size;    /* tokens per block: power of two in [1, 256] */
+  int32_t num_kv_heads;
+  int32_t head_dim;      /* 64 or 128 */
+  int32_t cache_dtype;   /* pa_dtype */
+  /* E4M3 caches only (NULL otherwise): device fp32 arrays [num_kv_heads *
+   * head_dim]. A stored code c of head h, channel d stands for
+   * e4m3(c) * scale[h*head_dim + d]; append stores
+   * e4m3_rn_satfinite(fp32(x) * inv_scale[h*head_dim + d]). */
+  const float* k_scale;
+  const float* v_scale;
+  const float* k_inv_scale;
+  const float* v_inv_scale;
+} pa_cache_desc;
+
+/* Store new tokens' K and V into their cache slots.
+ *   k, v          [num_tokens][num_kv_heads][head_dim] in in_dtype (PA_F16
+ *                 or PA_BF16).
+ *   slot_mapping  [num_tokens] int64; slot < 0 skips the token (padding).
+ *   k_cache, v_cache  caches described by `cache`; a 16-bit cache receives
+ *                 the input bits unchanged (its dtype must equal in_dtype);
+ *                 an E4M3 cache receives the quantised codes.
+ * Slots of one call must be distinct (two tokens written to one slot race).
+ * num_tokens == 0 is a no-op. */
+pa_status pa_append_kv(const void* k, const void* v, int32_t in_dtype, int64_t num_tokens,
+                       const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                       const pa_cache_desc* cache, void* stream);
+
+/* Bytes of workspace pa_decode needs for these sizes and this partition
+ * choice (0 when one partition covers max_context). Pure host function. */
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t max_context,
+                                int32_t partition_tokens, const pa_cache_desc* cache);
+
+/* Tokens per split-K partition that pa_decode uses for these sizes when
+ * called with partition_tokens == 0. Pure host function. */
+int32_t pa_decode_partition_tokens(int32_t batch, int32_t max_context,
+                                   const pa_cache_desc* cache);
+
+/* Single-query paged attention for a batch of sequences:
+ *   out[b][i][:] = softmax_j(scale * q[b][i] . K_j) V_j over the
+ *   context_lens[b] cached tokens of sequence b, KV head i / group.
+ *   q             [batch][num_q_heads][head_dim], q_dtype PA_F16 or PA_BF16
+ *                 (for a 16-bit cache q_dtype must equal the cache dtype).
+ *   block_tables  [batch][max_blocks_per_seq] int32 physical block ids;
+ *                 entries past ceil(context_lens[b] / block_size) are not read.
+ *   context_lens  [batch] int32, each in [0, max_context]; 0 gives a zero row.
+ *   max_context   host-side upper bound of context_lens (sizes the launch).
+ *   scale         multiplies q.K before the softmax (1/sqrt(head_dim)).
+ *   out           [batch][num_q_heads][head_dim] in q_dtype.
+ *   partition_tokens  0 lets the library split long contexts; otherwise a
+ *                 multiple of 16 in [16, 1 << 20] fixes the split-K partition
+ *                 length (results agree up to rounding for any choice).
+ *   workspace     device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes (may be NULL when that size is 0), 256-byte aligned.
+ * Blocks may be shared between sequences (shared prefixes, beams); the
+ * caches are only read. */
+pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                    const void* k_cache, const void* v_cache, const pa_cache_desc* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context, float scale, void* out,
+                    int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Copy whole blocks: for p in [0, num_pairs), K block pairs_host[2p] ->
+ * K block pairs_host[2p+1], and the same for V.
+ *   pairs_host    HOST array of num_pairs (src, dst) int32 pairs, read before
+ *                 the call returns (passed to the kernel by value).
+ * Every id must be in [0, num_blocks), destinations distinct, and no
+ * destination may also be a source (then the order of copies cannot
+ * matter); otherwise PA_ERR_INVALID_ARG. num_pairs == 0 is a no-op. */
+pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_cache,
+                         void* v_cache, const pa_cache_desc* cache, void* stream);
+
+/* Synchronise `stream`, then read and clear the current device's error
+ * word into *flags (PA_DEVERR_* bits). Returns PA_ERR_DEVICE_BOUNDS when
+ * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure. */
+pa_status pa_get_device_error(void* stream, uint32_t* flags);
+
+/* Static text for a status code. */
+const char* pa_status_string(int32_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_API_H */

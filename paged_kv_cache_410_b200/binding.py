@@ -1,0 +1,197 @@
+"""Python binding of libpagedattn.so (ctypes, argument marshalling only).
+
+Each function forwards torch tensors' device pointers and sizes to the C
+entry point of the same name (include/pa_api.h); every step of the hot path
+runs in the library's CUDA kernels. Torch provides device memory and
+streams. If the library is not built the first call raises: there is no
+fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpagedattn.so")
+
+PA_F16, PA_BF16, PA_E4M3 = 0, 1, 2
+PA_OK = 0
+STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
+          4: "PA_ERR_WORKSPACE", 5: "PA_ERR_DEVICE_BOUNDS"}
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT = 0x1, 0x2, 0x4
+
+# names of every symbol include/pa_api.h declares
+EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tokens",
+            "pa_decode", "pa_copy_blocks", "pa_get_device_error", "pa_status_string",
+            "pa_version"]
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class _CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("cache_dtype", ctypes.c_int32), ("k_scale", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("k_inv_scale", ctypes.c_void_p),
+                ("v_inv_scale", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libpagedattn.so and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built (run paged_kv_cache_410_b200.build.build());"
+                           " the paged-attention path has no fallback")
+    lib = ctypes.CDLL(path)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    D = ctypes.POINTER(_CacheDesc)
+    lib.pa_append_kv.argtypes = [P, P, i32, i64, P, P, P, D, P]
+    lib.pa_append_kv.restype = ctypes.c_int
+    lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, D]
+    lib.pa_decode_workspace_size.restype = ctypes.c_size_t
+    lib.pa_decode_partition_tokens.argtypes = [i32, i32, D]
+    lib.pa_decode_partition_tokens.restype = i32
+    lib.pa_decode.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, ctypes.c_float, P, i32,
+                              P, ctypes.c_size_t, P]
+    lib.pa_decode.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [P, i32, P, P, D, P]
+    lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.pa_get_device_error.restype = ctypes.c_int
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float16:
+        return PA_F16
+    if t == torch.bfloat16:
+        return PA_BF16
+    if t in (torch.uint8, torch.float8_e4m3fn):
+        return PA_E4M3
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+@dataclass
+class PagedCache:
+    """Shape and (for E4M3) scales of one layer's paged K and V caches,
+    laid out [num_blocks, block_size, num_kv_heads, head_dim]."""
+    num_blocks: int
+    block_size: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: torch.dtype
+    k_scale: torch.Tensor | None = None      # fp32 [num_kv_heads, head_dim], device
+    v_scale: torch.Tensor | None = None
+    k_inv_scale: torch.Tensor | None = None
+    v_inv_scale: torch.Tensor | None = None
+
+    def desc(self) -> _CacheDesc:
+        return _CacheDesc(self.num_blocks, self.block_size, self.num_kv_heads, self.head_dim,
+                          _dtype_code(self.dtype), _ptr(self.k_scale), _ptr(self.v_scale),
+                          _ptr(self.k_inv_scale), _ptr(self.v_inv_scale))
+
+    @staticmethod
+    def for_tensor(cache: torch.Tensor, **scales) -> "PagedCache":
+        nb, bs, hkv, d = cache.shape
+        return PagedCache(nb, bs, hkv, d, cache.dtype, **scales)
+
+
+def _check(rc: int, what: str):
+    if rc != PA_OK:
+        raise PagedAttentionError(rc, what)
+
+
+def pa_append_kv(k, v, slot_mapping, k_cache, v_cache, cache: PagedCache, stream=None):
+    """Store k, v ([T, Hkv, D], fp16/bf16) at slot_mapping ([T] int64)."""
+    lib = load_library()
+    d = cache.desc()
+    rc = lib.pa_append_kv(_ptr(k), _ptr(v), _dtype_code(k.dtype), k.shape[0],
+                          _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+                          _stream(stream))
+    _check(rc, "pa_append_kv")
+
+
+def pa_decode_workspace_size(batch, num_q_heads, max_context, cache: PagedCache,
+                             partition_tokens=0) -> int:
+    lib = load_library()
+    d = cache.desc()
+    return int(lib.pa_decode_workspace_size(batch, num_q_heads, max_context, partition_tokens,
+                                            ctypes.byref(d)))
+
+
+def pa_decode_partition_tokens(batch, max_context, cache: PagedCache) -> int:
+    lib = load_library()
+    d = cache.desc()
+    return int(lib.pa_decode_partition_tokens(batch, max_context, ctypes.byref(d)))
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache: PagedCache,
+              max_context: int, partition_tokens: int = 0, workspace=None, stream=None):
+    """out[b, i] = softmax(scale * q[b, i] . K^T) V over sequence b's paged
+    history. `workspace` is a uint8 device tensor of at least
+    pa_decode_workspace_size(...) bytes (or None when that is 0)."""
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.pa_decode(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache), _ptr(v_cache),
+                       ctypes.byref(d), _ptr(block_tables), block_tables.shape[1],
+                       _ptr(context_lens), int(max_context), float(scale), _ptr(out),
+                       int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "pa_decode")
+
+
+def pa_copy_blocks(pairs, k_cache, v_cache, cache: PagedCache, stream=None):
+    """Copy K and V block pairs[p][0] -> pairs[p][1]; `pairs` is host data."""
+    lib = load_library()
+    d = cache.desc()
+    arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    rc = lib.pa_copy_blocks(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], _ptr(k_cache),
+                            _ptr(v_cache), ctypes.byref(d), _stream(stream))
+    _check(rc, "pa_copy_blocks")
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error bits."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    rc = lib.pa_get_device_error(_stream(stream), ctypes.byref(flags))
+    if rc not in (PA_OK, 5):
+        raise PagedAttentionError(rc, "pa_get_device_error")
+    return int(flags.value)
+
+
+def pa_status_string(status: int) -> str:
+    return load_library().pa_status_string(status).decode()
+
+
+def pa_version() -> int:
+    return int(load_library().pa_version())

@@ -1,0 +1,330 @@
+// Host side of the C ABI declared in include/pa_api.h: argument checks,
+// split-K planning, template dispatch and launches. All kernels of the
+// library live in this one translation unit (they share the device error
+// word).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <type_traits>
+#include <unordered_set>
+
+#include "pa_api.h"
+#include "pa_append_copy.cuh"
+#include "pa_common.cuh"
+#include "pa_decode.cuh"
+
+namespace {
+
+constexpr int kNumSMs = 148;         // B200
+constexpr int kDecodeWarps = 4;      // warps per decode CTA
+constexpr int kDecodeStages = 3;     // cp.async stages per warp
+constexpr int kDefaultPartition = 512;
+constexpr int kMinAutoPartition = 64;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool pow2_log(int v, int* lg) {
+  if (v <= 0 || (v & (v - 1)) != 0) return false;
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  *lg = l;
+  return true;
+}
+
+pa_status check_cache(const pa_cache_desc* cd, int* bs_log2) {
+  if (!cd) return PA_ERR_INVALID_ARG;
+  if (cd->num_blocks <= 0 || cd->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
+  if (!pow2_log(cd->block_size, bs_log2) || cd->block_size > 256) return PA_ERR_INVALID_ARG;
+  if (cd->cache_dtype != PA_F16 && cd->cache_dtype != PA_BF16 && cd->cache_dtype != PA_E4M3)
+    return PA_ERR_INVALID_ARG;
+  if (cd->head_dim != 64 && cd->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+int64_t elem_bytes(int dtype) { return dtype == PA_E4M3 ? 1 : 2; }
+
+// Partition length used when the caller passes 0: 512 tokens, halved (down
+// to 64) while the launch would have fewer than two CTAs per SM.
+int auto_partition(int64_t batch, int64_t max_context, int64_t num_kv_heads) {
+  int pt = kDefaultPartition;
+  auto ctas = [&](int p) { return batch * num_kv_heads * ((max_context + p - 1) / p); };
+  while (pt > kMinAutoPartition && ctas(pt) < 2 * kNumSMs) pt >>= 1;
+  return pt;
+}
+
+struct Plan {
+  int partition_tokens;
+  int num_partitions;
+  size_t ws_o_bytes;
+  size_t ws_bytes;
+};
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int partition_tokens,
+               const pa_cache_desc* cd) {
+  Plan pl{};
+  pl.partition_tokens = partition_tokens > 0
+                            ? partition_tokens
+                            : auto_partition(batch, max_context, cd->num_kv_heads);
+  const int64_t np = (max_context + pl.partition_tokens - 1) / pl.partition_tokens;
+  pl.num_partitions = static_cast<int>(std::max<int64_t>(np, 1));
+  if (pl.num_partitions > 1) {
+    pl.ws_o_bytes = round_up(static_cast<size_t>(batch * num_q_heads) * pl.num_partitions *
+                                 cd->head_dim * sizeof(float),
+                             256);
+    pl.ws_bytes = pl.ws_o_bytes + round_up(static_cast<size_t>(batch * num_q_heads) *
+                                               pl.num_partitions * sizeof(float2),
+                                           256);
+  }
+  return pl;
+}
+
+// cudaFuncSetAttribute once per (kernel, device).
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes) {
+  static std::atomic<uint64_t> done_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <typename TQ, int CK, int D, bool TWO>
+pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
+  using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
+  auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, TWO>;
+  const int bt_entries = (p.partition_tokens >> p.bs_log2) + 2;
+  const int smem = S::kMainBytes + bt_entries * 4;
+  if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
+  if (ensure_smem(kern, smem) != cudaSuccess) return PA_ERR_CUDA;
+  dim3 grid(p.num_partitions, p.num_kv_heads * p.head_groups, p.batch);
+  kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (p.num_partitions > 1) {
+    pa::pa_decode_reduce_kernel<TQ, D><<<dim3(p.num_q_heads, p.batch), 128, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+template <typename TQ, int CK>
+pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, cudaStream_t st) {
+  const bool two = std::min(p.group, 16) > 8;
+  if (head_dim == 64)
+    return two ? launch_decode_t<TQ, CK, 64, true>(p, st) : launch_decode_t<TQ, CK, 64, false>(p, st);
+  return two ? launch_decode_t<TQ, CK, 128, true>(p, st)
+             : launch_decode_t<TQ, CK, 128, false>(p, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(int32_t s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported dtype or shape";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_DEVICE_BOUNDS: return "a kernel saw an out-of-range slot, block id or length";
+    default: return "unknown status";
+  }
+}
+
+int32_t pa_version(void) { return 100; }
+
+pa_status pa_append_kv(const void* k, const void* v, int32_t in_dtype, int64_t num_tokens,
+                       const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                       const pa_cache_desc* cache, void* stream) {
+  int bs_log2 = 0;
+  pa_status st = check_cache(cache, &bs_log2);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (in_dtype != PA_F16 && in_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype != PA_E4M3 && cache->cache_dtype != in_dtype) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  pa::AppendParams p{};
+  p.k = k;
+  p.v = v;
+  p.slots = slot_mapping;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.num_slots = cache->num_blocks * cache->block_size;
+  p.row_elems = cache->num_kv_heads * cache->head_dim;
+  const cudaStream_t s = as_stream(stream);
+  const dim3 grid(static_cast<unsigned>(num_tokens));
+  if (cache->cache_dtype == PA_E4M3) {
+    if (!cache->k_inv_scale || !cache->v_inv_scale) return PA_ERR_INVALID_ARG;
+    if (!aligned16(cache->k_inv_scale) || !aligned16(cache->v_inv_scale))
+      return PA_ERR_INVALID_ARG;
+    p.k_inv_scale = cache->k_inv_scale;
+    p.v_inv_scale = cache->v_inv_scale;
+    if (in_dtype == PA_F16)
+      pa::pa_append_kernel<1><<<grid, 128, 0, s>>>(p);
+    else
+      pa::pa_append_kernel<2><<<grid, 128, 0, s>>>(p);
+  } else {
+    pa::pa_append_kernel<0><<<grid, 128, 0, s>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t max_context,
+                                int32_t partition_tokens, const pa_cache_desc* cache) {
+  int bs_log2 = 0;
+  if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || num_q_heads <= 0 ||
+      max_context < 0 || partition_tokens < 0)
+    return 0;
+  return make_plan(batch, num_q_heads, max_context, partition_tokens, cache).ws_bytes;
+}
+
+int32_t pa_decode_partition_tokens(int32_t batch, int32_t max_context,
+                                   const pa_cache_desc* cache) {
+  int bs_log2 = 0;
+  if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || max_context < 0) return 0;
+  return auto_partition(batch, max_context, cache->num_kv_heads);
+}
+
+pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                    const void* k_cache, const void* v_cache, const pa_cache_desc* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context, float scale, void* out,
+                    int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  int bs_log2 = 0;
+  pa_status st = check_cache(cache, &bs_log2);
+  if (st != PA_OK) return st;
+  if (batch < 0 || num_q_heads <= 0 || max_context < 0 || max_blocks_per_seq <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype != PA_E4M3 && cache->cache_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  if (partition_tokens != 0 &&
+      (partition_tokens < 16 || partition_tokens > (1 << 20) || partition_tokens % 16 != 0))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (batch == 0) return PA_OK;
+  if (batch > 65535) return PA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype == PA_E4M3 && (!cache->k_scale || !cache->v_scale))
+    return PA_ERR_INVALID_ARG;
+
+  const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (pl.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
+  }
+  const int group = num_q_heads / cache->num_kv_heads;
+  const int head_groups = (group + 15) / 16;
+  if (static_cast<int64_t>(cache->num_kv_heads) * head_groups > 65535) return PA_ERR_UNSUPPORTED;
+
+  pa::DecodeParams p{};
+  p.q = q;
+  p.out = out;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
+  p.ws_ml = pl.ws_bytes
+                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
+                : nullptr;
+  p.num_blocks = cache->num_blocks;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.group = group;
+  p.head_groups = head_groups;
+  p.bs_log2 = bs_log2;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context = max_context;
+  p.partition_tokens = pl.partition_tokens;
+  p.num_partitions = pl.num_partitions;
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  const cudaStream_t s = as_stream(stream);
+  switch (cache->cache_dtype) {
+    case PA_F16: return launch_decode_d<__half, pa::kF16>(p, cache->head_dim, s);
+    case PA_BF16: return launch_decode_d<__nv_bfloat16, pa::kBF16>(p, cache->head_dim, s);
+    default:
+      return q_dtype == PA_F16 ? launch_decode_d<__half, pa::kE4M3>(p, cache->head_dim, s)
+                               : launch_decode_d<__nv_bfloat16, pa::kE4M3>(p, cache->head_dim, s);
+  }
+}
+
+pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_cache,
+                         void* v_cache, const pa_cache_desc* cache, void* stream) {
+  int bs_log2 = 0;
+  pa_status st = check_cache(cache, &bs_log2);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!pairs_host || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  std::unordered_set<int32_t> srcs, dsts;
+  for (int32_t i = 0; i < num_pairs; ++i) {
+    const int32_t s = pairs_host[2 * i], d = pairs_host[2 * i + 1];
+    if (s < 0 || d < 0 || s >= cache->num_blocks || d >= cache->num_blocks)
+      return PA_ERR_INVALID_ARG;
+    if (!dsts.insert(d).second) return PA_ERR_INVALID_ARG;
+    srcs.insert(s);
+  }
+  for (int32_t d : dsts)
+    if (srcs.count(d)) return PA_ERR_INVALID_ARG;
+
+  const int64_t block_bytes = static_cast<int64_t>(cache->block_size) * cache->num_kv_heads *
+                              cache->head_dim * elem_bytes(cache->cache_dtype);
+  pa::CopyParams p{};
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_vec16 = block_bytes / 16;
+  const int64_t slices = std::min<int64_t>(std::max<int64_t>(p.block_vec16 / (256 * 4), 1), 64);
+  const cudaStream_t s = as_stream(stream);
+  for (int32_t base = 0; base < num_pairs; base += pa::kCopyPairsPerLaunch) {
+    const int n = std::min(num_pairs - base, pa::kCopyPairsPerLaunch);
+    p.num_pairs = n;
+    for (int i = 0; i < n; ++i)
+      p.pairs[i] = make_int2(pairs_host[2 * (base + i)], pairs_host[2 * (base + i) + 1]);
+    pa::pa_copy_blocks_kernel<<<dim3(n, static_cast<unsigned>(slices)), 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+pa_status pa_get_device_error(void* stream, uint32_t* flags) {
+  if (!flags) return PA_ERR_INVALID_ARG;
+  *flags = 0;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_pa_error_word, sizeof(v)) != cudaSuccess) return PA_ERR_CUDA;
+  if (v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(pa::g_pa_error_word, &zero, sizeof(zero)) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  *flags = v;
+  return v ? PA_ERR_DEVICE_BOUNDS : PA_OK;
+}
+
+}  // extern "C"

@@ -344,7 +344,24 @@ def fp8_beams(batch=256, block_size=16, beam_groups=16, beam_width=4, median_len
               "group_lens": group_lens.tolist()})
 
 
+def custom(lens, num_q_heads=8, num_kv_heads=8, head_dim=64, block_size=16, dtype="f16",
+           headroom=0.25, seed=SEED_BASE) -> Workload:
+    """Any shape, for edge cases: decode lengths ``lens`` (0 allowed: such a
+    sequence appends nothing), private blocks from a seeded permutation of a
+    pool with ``headroom`` spare blocks, 16-bit cache."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, dtype=np.int64)
+    need = int(sum(-(-int(L) // block_size) for L in lens))
+    NB = max(_pool_size(need, headroom), 1)
+    placer = _Placer(rng, NB)
+    block_lists = [placer.take(-(-int(L) // block_size)) for L in lens]
+    return _finish_16bit("custom", rng, B=len(lens), Hq=num_q_heads, Hkv=num_kv_heads,
+                         D=head_dim, BS=block_size, NB=NB, dtype=dtype, lens=lens,
+                         block_lists=block_lists, meta={})
+
+
 FAMILIES = {
+    "custom": custom,
     "tiny_mha": tiny_mha,
     "llama2_7b": llama2_7b,
     "llama2_70b_prefix": llama2_70b_prefix,

@@ -1,0 +1,127 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad host-side arguments before touching the
+GPU (every call below returns from its argument checks, so no device is
+needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from paged_kv_cache_410_b200 import binding as B
+from paged_kv_cache_410_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa_api.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return B.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names == sorted(B.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pa_version() >= 100
+    for s in range(6):
+        assert lib.pa_status_string(s)
+    assert B.pa_status_string(1) == "invalid argument"
+
+
+def _desc(**kw):
+    d = dict(num_blocks=8, block_size=16, num_kv_heads=2, head_dim=64, cache_dtype=B.PA_F16,
+             k_scale=None, v_scale=None, k_inv_scale=None, v_inv_scale=None)
+    d.update(kw)
+    return B._CacheDesc(**d)
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced here
+
+
+def test_copy_blocks_rejects_conflicting_pairs(lib):
+    d = _desc()
+    for pairs in ([[1, 2], [3, 2]],      # duplicate destination
+                  [[1, 2], [2, 3]],      # destination is also a source
+                  [[1, 8]],              # out of range
+                  [[-1, 2]]):
+        arr = np.asarray(pairs, np.int32)
+        rc = lib.pa_copy_blocks(arr.ctypes.data_as(ctypes.c_void_p), len(arr), FAKE, FAKE,
+                                ctypes.byref(d), None)
+        assert rc == 1, pairs
+    assert lib.pa_copy_blocks(None, 0, FAKE, FAKE, ctypes.byref(d), None) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("block_size", 24, 1), ("block_size", 512, 1), ("head_dim", 96, 2), ("cache_dtype", 7, 1),
+    ("num_blocks", 0, 1), ("num_kv_heads", 0, 1),
+])
+def test_bad_cache_descriptors(lib, field, value, status):
+    d = _desc(**{field: value})
+    rc = lib.pa_decode(FAKE, 0, 1, 2, FAKE, FAKE, ctypes.byref(d), FAKE, 4, FAKE, 64, 0.1, FAKE,
+                       0, None, 0, None)
+    assert rc == status
+
+
+def test_decode_argument_checks(lib):
+    d = _desc()
+    call = lambda **kw: lib.pa_decode(*[kw.get(k, v) for k, v in [
+        ("q", FAKE), ("q_dtype", 0), ("batch", 2), ("hq", 4), ("k", FAKE), ("v", FAKE),
+        ("desc", ctypes.byref(d)), ("bt", FAKE), ("mb", 4), ("lens", FAKE), ("maxc", 64),
+        ("scale", 0.1), ("out", FAKE), ("pt", 0), ("ws", None), ("wsb", 0), ("s", None)]])
+    assert call(hq=3) == 1                    # not a multiple of num_kv_heads
+    assert call(q_dtype=1) == 2               # bf16 query on an fp16 cache
+    assert call(pt=24) == 1                   # partition not a multiple of 16
+    assert call(q=FAKE + 4) == 1              # misaligned
+    assert call(scale=float("nan")) == 1
+    assert call(batch=0) == 0                 # nothing to do
+    assert call(out=None) == 1
+    # a split plan needs a workspace
+    need = lib.pa_decode_workspace_size(2, 4, 5000, 64, ctypes.byref(d))
+    assert need > 0
+    assert call(maxc=5000, pt=64) == 4
+    assert call(maxc=5000, pt=64, ws=FAKE + 16, wsb=need) == 4  # not 256-byte aligned
+    assert call(maxc=5000, pt=64, ws=FAKE, wsb=need - 1) == 4
+    # E4M3 caches need scales
+    d8 = _desc(cache_dtype=B.PA_E4M3)
+    assert lib.pa_decode(FAKE, 0, 1, 2, FAKE, FAKE, ctypes.byref(d8), FAKE, 4, FAKE, 64, 0.1,
+                         FAKE, 0, None, 0, None) == 1
+
+
+def test_append_argument_checks(lib):
+    d = _desc()
+    assert lib.pa_append_kv(FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, ctypes.byref(d), None) == 2
+    assert lib.pa_append_kv(FAKE, FAKE, 2, 4, FAKE, FAKE, FAKE, ctypes.byref(d), None) == 1
+    assert lib.pa_append_kv(FAKE, FAKE, 0, -1, FAKE, FAKE, FAKE, ctypes.byref(d), None) == 1
+    assert lib.pa_append_kv(None, None, 0, 0, None, None, None, ctypes.byref(d), None) == 0
+    d8 = _desc(cache_dtype=B.PA_E4M3)
+    assert lib.pa_append_kv(FAKE, FAKE, 0, 4, FAKE, FAKE, FAKE, ctypes.byref(d8), None) == 1
+
+
+def test_workspace_plan(lib):
+    d = _desc(num_kv_heads=8, head_dim=128)
+    # one partition covers the context: no workspace
+    assert lib.pa_decode_workspace_size(4, 64, 100, 512, ctypes.byref(d)) == 0
+    # split: partial outputs (fp32, head_dim) + (max, sum) per partition, 256-byte sections
+    ws = lib.pa_decode_workspace_size(4, 64, 131072, 512, ctypes.byref(d))
+    parts = 131072 // 512
+    o = 4 * 64 * parts * 128 * 4
+    ml = 4 * 64 * parts * 8
+    assert ws == -(-o // 256) * 256 + -(-ml // 256) * 256
+    # automatic partition: halves from 512 while the grid is under two CTAs per SM
+    assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(_desc(num_kv_heads=32))) == 512
+    assert lib.pa_decode_partition_tokens(1, 4096, ctypes.byref(d)) == 64
+    assert lib.pa_decode_partition_tokens(1, 100, ctypes.byref(d)) == 64

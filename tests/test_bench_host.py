@@ -1,0 +1,70 @@
+"""Host-side logic of bench.py on the CPU: the multi-rank reductions over a
+2-rank gloo group, per-rank workloads, and the reference (CPU oracle) arm."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = bench.make_workload("tiny_mha", rank, None)
+        got_max = bench.max_over_ranks(10.0 + rank)
+        got_sum = bench.sum_over_ranks(float(w.batch))
+        q.put((rank, got_max, got_sum, int(w.context_lens.sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_reductions_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [11.0, 11.0]     # max over ranks, seen by every rank
+    assert [r[2] for r in res] == [8.0, 8.0]       # 4 sequences per rank
+    assert res[0][3] != res[1][3]                  # ranks draw different batches
+
+
+def test_rank_seed_offsets_are_distinct():
+    a = bench.make_workload("llama2_7b", 0, 2)
+    b = bench.make_workload("llama2_7b", 1, 2)
+    assert not np.array_equal(a.context_lens, b.context_lens)
+
+
+def test_reference_arm_prints_one_json_line():
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_mha", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, PYTHONPATH=ROOT, RANK="1", WORLD_SIZE="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_mha", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
