@@ -5,11 +5,13 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
+#include <array>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <type_traits>
+#include <mutex>
+#include <unordered_map>
 #include <unordered_set>
 
 #include "pa_api.h"
@@ -86,17 +88,21 @@ Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int part
   return pl;
 }
 
-// cudaFuncSetAttribute once per (kernel, device).
-template <typename K>
-cudaError_t ensure_smem(K kernel, int bytes) {
-  static std::atomic<uint64_t> done_mask{0};
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device),
+// raised to the largest size requested so far.
+cudaError_t ensure_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, std::array<int, 64>> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find(kernel);
+  if (it == done.end()) it = done.emplace(kernel, std::array<int, 64>{}).first;
+  int& have = it->second[dev & 63];
+  if (have >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  if (e == cudaSuccess) have = bytes;
   return e;
 }
 
@@ -104,10 +110,11 @@ template <typename TQ, int CK, int D, bool TWO>
 pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, TWO>;
-  const int bt_entries = (p.partition_tokens >> p.bs_log2) + 2;
+  const int bt_entries =
+      std::min((p.partition_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
   const int smem = S::kMainBytes + bt_entries * 4;
   if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
-  if (ensure_smem(kern, smem) != cudaSuccess) return PA_ERR_CUDA;
+  if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
   dim3 grid(p.num_partitions, p.num_kv_heads * p.head_groups, p.batch);
   kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;

@@ -57,6 +57,10 @@ struct DecodeParams {
 
 enum CacheKind { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
 
+// Block ids of one partition staged in shared memory (longer slices are read
+// from global memory row by row).
+constexpr int kBlockIdsInSmem = 1024;
+
 template <int CK, int D>
 struct TileGeom {
   static constexpr int ES = (CK == kE4M3) ? 1 : 2;  // bytes per cache element
@@ -138,15 +142,21 @@ __global__ void __launch_bounds__(NW * 32)
   const int ntiles = (t1 - t0 + 15) >> 4;
 
   // ---- block ids of this partition -> shared memory ----------------------
+  // (up to kBlockIdsInSmem of them; a longer slice is read from global
+  // memory per row instead)
   const int bt0 = t0 >> p.bs_log2;
   const int nbt = ((t1 - 1) >> p.bs_log2) - bt0 + 1;
-  for (int i = threadIdx.x; i < nbt; i += NW * 32) {
-    int id = p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq + bt0 + i];
-    if (id < 0 || id >= p.num_blocks) {
-      flag_error(PA_DEVERR_BLOCK_ID);
-      id = -1;
+  const bool bt_in_smem = nbt <= kBlockIdsInSmem;
+  const int32_t* gbt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + bt0;
+  if (bt_in_smem) {
+    for (int i = threadIdx.x; i < nbt; i += NW * 32) {
+      int id = gbt[i];
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PA_DEVERR_BLOCK_ID);
+        id = -1;
+      }
+      s_bt[i] = id;
     }
-    s_bt[i] = id;
   }
 
   // ---- query fragments (A operand, rows = query heads) -------------------
@@ -222,7 +232,18 @@ __global__ void __launch_bounds__(NW * 32)
       const int ch = c % G::CPR;
       const int j = tb + r;
       int blk = -1;
-      if (j < t1) blk = s_bt[(j >> p.bs_log2) - bt0];
+      if (j < t1) {
+        const int bi = (j >> p.bs_log2) - bt0;
+        if (bt_in_smem) {
+          blk = s_bt[bi];
+        } else {
+          blk = __ldg(gbt + bi);
+          if (blk < 0 || blk >= p.num_blocks) {
+            flag_error(PA_DEVERR_BLOCK_ID);
+            blk = -1;
+          }
+        }
+      }
       const bool ok = blk >= 0;
       const int64_t off = ok ? ((static_cast<int64_t>(blk) << p.bs_log2) + (j & bs_mask)) *
                                        slot_stride +
