@@ -154,6 +154,35 @@ pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_c
  * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure. */
 pa_status pa_get_device_error(void* stream, uint32_t* flags);
 
+/* pa_decode without a caller-supplied workspace and without allocating any.
+ * (The pages have no counterpart: this is an integration convenience.)
+ *
+ * For callers that cannot call cudaMalloc or take memory from an allocator
+ * on this path -- for example a plug-in inside an engine that owns all device
+ * memory through its own pool, or code on a latency-critical path where an
+ * allocation's implicit synchronisation is not acceptable. The split-K
+ * workspace is a fixed 32 MiB array in the library's own device memory
+ * (reserved on every GPU that loads the library, until the process exits),
+ * so the call allocates nothing; inputs and outputs are still the caller's.
+ * Arguments and results are those of pa_decode (same partition choice), minus
+ * the workspace. If the plan needs more than 32 MiB of workspace
+ * (pa_decode_workspace_size(...) > 32 MiB) the call returns
+ * PA_ERR_WORKSPACE and enqueues nothing; use pa_decode with a larger buffer
+ * or a longer partition.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) while that device is current; make that first call
+ * before any stream capture. Every call on a device shares the one array,
+ * which keeps the previous call's contents (nothing in it needs a starting
+ * value); calls whose kernels overlap on the GPU -- concurrent streams, or
+ * several host threads -- race on it and must be serialised by the caller. */
+pa_status pa_decode_static_workspace(const void* q, int32_t q_dtype, int32_t batch,
+                                     int32_t num_q_heads, const void* k_cache,
+                                     const void* v_cache, const pa_cache_desc* cache,
+                                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t* context_lens, int32_t max_context,
+                                     float scale, void* out, int32_t partition_tokens,
+                                     void* stream);
+
 /* Static text for a status code. */
 const char* pa_status_string(int32_t status);
 

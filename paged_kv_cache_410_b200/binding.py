@@ -27,7 +27,7 @@ DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT = 0x1, 0x2, 0x4
 # names of every symbol include/pa_api.h declares
 EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tokens",
             "pa_decode", "pa_copy_blocks", "pa_get_device_error", "pa_status_string",
-            "pa_version"]
+            "pa_version", "pa_decode_static_workspace"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -75,6 +75,9 @@ def load_library(path: str = LIB_PATH):
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
     lib.pa_version.restype = i32
+    lib.pa_decode_static_workspace.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32,
+                                               ctypes.c_float, P, i32, P]
+    lib.pa_decode_static_workspace.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -167,6 +170,24 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache
                        _ptr(context_lens), int(max_context), float(scale), _ptr(out),
                        int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                               cache: PagedCache, max_context: int, partition_tokens: int = 0,
+                               stream=None):
+    """pa_decode for callers that cannot allocate device memory: the split-K
+    workspace is the library's own fixed 32 MiB array (see include/pa_api.h
+    for the limit, the first-call set-up and the rule that overlapping calls
+    race on the shared array)."""
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    rc = lib.pa_decode_static_workspace(_ptr(q), _dtype_code(q.dtype), batch, hq,
+                                        _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+                                        _ptr(block_tables), block_tables.shape[1],
+                                        _ptr(context_lens), int(max_context), float(scale),
+                                        _ptr(out), int(partition_tokens), _stream(stream))
+    _check(rc, "pa_decode_static_workspace")
 
 
 def pa_copy_blocks(pairs, k_cache, v_cache, cache: PagedCache, stream=None):

@@ -335,3 +335,60 @@ pa_status pa_get_device_error(void* stream, uint32_t* flags) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation, for callers that cannot call
+// cudaMalloc: the split-K workspace lives in a fixed array in the library's
+// own device memory instead of a caller-provided buffer.
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;  // 32 MiB per device
+
+// Reserved in every device context that loads this library, until exit.
+static __device__ __align__(256) unsigned char g_pa_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_pa_static_workspace on the current device. In host code
+// the array's name is only a host-side handle, so the address is looked up
+// once per device with cudaGetSymbolAddress (the first call on each device).
+pa_status static_workspace_address(void** out) {
+  static std::mutex mu;
+  static std::array<void*, 64> addr{};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_pa_static_workspace) != cudaSuccess || !p) return PA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_static_workspace(
+    const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads, const void* k_cache,
+    const void* v_cache, const pa_cache_desc* cache, const int32_t* block_tables,
+    int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context, float scale,
+    void* out, int32_t partition_tokens, void* stream) {
+  int bs_log2 = 0;
+  pa_status st = check_cache(cache, &bs_log2);
+  if (st != PA_OK) return st;
+  if (batch < 0 || num_q_heads <= 0 || max_context < 0 || partition_tokens < 0)
+    return PA_ERR_INVALID_ARG;
+  const size_t need =
+      batch > 0 ? pa_decode_workspace_size(batch, num_q_heads, max_context, partition_tokens, cache)
+                : 0;
+  if (need > kStaticWorkspaceBytes) return PA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    st = static_workspace_address(&ws);
+    if (st != PA_OK) return st;
+  }
+  // The split-K partials need no initial value: every partial the reduce
+  // kernel reads is written earlier in the same call.
+  return pa_decode(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache, block_tables,
+                   max_blocks_per_seq, context_lens, max_context, scale, out, partition_tokens,
+                   ws, need > 0 ? kStaticWorkspaceBytes : 0, stream);
+}
