@@ -21,10 +21,18 @@
 
 namespace {
 
+// Build-time tuning of the decode CTA (warps, and cp.async stages per warp).
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+
 constexpr int kNumSMs = 148;         // B200
-constexpr int kDecodeWarps = 4;      // warps per decode CTA
-constexpr int kDecodeStages = 3;     // cp.async stages per warp
-constexpr int kDefaultPartition = 512;
+constexpr int kDecodeWarps = PA_DECODE_WARPS;
+constexpr int kDecodeStages = PA_DECODE_STAGES;
+constexpr int kPartitionRowBytes = 128 * 1024;  // K bytes of one KV head per partition
 constexpr int kMinAutoPartition = 64;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -51,11 +59,13 @@ pa_status check_cache(const pa_cache_desc* cd, int* bs_log2) {
 
 int64_t elem_bytes(int dtype) { return dtype == PA_E4M3 ? 1 : 2; }
 
-// Partition length used when the caller passes 0: 512 tokens, halved (down
-// to 64) while the launch would have fewer than two CTAs per SM.
-int auto_partition(int64_t batch, int64_t max_context, int64_t num_kv_heads) {
-  int pt = kDefaultPartition;
-  auto ctas = [&](int p) { return batch * num_kv_heads * ((max_context + p - 1) / p); };
+// Partition length used when the caller passes 0: the tokens whose K rows of
+// one KV head take 128 KB (512 at fp16/bf16 and head_dim 128, 1024 for E4M3
+// or head_dim 64), halved (down to 64) while the launch would have fewer
+// than two CTAs per SM.
+int auto_partition(int64_t batch, int64_t max_context, const pa_cache_desc* cd) {
+  int pt = kPartitionRowBytes / static_cast<int>(cd->head_dim * elem_bytes(cd->cache_dtype));
+  auto ctas = [&](int p) { return batch * cd->num_kv_heads * ((max_context + p - 1) / p); };
   while (pt > kMinAutoPartition && ctas(pt) < 2 * kNumSMs) pt >>= 1;
   return pt;
 }
@@ -74,7 +84,7 @@ Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int part
   Plan pl{};
   pl.partition_tokens = partition_tokens > 0
                             ? partition_tokens
-                            : auto_partition(batch, max_context, cd->num_kv_heads);
+                            : auto_partition(batch, max_context, cd);
   const int64_t np = (max_context + pl.partition_tokens - 1) / pl.partition_tokens;
   pl.num_partitions = static_cast<int>(std::max<int64_t>(np, 1));
   if (pl.num_partitions > 1) {
@@ -106,10 +116,10 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
   return e;
 }
 
-template <typename TQ, int CK, int D, bool TWO>
+template <typename TQ, int CK, int D, int NH>
 pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
-  auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, TWO>;
+  auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH>;
   const int bt_entries =
       std::min((p.partition_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
   const int smem = S::kMainBytes + bt_entries * 4;
@@ -119,7 +129,8 @@ pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
   kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (p.num_partitions > 1) {
-    pa::pa_decode_reduce_kernel<TQ, D><<<dim3(p.num_q_heads, p.batch), 128, 0, st>>>(p);
+    pa::pa_decode_reduce_kernel<TQ, D>
+        <<<dim3(p.num_q_heads, p.batch), pa::kReduceWarps * 32, 0, st>>>(p);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
@@ -127,11 +138,11 @@ pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
 
 template <typename TQ, int CK>
 pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, cudaStream_t st) {
+  // query heads per CTA: the whole group up to 16; 8-head column blocks
   const bool two = std::min(p.group, 16) > 8;
   if (head_dim == 64)
-    return two ? launch_decode_t<TQ, CK, 64, true>(p, st) : launch_decode_t<TQ, CK, 64, false>(p, st);
-  return two ? launch_decode_t<TQ, CK, 128, true>(p, st)
-             : launch_decode_t<TQ, CK, 128, false>(p, st);
+    return two ? launch_decode_t<TQ, CK, 64, 2>(p, st) : launch_decode_t<TQ, CK, 64, 1>(p, st);
+  return two ? launch_decode_t<TQ, CK, 128, 2>(p, st) : launch_decode_t<TQ, CK, 128, 1>(p, st);
 }
 
 }  // namespace
@@ -205,7 +216,7 @@ int32_t pa_decode_partition_tokens(int32_t batch, int32_t max_context,
                                    const pa_cache_desc* cache) {
   int bs_log2 = 0;
   if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || max_context < 0) return 0;
-  return auto_partition(batch, max_context, cache->num_kv_heads);
+  return auto_partition(batch, max_context, cache);
 }
 
 pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,

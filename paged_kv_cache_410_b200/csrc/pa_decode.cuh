@@ -17,13 +17,19 @@
 // that spans one partition writes its output directly, longer ones write
 // (max, sum, normalised output) partials that the reduce kernel combines.
 //
-// Tensor cores. Rows of the m16n8k16 MMA are the group's query heads (up to
-// 16; padding rows are zero), columns are 8 tokens: S = Q K^T with K tiles
-// loaded by ldmatrix, then O += P V with P taken straight from the S
-// accumulators and V tiles loaded by ldmatrix.trans. For an E4M3 cache the
-// codes are widened to f16 (exactly) in registers; the K scale is folded into
-// the query (as an f16 hi + lo pair so the fold costs no precision) and the V
-// scale is applied to the merged output.
+// Tensor cores, transposed products. With 16 tokens per tile and up to 8
+// query heads per MMA column block:
+//   S^T (16 tokens x 8 heads) = K_tile (16 x D) . Q^T (D x 8)   [m16n8k16]
+//   O^T (D x 8 heads)        += V_tile^T (D x 16) . P^T (16 x 8)
+// K tiles feed the A operand through ldmatrix, V tiles through
+// ldmatrix.trans; Q^T stays in registers as the B operand for the whole
+// partition; P^T is the S^T accumulator after the softmax, converted to
+// 16 bits and transposed in registers with movmatrix. Rows of every MMA are
+// tokens or channels, so no accumulator row is padding; groups of 9..16
+// query heads use two column blocks. For an E4M3 cache the codes are widened
+// to f16 (exactly) in registers; the K scale is folded into the query (as an
+// f16 hi + lo pair, so the fold costs no precision) and the V scale is
+// applied to the merged output.
 #pragma once
 
 #include "pa_common.cuh"
@@ -93,21 +99,25 @@ struct DecodeSmem {
   // + block-table slice of the partition (int32), sized at launch
 };
 
-template <typename TQ, int CK, int D, int NW, int NSTAGE, bool TWO_ROWS>
+// NH: 8-head column blocks per CTA (1 for groups of up to 8 query heads, 2
+// for 9..16).
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH>
 __global__ void __launch_bounds__(NW * 32)
     pa_decode_kernel(const DecodeParams p) {
   using G = TileGeom<CK, D>;
   using S = DecodeSmem<CK, D, NW, NSTAGE>;
   constexpr bool kMmaBF16 = (CK == kBF16);  // MMA operand type (E4M3 widens to f16)
-  constexpr int KSTEPS = D / 16;
-  constexpr int NT = D / 8;  // n-tiles of the P.V product
+  constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T
+  constexpr int MT = D / 16;                // 16-channel row blocks of O^T
+  constexpr int RPI = 32 / G::CPR;          // tile rows one load instruction covers
+  constexpr int LITERS = 16 / RPI;          // load instructions per lane per tile and tensor
 
   extern __shared__ __align__(128) uint8_t smem[];
   int* s_bt = reinterpret_cast<int*>(smem + S::kMainBytes);
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int g = lane >> 2;  // MMA group id: query-head row / token column
+  const int g = lane >> 2;  // MMA group id
   const int t = lane & 3;   // thread in group
 
   const int b = blockIdx.z;
@@ -115,7 +125,7 @@ __global__ void __launch_bounds__(NW * 32)
   const int hgrp = blockIdx.y - hk * p.head_groups;
   const int part = blockIdx.x;
   const int row0 = hgrp * 16;
-  const int nrows = min(16, p.group - row0);
+  const int nrows = min(16, p.group - row0);  // query heads of this CTA
   const int hq0 = hk * p.group + row0;
 
   // ---- sequence length, checked against what the launch covers ----------
@@ -159,53 +169,48 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
 
-  // ---- query fragments (A operand, rows = query heads) -------------------
+  // ---- Q^T fragments (B operand: k = channel, n = query head) -------------
+  // qb[kk][nh] = {channels of slots 2t,2t+1 ; slots 2t+8,2t+9} of head
+  // 8*nh + g.
   const TQ* qbase = reinterpret_cast<const TQ*>(p.q) +
                     (static_cast<int64_t>(b) * p.num_q_heads + hq0) * D;
-  const bool rlo = g < nrows;
-  const bool rhi = TWO_ROWS && (g + 8 < nrows);
-  uint32_t qa[KSTEPS][4];
-  uint32_t qlo[CK == kE4M3 ? KSTEPS : 1][4];
-  if constexpr (CK != kE4M3) {
+  uint32_t qb[KSTEPS][NH][2];
+  uint32_t qlo[CK == kE4M3 ? KSTEPS : 1][NH][2];
 #pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      const int c0 = kk * 16 + 2 * t;
-      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qbase + g * D);
-      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qbase + (g + 8) * D);
-      qa[kk][0] = rlo ? r0[c0 / 2] : 0u;
-      qa[kk][1] = rhi ? r1[c0 / 2] : 0u;
-      qa[kk][2] = rlo ? r0[(c0 + 8) / 2] : 0u;
-      qa[kk][3] = rhi ? r1[(c0 + 8) / 2] : 0u;
-    }
-  } else {
-    // E4M3: q' = q * k_scale[hk][:], split into f16 hi + lo. K-slot mapping
-    // per 32-channel group gq: k-step 2gq holds channels 8t+{0,1} (slots
-    // 2t,2t+1) and 8t+{2,3} (slots 2t+8,2t+9); k-step 2gq+1 holds 8t+{4,5}
-    // and 8t+{6,7}. The K fragments below use the same mapping.
-    const float* ks = p.k_scale + static_cast<int64_t>(hk) * D;
+  for (int nh = 0; nh < NH; ++nh) {
+    const int hrow = 8 * nh + g;
+    const bool ok = hrow < nrows;
+    const TQ* qr = qbase + hrow * D;
+    if constexpr (CK != kE4M3) {
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qr);
 #pragma unroll
-    for (int gq = 0; gq < D / 32; ++gq) {
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        qb[kk][nh][0] = ok ? q32[(kk * 16 + 2 * t) / 2] : 0u;
+        qb[kk][nh][1] = ok ? q32[(kk * 16 + 8 + 2 * t) / 2] : 0u;
+      }
+    } else {
+      // q' = q * k_scale[hk][:], as f16 hi + lo. Channel order inside each
+      // 32-channel group gq (shared with the K fragments below): k-step
+      // 2gq + h holds channels 8t + 4h + {0,1} in slots 2t, 2t+1 and
+      // 8t + 4h + {2,3} in slots 2t+8, 2t+9.
+      const float* ks = p.k_scale + static_cast<int64_t>(hk) * D;
 #pragma unroll
-      for (int half_ = 0; half_ < 2; ++half_) {
-        const int kk = 2 * gq + half_;
-        const int cA = gq * 32 + 8 * t + 4 * half_;  // channels cA, cA+1 | cA+2, cA+3
+      for (int gq = 0; gq < D / 32; ++gq) {
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const bool ok = rr == 0 ? rlo : rhi;
-          const TQ* qr = qbase + (g + 8 * rr) * D;
-          float x[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) x[e] = ok ? to_f32<TQ>(qr[cA + e]) * ks[cA + e] : 0.f;
-          float h[4], l[4];
+        for (int h = 0; h < 2; ++h) {
+          const int kk = 2 * gq + h;
+          const int c = gq * 32 + 8 * t + 4 * h;
+          float x[4], hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            h[e] = __half2float(__float2half_rn(x[e]));
-            l[e] = x[e] - h[e];
+            x[e] = ok ? to_f32<TQ>(qr[c + e]) * ks[c + e] : 0.f;
+            hi[e] = __half2float(__float2half_rn(x[e]));
+            lo[e] = x[e] - hi[e];
           }
-          qa[kk][rr] = pack2<false>(h[0], h[1]);
-          qa[kk][2 + rr] = pack2<false>(h[2], h[3]);
-          qlo[kk][rr] = pack2<false>(l[0], l[1]);
-          qlo[kk][2 + rr] = pack2<false>(l[2], l[3]);
+          qb[kk][nh][0] = pack2<false>(hi[0], hi[1]);
+          qb[kk][nh][1] = pack2<false>(hi[2], hi[3]);
+          qlo[kk][nh][0] = pack2<false>(lo[0], lo[1]);
+          qlo[kk][nh][1] = pack2<false>(lo[2], lo[3]);
         }
       }
     }
@@ -216,50 +221,71 @@ __global__ void __launch_bounds__(NW * 32)
   uint8_t* wbuf = smem + warp * NSTAGE * S::kStageBytes;
   const uint8_t* kc = reinterpret_cast<const uint8_t*>(p.k_cache);
   const uint8_t* vc = reinterpret_cast<const uint8_t*>(p.v_cache);
-  const int64_t head_off = static_cast<int64_t>(hk) * G::RB;
   const int64_t slot_stride = static_cast<int64_t>(p.num_kv_heads) * G::RB;
   const int bs_mask = (1 << p.bs_log2) - 1;
+  const bool block_aligned = p.bs_log2 >= 4;  // a 16-token tile lies inside one block
+  // this lane's load slots: rows lrow + i*RPI, 16-byte chunk lch
+  const int lrow = lane / G::CPR;
+  const int lch = lane % G::CPR;
+  const int64_t lane_goff = static_cast<int64_t>(hk) * G::RB + lch * 16;
+
+  auto block_id = [&](int bi) -> int {
+    if (bt_in_smem) return s_bt[bi];
+    int id = __ldg(gbt + bi);
+    if (id < 0 || id >= p.num_blocks) {
+      flag_error(PA_DEVERR_BLOCK_ID);
+      id = -1;
+    }
+    return id;
+  };
 
   auto load_tile = [&](int tile, int stage) {
-    uint8_t* sk = wbuf + stage * S::kStageBytes;
-    const uint32_t sk_a = smem_addr(sk);
+    const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
     const int tb = t0 + tile * 16;
+    if (block_aligned) {
+      const int blk = block_id((tb >> p.bs_log2) - bt0);
+      const int64_t base =
+          ((static_cast<int64_t>(blk) << p.bs_log2) + (tb & bs_mask) + lrow) * slot_stride +
+          lane_goff;
 #pragma unroll
-    for (int i = 0; i < G::CPR / 2; ++i) {
-      const int c = lane + 32 * i;
-      const int r = c / G::CPR;
-      const int ch = c % G::CPR;
-      const int j = tb + r;
-      int blk = -1;
-      if (j < t1) {
-        const int bi = (j >> p.bs_log2) - bt0;
-        if (bt_in_smem) {
-          blk = s_bt[bi];
-        } else {
-          blk = __ldg(gbt + bi);
-          if (blk < 0 || blk >= p.num_blocks) {
-            flag_error(PA_DEVERR_BLOCK_ID);
-            blk = -1;
-          }
-        }
+      for (int i = 0; i < LITERS; ++i) {
+        const int r = lrow + i * RPI;
+        const bool ok = blk >= 0 && tb + r < t1;
+        const int64_t off = ok ? base + static_cast<int64_t>(i * RPI) * slot_stride : 0;
+        const uint32_t so = G::off(r, lch);
+        cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
+        cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
       }
-      const bool ok = blk >= 0;
-      const int64_t off = ok ? ((static_cast<int64_t>(blk) << p.bs_log2) + (j & bs_mask)) *
-                                       slot_stride +
-                                   head_off + ch * 16
-                             : 0;
-      const uint32_t so = G::off(r, ch);
-      cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
-      cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
+    } else {
+#pragma unroll
+      for (int i = 0; i < LITERS; ++i) {
+        const int r = lrow + i * RPI;
+        const int j = tb + r;
+        const int blk = j < t1 ? block_id((j >> p.bs_log2) - bt0) : -1;
+        const bool ok = blk >= 0;
+        const int64_t off =
+            ok ? ((static_cast<int64_t>(blk) << p.bs_log2) + (j & bs_mask)) * slot_stride +
+                     lane_goff
+               : 0;
+        const uint32_t so = G::off(r, lch);
+        cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
+        cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
+      }
     }
   };
 
-  float o[NT][4];
+  float o[MT][NH][4];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
+  float m_run[NH][2], l_run[NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    m_run[nh][0] = m_run[nh][1] = -INFINITY;
+    l_run[nh][0] = l_run[nh][1] = 0.f;
+  }
 
   const int my_tiles = warp < ntiles ? (ntiles - warp + NW - 1) / NW : 0;
 #pragma unroll
@@ -283,92 +309,109 @@ __global__ void __launch_bounds__(NW * 32)
     const int tile = warp + it * NW;
     const int nvalid = t1 - (t0 + tile * 16);  // tokens of this tile that exist (>= 1)
 
-    // S = Q K^T for 16 tokens: s[nt] covers tokens 8nt .. 8nt+7
-    float s[2][4];
+    // S^T = K Q^T: s[nh] = {(token g, heads 2t, 2t+1), (token g+8, heads 2t, 2t+1)}
+    float s[NH][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
     if constexpr (CK != kE4M3) {
-      const int lr = (lane & 7) + ((lane >> 4) << 3);
-      const int lc = (lane >> 3) & 1;
+      const int mi = lane >> 3;
+      const int tok = (lane & 7) + 8 * (mi & 1);
+      const int chk = mi >> 1;
 #pragma unroll
       for (int kk = 0; kk < KSTEPS; ++kk) {
-        uint32_t k0, k1, k2, k3;
-        ldmatrix_x4(k0, k1, k2, k3, sk_a + G::off(lr, 2 * kk + lc));
-        mma_16816<kMmaBF16>(s[0], qa[kk], k0, k1);
-        mma_16816<kMmaBF16>(s[1], qa[kk], k2, k3);
+        uint32_t a[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(tok, 2 * kk + chk));
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(s[nh], a, qb[kk][nh][0], qb[kk][nh][1]);
       }
     } else {
 #pragma unroll
       for (int gq = 0; gq < D / 32; ++gq) {
+        const int c = 2 * gq + (t >> 1);
+        const int bo = (t & 1) * 8;
+        const uint2 wl = lds64(sk_a + G::off(g, c) + bo);      // token g
+        const uint2 wh = lds64(sk_a + G::off(g + 8, c) + bo);  // token g + 8
+        uint32_t a0[4], a1[4];
+        e4m3x4_to_f16x2x2(wl.x, a0[0], a0[2]);
+        e4m3x4_to_f16x2x2(wh.x, a0[1], a0[3]);
+        e4m3x4_to_f16x2x2(wl.y, a1[0], a1[2]);
+        e4m3x4_to_f16x2x2(wh.y, a1[1], a1[3]);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int r = g + 8 * nt;
-          const uint2 w = lds64(sk_a + G::off(r, 2 * gq + (t >> 1)) + (t & 1) * 8);
-          uint32_t a0, a1, b0, b1;
-          e4m3x4_to_f16x2x2(w.x, a0, a1);
-          e4m3x4_to_f16x2x2(w.y, b0, b1);
-          mma_16816<false>(s[nt], qa[2 * gq], a0, a1);
-          mma_16816<false>(s[nt], qlo[2 * gq], a0, a1);
-          mma_16816<false>(s[nt], qa[2 * gq + 1], b0, b1);
-          mma_16816<false>(s[nt], qlo[2 * gq + 1], b0, b1);
+        for (int nh = 0; nh < NH; ++nh) {
+          mma_16816<false>(s[nh], a0, qb[2 * gq][nh][0], qb[2 * gq][nh][1]);
+          mma_16816<false>(s[nh], a0, qlo[2 * gq][nh][0], qlo[2 * gq][nh][1]);
+          mma_16816<false>(s[nh], a1, qb[2 * gq + 1][nh][0], qb[2 * gq + 1][nh][1]);
+          mma_16816<false>(s[nh], a1, qlo[2 * gq + 1][nh][0], qlo[2 * gq + 1][nh][1]);
         }
       }
     }
 
-    // online softmax over the tile (log2 domain); row halves rr: g, g + 8
-    uint32_t pa[4];
+    // online softmax per query head (column), log2 domain; the max is
+    // reduced over the 16 tokens (lanes with the same t, both row halves)
+    const bool va = g < nvalid;
+    const bool vb = g + 8 < nvalid;
+    uint32_t pb[NH][2];
+    bool grew = false;
+    float alpha[NH][2];
 #pragma unroll
-    for (int rr = 0; rr < (TWO_ROWS ? 2 : 1); ++rr) {
-      float x[4];
+    for (int nh = 0; nh < NH; ++nh) {
+      float pr[2][2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = (e >> 1) * 8 + 2 * t + (e & 1);
-        const float v = s[e >> 1][2 * rr + (e & 1)] * p.scale_log2;
-        x[e] = tok < nvalid ? v : -INFINITY;
+      for (int e = 0; e < 2; ++e) {
+        const float x0 = va ? s[nh][e] * p.scale_log2 : -INFINITY;
+        const float x1 = vb ? s[nh][2 + e] * p.scale_log2 : -INFINITY;
+        float mx = fmaxf(x0, x1);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m_run[nh][e], mx);  // finite: token 0 of the tile exists
+        const bool up = m_new > m_run[nh][e];
+        grew |= up;
+        alpha[nh][e] = up ? ex2(m_run[nh][e] - m_new) : 1.f;  // exactly 1 when unchanged
+        pr[0][e] = ex2(x0 - m_new);
+        pr[1][e] = ex2(x1 - m_new);
+        l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + (pr[0][e] + pr[1][e]);
+        m_run[nh][e] = m_new;
       }
-      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_run[rr], mx);  // finite: token 0 of the tile exists
-      const float alpha = ex2(m_run[rr] - m_new);
-      float pe[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pe[e] = ex2(x[e] - m_new);
-      l_run[rr] = l_run[rr] * alpha + (pe[0] + pe[1]) + (pe[2] + pe[3]);
-      m_run[rr] = m_new;
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        o[i][2 * rr] *= alpha;
-        o[i][2 * rr + 1] *= alpha;
-      }
-      pa[rr] = pack2<kMmaBF16>(pe[0], pe[1]);      // tokens 2t, 2t+1
-      pa[2 + rr] = pack2<kMmaBF16>(pe[2], pe[3]);  // tokens 8+2t, 9+2t
+      // (token, head) 8x8 blocks -> transposed: head g, tokens 2t,2t+1 | 2t+8,2t+9
+      pb[nh][0] = movmatrix_trans(pack2<kMmaBF16>(pr[0][0], pr[0][1]));
+      pb[nh][1] = movmatrix_trans(pack2<kMmaBF16>(pr[1][0], pr[1][1]));
     }
-    if constexpr (!TWO_ROWS) {
-      pa[1] = 0u;
-      pa[3] = 0u;
+    if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) {
+          o[mt][nh][0] *= alpha[nh][0];
+          o[mt][nh][1] *= alpha[nh][1];
+          o[mt][nh][2] *= alpha[nh][0];
+          o[mt][nh][3] *= alpha[nh][1];
+        }
     }
 
-    // O += P V
+    // O^T += V^T P^T
     if constexpr (CK != kE4M3) {
-      const int lr = (lane & 7) + (((lane >> 3) & 1) << 3);
-      const int lc = lane >> 4;
+      const int mi = lane >> 3;
+      const int tok = (lane & 7) + 8 * (mi >> 1);
+      const int chk = mi & 1;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t v0, v1, v2, v3;
-        ldmatrix_x4_trans(v0, v1, v2, v3, sv_a + G::off(lr, 2 * c + lc));
-        mma_16816<kMmaBF16>(o[2 * c], pa, v0, v1);
-        mma_16816<kMmaBF16>(o[2 * c + 1], pa, v2, v3);
+      for (int mt = 0; mt < MT; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], sv_a + G::off(tok, 2 * mt + chk));
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(o[mt][nh], a, pb[nh][0], pb[nh][1]);
       }
     } else {
-      // n-tile i, column n <-> channel NT*n + i: this thread (column g) owns
-      // channels [NT*g, NT*g + NT) of token rows 2t, 2t+1, 2t+8, 2t+9.
-      constexpr int WORDS = NT / 4;
+      // Row m of O^T block mt is channel DPT*g + 2*mt (m = g) or that + 1
+      // (m = g + 8): this thread reads channels [DPT*g, DPT*g + DPT) of token
+      // rows 2t, 2t+1, 2t+8, 2t+9 and pairs tokens with byte permutes.
+      constexpr int DPT = D / 8;
+      constexpr int WORDS = DPT / 4;
       uint32_t ra[4][WORDS];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int r = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
-        const int byte0 = NT * g;
+        const int byte0 = DPT * g;
         const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
         if constexpr (WORDS == 4) {
           const uint4 w = lds128(addr);
@@ -384,19 +427,18 @@ __global__ void __launch_bounds__(NW * 32)
       }
 #pragma unroll
       for (int w = 0; w < WORDS; ++w) {
-        uint32_t lo01, hi01, lo89, hi89, f0, f1, f2, f3, e0, e1, e2, e3;
-        lo01 = __byte_perm(ra[0][w], ra[1][w], 0x5140);
-        hi01 = __byte_perm(ra[0][w], ra[1][w], 0x7362);
-        lo89 = __byte_perm(ra[2][w], ra[3][w], 0x5140);
-        hi89 = __byte_perm(ra[2][w], ra[3][w], 0x7362);
-        e4m3x4_to_f16x2x2(lo01, f0, f1);
-        e4m3x4_to_f16x2x2(hi01, f2, f3);
-        e4m3x4_to_f16x2x2(lo89, e0, e1);
-        e4m3x4_to_f16x2x2(hi89, e2, e3);
-        mma_16816<false>(o[4 * w + 0], pa, f0, e0);
-        mma_16816<false>(o[4 * w + 1], pa, f1, e1);
-        mma_16816<false>(o[4 * w + 2], pa, f2, e2);
-        mma_16816<false>(o[4 * w + 3], pa, f3, e3);
+        uint32_t f[4], e[4];
+        e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x5140), f[0], f[1]);
+        e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x7362), f[2], f[3]);
+        e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x5140), e[0], e[1]);
+        e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x7362), e[2], e[3]);
+        const uint32_t a0[4] = {f[0], f[1], e[0], e[1]};  // channel block 2w
+        const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) {
+          mma_16816<false>(o[2 * w][nh], a0, pb[nh][0], pb[nh][1]);
+          mma_16816<false>(o[2 * w + 1][nh], a1, pb[nh][0], pb[nh][1]);
+        }
       }
     }
     __syncwarp();  // this stage is reloaded by the next iteration
@@ -405,38 +447,43 @@ __global__ void __launch_bounds__(NW * 32)
 
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
-    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
-  }
+  for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      l_run[nh][e] += __shfl_xor_sync(0xffffffffu, l_run[nh][e], 4);
+      l_run[nh][e] += __shfl_xor_sync(0xffffffffu, l_run[nh][e], 8);
+      l_run[nh][e] += __shfl_xor_sync(0xffffffffu, l_run[nh][e], 16);
+    }
   __syncthreads();  // pipeline buffers are reused below
   float* w_o = reinterpret_cast<float*>(smem);  // [NW][16][D]
   float* w_m = w_o + NW * 16 * D;               // [NW][16]
   float* w_l = w_m + NW * 16;                   // [NW][16]
   float* r_w = w_l + NW * 16;                   // [NW][16] merge weights
-  float* r_stat = r_w + NW * 16;                // [16][2] merged max, 1/sum
+  float* r_stat = r_w + NW * 16;                // [16][2] merged max, sum
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int row = g + 8 * rr;
-    if (rr == 1 && !TWO_ROWS) break;
-    if (row < nrows) {
-      float* dst = w_o + (warp * 16 + row) * D;
+  for (int nh = 0; nh < NH; ++nh) {
 #pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        int c0, c1;
-        if constexpr (CK != kE4M3) {
-          c0 = 8 * i + 2 * t;
-          c1 = c0 + 1;
-        } else {
-          c0 = NT * (2 * t) + i;
-          c1 = NT * (2 * t + 1) + i;
+    for (int e = 0; e < 2; ++e) {
+      const int head = 8 * nh + 2 * t + e;
+      if (head < nrows) {
+        float* dst = w_o + (warp * 16 + head) * D;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          int c_lo, c_hi;
+          if constexpr (CK != kE4M3) {
+            c_lo = 16 * mt + g;
+            c_hi = c_lo + 8;
+          } else {
+            c_lo = (D / 8) * g + 2 * mt;
+            c_hi = c_lo + 1;
+          }
+          dst[c_lo] = o[mt][nh][e];
+          dst[c_hi] = o[mt][nh][2 + e];
         }
-        dst[c0] = o[i][2 * rr];
-        dst[c1] = o[i][2 * rr + 1];
-      }
-      if (t == 0) {
-        w_m[warp * 16 + row] = m_run[rr];
-        w_l[warp * 16 + row] = l_run[rr];
+        if (g == 0) {
+          w_m[warp * 16 + head] = m_run[nh][e];
+          w_l[warp * 16 + head] = l_run[nh][e];
+        }
       }
     }
   }
@@ -481,10 +528,22 @@ __global__ void __launch_bounds__(NW * 32)
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
 // and normalised output o_p, out = sum_p w_p o_p / sum_p w_p where
 // w_p = l_p * 2^(m_p - max_p m_p).
+//
+// One CTA of kReduceWarps warps per (sequence, query head): the weights are
+// computed once per partition into shared memory, then each warp sums a
+// strided subset of the partitions with float4 loads (lane l owns channels
+// 4l .. 4l+3) and the warps' sums are added in shared memory.
+constexpr int kReduceWarps = 8;
+constexpr int kReduceChunk = 1024;  // partitions weighted per pass
+
 template <typename TQ, int D>
-__global__ void __launch_bounds__(128) pa_decode_reduce_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p) {
+  static_assert(D % 4 == 0 && D <= 128, "one float4 per lane");
+  constexpr int NT = kReduceWarps * 32;
   const int hq = blockIdx.x;
   const int b = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   int L = p.context_lens[b];
   const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
   const int cap = static_cast<int>(table_cap < p.max_context ? table_cap : p.max_context);
@@ -493,44 +552,59 @@ __global__ void __launch_bounds__(128) pa_decode_reduce_kernel(const DecodeParam
   if (nparts <= 1) return;
   const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq;
   const float2* ml = p.ws_ml + bh * p.num_partitions;
-  const float* po = p.ws_o + bh * p.num_partitions * D;
+  const float4* po = reinterpret_cast<const float4*>(p.ws_o + bh * p.num_partitions * D);
 
-  __shared__ float s_w[256];
-  __shared__ float s_red[4];
+  __shared__ float s_w[kReduceChunk];
+  __shared__ float s_red[kReduceWarps];
+  __shared__ float4 s_acc[kReduceWarps][D / 4];
+  __shared__ float s_wsum[kReduceWarps];
+
   // max over partitions
   float M = -INFINITY;
-  for (int i = threadIdx.x; i < nparts; i += blockDim.x) M = fmaxf(M, ml[i].x);
+  for (int i = threadIdx.x; i < nparts; i += NT) M = fmaxf(M, ml[i].x);
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = M;
+  if (lane == 0) s_red[warp] = M;
   __syncthreads();
-  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-  __syncthreads();
+  M = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, s_red[w]);
 
-  float acc[(D + 127) / 128] = {};
+  const bool active = lane < D / 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  for (int base = 0; base < nparts; base += 256) {
-    const int n = min(256, nparts - base);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+  for (int base = 0; base < nparts; base += kReduceChunk) {
+    const int n = min(kReduceChunk, nparts - base);
+    __syncthreads();  // previous chunk's weights consumed
+    for (int i = threadIdx.x; i < n; i += NT) {
       const float2 v = ml[base + i];
       s_w[i] = v.y * ex2(v.x - M);
     }
     __syncthreads();
-    for (int i = 0; i < n; ++i) {
+#pragma unroll 8
+    for (int i = warp; i < n; i += kReduceWarps) {
       const float w = s_w[i];
       wsum += w;
-#pragma unroll
-      for (int k = 0; k < (D + 127) / 128; ++k) {
-        const int c = threadIdx.x + 128 * k;
-        if (c < D) acc[k] += w * po[static_cast<int64_t>(base + i) * D + c];
+      if (active) {
+        const float4 v = po[static_cast<int64_t>(base + i) * (D / 4) + lane];
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
       }
     }
-    __syncthreads();
   }
-  TQ* out = reinterpret_cast<TQ*>(p.out);
+  if (active) s_acc[warp][lane] = acc;
+  if (lane == 0) s_wsum[warp] = wsum;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float a = 0.f, ws = 0.f;
 #pragma unroll
-  for (int k = 0; k < (D + 127) / 128; ++k) {
-    const int c = threadIdx.x + 128 * k;
-    if (c < D) out[bh * D + c] = from_f32<TQ>(acc[k] / wsum);
+    for (int w = 0; w < kReduceWarps; ++w) {
+      a += reinterpret_cast<const float*>(&s_acc[w][0])[c];
+      ws += s_wsum[w];
+    }
+    reinterpret_cast<TQ*>(p.out)[bh * D + c] = from_f32<TQ>(a / ws);
   }
 }
 

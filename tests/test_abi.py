@@ -121,7 +121,13 @@ def test_workspace_plan(lib):
     o = 4 * 64 * parts * 128 * 4
     ml = 4 * 64 * parts * 8
     assert ws == -(-o // 256) * 256 + -(-ml // 256) * 256
-    # automatic partition: halves from 512 while the grid is under two CTAs per SM
-    assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(_desc(num_kv_heads=32))) == 512
+    # automatic partition: 128 KB of K rows per KV head (512 tokens at fp16 and
+    # head_dim 128, 1024 at head_dim 64 or E4M3), halved while the grid is
+    # under two CTAs per SM
+    d32 = _desc(num_kv_heads=32, head_dim=128)
+    assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(d32)) == 512
+    assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(_desc(num_kv_heads=32))) == 1024
+    d8 = _desc(num_kv_heads=8, head_dim=128, cache_dtype=B.PA_E4M3)
+    assert lib.pa_decode_partition_tokens(256, 8192, ctypes.byref(d8)) == 1024
     assert lib.pa_decode_partition_tokens(1, 4096, ctypes.byref(d)) == 64
     assert lib.pa_decode_partition_tokens(1, 100, ctypes.byref(d)) == 64
