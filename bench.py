@@ -48,6 +48,7 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama2_7b.md")
 KERNEL_SOURCES = ["paged_kv_cache_410_b200/csrc/pa_api.cu",
                   "paged_kv_cache_410_b200/csrc/pa_common.cuh",
                   "paged_kv_cache_410_b200/csrc/pa_decode.cuh",
+                  "paged_kv_cache_410_b200/csrc/pa_prefix.cuh",
                   "paged_kv_cache_410_b200/csrc/pa_append_copy.cuh"]
 
 
@@ -304,14 +305,24 @@ def run_ours(args):
         raise RuntimeError("libpagedattn.so is not built; run __graft_entry__.build()")
 
     w = make_workload(args.workload, rank, args.batch)
-    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens)
+    spb = w.meta.get("shared_prefix_blocks", 0) if args.cascade == "auto" else 0
+    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb)
     stream = torch.cuda.current_stream(dev)
     sb = A.step_bytes(w)
-    plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context,
-                                                                     step.cache)
-    n_parts = max(1, math.ceil(w.max_context / plan_pt))
-    launches_per_step = (1 + 1 + (1 if n_parts > 1 else 0) +
-                         math.ceil(len(w.copy_pairs) / 256))
+    if spb:
+        prefix_len = spb * w.block_size
+        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
+            w.batch, max(w.max_context - prefix_len, 0), step.cache)
+        n_parts = max(1, math.ceil((w.max_context - prefix_len) / plan_pt))
+        decode_launches = 3  # prefix kernel, suffix kernel, merge
+        decode_name = "pa_decode_shared_prefix (prefix + suffix + merge kernels)"
+    else:
+        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context,
+                                                                         step.cache)
+        n_parts = max(1, math.ceil(w.max_context / plan_pt))
+        decode_launches = 1 + (1 if n_parts > 1 else 0)
+        decode_name = "pa_decode (main + split-K reduce)"
+    launches_per_step = 1 + decode_launches + math.ceil(len(w.copy_pairs) / 256)
 
     for _ in range(args.warmup):
         step.run()
@@ -395,7 +406,7 @@ def run_ours(args):
         "tokens_per_s_per_layer": tokens_per_s,
         "frac_of_hbm_peak": value / peak,
         "frac_of_hbm_spec_8tbs": value / SPEC_HBM_GBS,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (main + split-K reduce)",
+        "roofline": {"bound": "hbm", "kernel": decode_name,
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
@@ -431,6 +442,9 @@ def main(argv=None):
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cascade", choices=["auto", "off"], default="auto",
+                    help="decode a workload whose sequences share prefix blocks through "
+                         "pa_decode_shared_prefix (auto) or plain pa_decode (off)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -73,6 +73,8 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
 #define PA_DEVERR_BLOCK_ID 0x1u    /* a block-table entry outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT_LEN 0x2u /* context_len < 0, > max_context, or beyond the table */
 #define PA_DEVERR_SLOT 0x4u        /* append slot >= num_blocks * block_size */
+#define PA_DEVERR_PREFIX 0x8u      /* pa_decode_shared_prefix: a sequence does not start
+                                      with the shared prefix blocks, or is shorter */
 
 /* Describes one paged KV cache (one layer's K cache and V cache). */
 typedef struct pa_cache_desc {
@@ -138,6 +140,39 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                     const int32_t* context_lens, int32_t max_context, float scale, void* out,
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                     void* stream);
+
+/* Workspace bytes for pa_decode_shared_prefix (equals
+ * pa_decode_workspace_size when prefix_blocks == 0). Pure host function. */
+size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads,
+                                              int32_t max_context, int32_t prefix_blocks,
+                                              int32_t partition_tokens,
+                                              const pa_cache_desc* cache);
+
+/* pa_decode for a batch whose sequences all begin with the same physical
+ * blocks -- a shared system prompt stored once and referenced by every
+ * sequence (KV cache article, section "PagedAttention：把操作系统的老智慧搬进
+ * 推理引擎": prefix sharing).
+ * Precondition: block_tables[b][0 .. prefix_blocks) are the same for every b,
+ * and every context_lens[b] >= prefix_blocks * block_size. Then the result
+ * equals pa_decode's (up to rounding): the attention over the shared prefix
+ * is computed once per KV head for all batch x group query columns (a dense
+ * tensor-core contraction that reads each prefix block a few times instead
+ * of once per sequence), each sequence's own tokens after the prefix are
+ * handled as in pa_decode, and the two are merged as split-K partials.
+ * A sequence whose table or length breaks the precondition sets
+ * PA_DEVERR_PREFIX (its output is then not meaningful).
+ *   prefix_blocks  number of shared leading blocks (0: plain pa_decode);
+ *                  prefix_blocks * block_size must not exceed max_context.
+ *   workspace      at least pa_decode_shared_prefix_workspace_size(...) bytes,
+ *                  256-byte aligned; always needed when prefix_blocks > 0.
+ * Other arguments as for pa_decode; partition_tokens applies to the suffixes. */
+pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
+                                  int32_t num_q_heads, const void* k_cache, const void* v_cache,
+                                  const pa_cache_desc* cache, const int32_t* block_tables,
+                                  int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                  int32_t max_context, int32_t prefix_blocks, float scale,
+                                  void* out, int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* Copy whole blocks: for p in [0, num_pairs), K block pairs_host[2p] ->
  * K block pairs_host[2p+1], and the same for V.

@@ -22,12 +22,13 @@ PA_F16, PA_BF16, PA_E4M3 = 0, 1, 2
 PA_OK = 0
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
           4: "PA_ERR_WORKSPACE", 5: "PA_ERR_DEVICE_BOUNDS"}
-DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT = 0x1, 0x2, 0x4
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_PREFIX = 0x1, 0x2, 0x4, 0x8
 
 # names of every symbol include/pa_api.h declares
 EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tokens",
             "pa_decode", "pa_copy_blocks", "pa_get_device_error", "pa_status_string",
-            "pa_version", "pa_decode_static_workspace"]
+            "pa_version", "pa_decode_static_workspace",
+            "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -78,6 +79,11 @@ def load_library(path: str = LIB_PATH):
     lib.pa_decode_static_workspace.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32,
                                                ctypes.c_float, P, i32, P]
     lib.pa_decode_static_workspace.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, D]
+    lib.pa_decode_shared_prefix_workspace_size.restype = ctypes.c_size_t
+    lib.pa_decode_shared_prefix.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, i32,
+                                            ctypes.c_float, P, i32, P, ctypes.c_size_t, P]
+    lib.pa_decode_shared_prefix.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -170,6 +176,34 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache
                        _ptr(context_lens), int(max_context), float(scale), _ptr(out),
                        int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_shared_prefix_workspace_size(batch, num_q_heads, max_context, prefix_blocks,
+                                           cache: PagedCache, partition_tokens=0) -> int:
+    lib = load_library()
+    d = cache.desc()
+    return int(lib.pa_decode_shared_prefix_workspace_size(batch, num_q_heads, max_context,
+                                                          prefix_blocks, partition_tokens,
+                                                          ctypes.byref(d)))
+
+
+def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                            cache: PagedCache, max_context: int, prefix_blocks: int,
+                            partition_tokens: int = 0, workspace=None, stream=None):
+    """pa_decode for a batch whose block tables all start with the same
+    `prefix_blocks` physical blocks: the shared prefix is attended once per
+    KV head for all sequences, then merged with each sequence's suffix."""
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.pa_decode_shared_prefix(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache),
+                                     _ptr(v_cache), ctypes.byref(d), _ptr(block_tables),
+                                     block_tables.shape[1], _ptr(context_lens), int(max_context),
+                                     int(prefix_blocks), float(scale), _ptr(out),
+                                     int(partition_tokens), _ptr(workspace), ws_bytes,
+                                     _stream(stream))
+    _check(rc, "pa_decode_shared_prefix")
 
 
 def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, scale, out,

@@ -18,6 +18,7 @@
 #include "pa_append_copy.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefix.cuh"
 
 namespace {
 
@@ -116,8 +117,26 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
   return e;
 }
 
+// Split-K merge: 1, 2, 4 or 8 warps per (sequence, query head) row by the
+// number of partials per row.
+template <typename TQ, int D>
+pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
+  auto go = [&](auto kern, int rows_per_cta) {
+    const int64_t ctas = (rows + rows_per_cta - 1) / rows_per_cta;
+    kern<<<static_cast<unsigned>(ctas), pa::kReduceWarps * 32, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  };
+  if (p.num_partitions <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1>, 8);
+  if (p.num_partitions <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2>, 4);
+  if (p.num_partitions <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4>, 2);
+  return go(pa::pa_decode_reduce_kernel<TQ, D, 8>, 1);
+}
+
+// Decode kernel over `grid_x` partition columns, then the split-K merge when
+// the plan has more than one partial per sequence (or always, in cascade mode).
 template <typename TQ, int CK, int D, int NH>
-pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
+pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH>;
   const int bt_entries =
@@ -125,24 +144,181 @@ pa_status launch_decode_t(const pa::DecodeParams& p, cudaStream_t st) {
   const int smem = S::kMainBytes + bt_entries * 4;
   if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
   if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
-  dim3 grid(p.num_partitions, p.num_kv_heads * p.head_groups, p.batch);
+  dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
   kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (p.num_partitions > 1) {
-    pa::pa_decode_reduce_kernel<TQ, D>
-        <<<dim3(p.num_q_heads, p.batch), pa::kReduceWarps * 32, 0, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (p.num_partitions > 1 || p.force_partials) {
+    const pa_status rs = launch_reduce<TQ, D>(p, st);
+    if (rs != PA_OK) return rs;
   }
   return PA_OK;
 }
 
 template <typename TQ, int CK>
-pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, cudaStream_t st) {
+pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, int grid_x,
+                          cudaStream_t st) {
   // query heads per CTA: the whole group up to 16; 8-head column blocks
   const bool two = std::min(p.group, 16) > 8;
   if (head_dim == 64)
-    return two ? launch_decode_t<TQ, CK, 64, 2>(p, st) : launch_decode_t<TQ, CK, 64, 1>(p, st);
-  return two ? launch_decode_t<TQ, CK, 128, 2>(p, st) : launch_decode_t<TQ, CK, 128, 1>(p, st);
+    return two ? launch_decode_t<TQ, CK, 64, 2>(p, grid_x, st)
+               : launch_decode_t<TQ, CK, 64, 1>(p, grid_x, st);
+  return two ? launch_decode_t<TQ, CK, 128, 2>(p, grid_x, st)
+             : launch_decode_t<TQ, CK, 128, 1>(p, grid_x, st);
+}
+
+pa_status launch_decode(const pa::DecodeParams& p, int q_dtype, const pa_cache_desc* cache,
+                        cudaStream_t s, int grid_x = -1) {
+  if (grid_x < 0) grid_x = p.num_partitions;
+  switch (cache->cache_dtype) {
+    case PA_F16: return launch_decode_d<__half, pa::kF16>(p, cache->head_dim, grid_x, s);
+    case PA_BF16: return launch_decode_d<__nv_bfloat16, pa::kBF16>(p, cache->head_dim, grid_x, s);
+    default:
+      return q_dtype == PA_F16
+                 ? launch_decode_d<__half, pa::kE4M3>(p, cache->head_dim, grid_x, s)
+                 : launch_decode_d<__nv_bfloat16, pa::kE4M3>(p, cache->head_dim, grid_x, s);
+  }
+}
+
+// Host-side checks shared by the decode entry points. *nothing is set when
+// the call is valid but has no work (batch == 0).
+pa_status check_decode_args(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                            const void* k_cache, const void* v_cache, const pa_cache_desc* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context, float scale,
+                            void* out, int32_t partition_tokens, int* bs_log2, bool* nothing) {
+  *nothing = false;
+  pa_status st = check_cache(cache, bs_log2);
+  if (st != PA_OK) return st;
+  if (batch < 0 || num_q_heads <= 0 || max_context < 0 || max_blocks_per_seq <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype != PA_E4M3 && cache->cache_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
+  if (partition_tokens != 0 &&
+      (partition_tokens < 16 || partition_tokens > (1 << 20) || partition_tokens % 16 != 0))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (batch == 0) {
+    *nothing = true;
+    return PA_OK;
+  }
+  if (batch > 65535) return PA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype == PA_E4M3 && (!cache->k_scale || !cache->v_scale))
+    return PA_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  if (static_cast<int64_t>(cache->num_kv_heads) * ((group + 15) / 16) > 65535)
+    return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa::DecodeParams decode_params(const void* q, int32_t batch, int32_t num_q_heads,
+                               const void* k_cache, const void* v_cache,
+                               const pa_cache_desc* cache, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* context_lens,
+                               int32_t max_context, float scale, void* out, int bs_log2) {
+  pa::DecodeParams p{};
+  p.q = q;
+  p.out = out;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.num_blocks = cache->num_blocks;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.group = num_q_heads / cache->num_kv_heads;
+  p.head_groups = (p.group + 15) / 16;
+  p.bs_log2 = bs_log2;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context = max_context;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return p;
+}
+
+// ---- shared-prefix (cascade) decode -----------------------------------------
+constexpr int kPrefixWarps = 4;   // 16 query columns per warp
+constexpr int kPrefixStages = 2;  // CTA-wide cp.async stages of one 32/64-token block
+constexpr int kPrefixChunkMax = 512;
+
+struct CascadePlan {
+  int prefix_len;
+  int chunk_tokens;
+  int num_chunks;
+  int suffix_partition_tokens;
+  int suffix_partitions;
+  int num_partitions;  // chunks + suffix partitions
+  size_t ws_o_bytes;
+  size_t ws_bytes;
+};
+
+CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_context,
+                              int prefix_blocks, int partition_tokens, const pa_cache_desc* cd) {
+  CascadePlan pl{};
+  pl.prefix_len = prefix_blocks * cd->block_size;
+  // prefix tokens per prefix CTA: the whole prefix up to kPrefixChunkMax
+  pl.chunk_tokens = std::min((pl.prefix_len + 15) / 16 * 16, kPrefixChunkMax);
+  pl.num_chunks = (pl.prefix_len + pl.chunk_tokens - 1) / pl.chunk_tokens;
+  const int64_t suffix_max = std::max<int64_t>(max_context - pl.prefix_len, 0);
+  pl.suffix_partition_tokens =
+      partition_tokens > 0 ? partition_tokens : auto_partition(batch, suffix_max, cd);
+  pl.suffix_partitions =
+      static_cast<int>((suffix_max + pl.suffix_partition_tokens - 1) / pl.suffix_partition_tokens);
+  pl.num_partitions = pl.num_chunks + pl.suffix_partitions;
+  pl.ws_o_bytes = round_up(static_cast<size_t>(batch * num_q_heads) * pl.num_partitions *
+                               cd->head_dim * sizeof(float),
+                           256);
+  pl.ws_bytes = pl.ws_o_bytes + round_up(static_cast<size_t>(batch * num_q_heads) *
+                                             pl.num_partitions * sizeof(float2),
+                                         256);
+  return pl;
+}
+
+// Prefix CTAs and suffix CTAs in one launch (so they overlap), then the merge.
+template <typename TQ, int CK, int D, int NH>
+pa_status launch_cascade_t(const pa::DecodeParams& p, const CascadePlan& pl, cudaStream_t st) {
+  using SD = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
+  using SP = pa::PrefixSmem<CK, D, kPrefixStages, pa::prefix_subtiles<CK>()>;
+  auto kern = pa::pa_cascade_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, kPrefixWarps,
+                                    kPrefixStages>;
+  const int bt_d = std::min((p.partition_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
+  const int bt_p = std::min((p.prefix_chunk_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
+  const int smem = std::max(SD::kMainBytes + bt_d * 4, SP::kPipeBytes + bt_p * 4);
+  if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
+  if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
+  pa::CascadeGrid cg{};
+  cg.n_chunks = pl.num_chunks;
+  const int64_t rows = static_cast<int64_t>(p.batch) * p.group;
+  cg.n_rowblocks = static_cast<int>((rows + 16 * kPrefixWarps - 1) / (16 * kPrefixWarps));
+  const int64_t n_prefix = static_cast<int64_t>(cg.n_chunks) * cg.n_rowblocks * p.num_kv_heads;
+  cg.n_suffix_parts = std::max(pl.suffix_partitions, 1);
+  const int64_t n_suffix =
+      static_cast<int64_t>(cg.n_suffix_parts) * p.num_kv_heads * p.head_groups * p.batch;
+  const int64_t total = n_prefix + n_suffix;
+  if (total > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  cg.n_prefix = static_cast<int>(n_prefix);
+  cg.n_suffix = static_cast<int>(n_suffix);
+  cg.ratio = static_cast<int>(n_suffix / std::max<int64_t>(n_prefix, 1));
+  kern<<<static_cast<unsigned>(total), kDecodeWarps * 32, smem, st>>>(p, cg);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  return launch_reduce<TQ, D>(p, st);
+}
+
+template <typename TQ, int CK>
+pa_status launch_cascade_d(const pa::DecodeParams& p, const CascadePlan& pl, int head_dim,
+                           cudaStream_t st) {
+  const bool two = std::min(p.group, 16) > 8;
+  if (head_dim == 64)
+    return two ? launch_cascade_t<TQ, CK, 64, 2>(p, pl, st)
+               : launch_cascade_t<TQ, CK, 64, 1>(p, pl, st);
+  return two ? launch_cascade_t<TQ, CK, 128, 2>(p, pl, st)
+             : launch_cascade_t<TQ, CK, 128, 1>(p, pl, st);
 }
 
 }  // namespace
@@ -226,68 +402,93 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                     void* stream) {
   int bs_log2 = 0;
-  pa_status st = check_cache(cache, &bs_log2);
-  if (st != PA_OK) return st;
-  if (batch < 0 || num_q_heads <= 0 || max_context < 0 || max_blocks_per_seq <= 0)
-    return PA_ERR_INVALID_ARG;
-  if (num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-  if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_INVALID_ARG;
-  if (cache->cache_dtype != PA_E4M3 && cache->cache_dtype != q_dtype) return PA_ERR_UNSUPPORTED;
-  if (partition_tokens != 0 &&
-      (partition_tokens < 16 || partition_tokens > (1 << 20) || partition_tokens % 16 != 0))
-    return PA_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  if (batch == 0) return PA_OK;
-  if (batch > 65535) return PA_ERR_UNSUPPORTED;
-  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out)
-    return PA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return PA_ERR_INVALID_ARG;
-  if (cache->cache_dtype == PA_E4M3 && (!cache->k_scale || !cache->v_scale))
-    return PA_ERR_INVALID_ARG;
-
+  bool nothing = false;
+  pa_status st = check_decode_args(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, out, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK || nothing) return st;
   const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
   }
-  const int group = num_q_heads / cache->num_kv_heads;
-  const int head_groups = (group + 15) / 16;
-  if (static_cast<int64_t>(cache->num_kv_heads) * head_groups > 65535) return PA_ERR_UNSUPPORTED;
-
-  pa::DecodeParams p{};
-  p.q = q;
-  p.out = out;
-  p.k_cache = k_cache;
-  p.v_cache = v_cache;
-  p.k_scale = cache->k_scale;
-  p.v_scale = cache->v_scale;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
+  pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
+                                     block_tables, max_blocks_per_seq, context_lens, max_context,
+                                     scale, out, bs_log2);
   p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
   p.ws_ml = pl.ws_bytes
                 ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
                 : nullptr;
-  p.num_blocks = cache->num_blocks;
-  p.batch = batch;
-  p.num_q_heads = num_q_heads;
-  p.num_kv_heads = cache->num_kv_heads;
-  p.group = group;
-  p.head_groups = head_groups;
-  p.bs_log2 = bs_log2;
-  p.max_blocks_per_seq = max_blocks_per_seq;
-  p.max_context = max_context;
   p.partition_tokens = pl.partition_tokens;
   p.num_partitions = pl.num_partitions;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  return launch_decode(p, q_dtype, cache, as_stream(stream));
+}
 
+size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads,
+                                              int32_t max_context, int32_t prefix_blocks,
+                                              int32_t partition_tokens,
+                                              const pa_cache_desc* cache) {
+  int bs_log2 = 0;
+  if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || num_q_heads <= 0 ||
+      max_context < 0 || partition_tokens < 0 || prefix_blocks < 0)
+    return 0;
+  if (prefix_blocks == 0)
+    return make_plan(batch, num_q_heads, max_context, partition_tokens, cache).ws_bytes;
+  return make_cascade_plan(batch, num_q_heads, max_context, prefix_blocks, partition_tokens,
+                           cache)
+      .ws_bytes;
+}
+
+pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
+                                  int32_t num_q_heads, const void* k_cache, const void* v_cache,
+                                  const pa_cache_desc* cache, const int32_t* block_tables,
+                                  int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                  int32_t max_context, int32_t prefix_blocks, float scale,
+                                  void* out, int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  int bs_log2 = 0;
+  bool nothing = false;
+  pa_status st = check_decode_args(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, out, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK) return st;
+  if (prefix_blocks < 0 || prefix_blocks > max_blocks_per_seq ||
+      static_cast<int64_t>(prefix_blocks) * cache->block_size > max_context)
+    return PA_ERR_INVALID_ARG;
+  if (nothing) return PA_OK;
+  if (prefix_blocks == 0)
+    return pa_decode(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache, block_tables,
+                     max_blocks_per_seq, context_lens, max_context, scale, out, partition_tokens,
+                     workspace, workspace_bytes, stream);
+  const CascadePlan pl = make_cascade_plan(batch, num_q_heads, max_context, prefix_blocks,
+                                           partition_tokens, cache);
+  if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
+
+  pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
+                                     block_tables, max_blocks_per_seq, context_lens, max_context,
+                                     scale, out, bs_log2);
+  p.ws_o = reinterpret_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes);
+  p.partition_tokens = pl.suffix_partition_tokens;
+  p.num_partitions = pl.num_partitions;
+  p.prefix_blocks = prefix_blocks;
+  p.token_start = pl.prefix_len;
+  p.part_offset = pl.num_chunks;
+  p.force_partials = 1;
+  p.prefix_chunk_tokens = pl.chunk_tokens;
+
+  // One launch: the shared prefix once per block of query rows, and every
+  // sequence's own suffix (at least one partition column, so that each
+  // sequence's table is checked against the shared prefix); then the merge.
   const cudaStream_t s = as_stream(stream);
   switch (cache->cache_dtype) {
-    case PA_F16: return launch_decode_d<__half, pa::kF16>(p, cache->head_dim, s);
-    case PA_BF16: return launch_decode_d<__nv_bfloat16, pa::kBF16>(p, cache->head_dim, s);
+    case PA_F16: return launch_cascade_d<__half, pa::kF16>(p, pl, cache->head_dim, s);
+    case PA_BF16: return launch_cascade_d<__nv_bfloat16, pa::kBF16>(p, pl, cache->head_dim, s);
     default:
-      return q_dtype == PA_F16 ? launch_decode_d<__half, pa::kE4M3>(p, cache->head_dim, s)
-                               : launch_decode_d<__nv_bfloat16, pa::kE4M3>(p, cache->head_dim, s);
+      return q_dtype == PA_F16
+                 ? launch_cascade_d<__half, pa::kE4M3>(p, pl, cache->head_dim, s)
+                 : launch_cascade_d<__nv_bfloat16, pa::kE4M3>(p, pl, cache->head_dim, s);
   }
 }
 

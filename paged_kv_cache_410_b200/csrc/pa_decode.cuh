@@ -59,13 +59,41 @@ struct DecodeParams {
   int partition_tokens;
   int num_partitions;
   float scale_log2;  // scale * log2(e)
+  // Shared-prefix (cascade) mode; all zero for a plain decode. Tokens before
+  // token_start (= prefix_blocks * block_size) are the prefix every sequence
+  // shares; the suffix kernel covers [token_start, L) and writes its
+  // partials after `part_offset` prefix partials, always as partials.
+  int prefix_blocks;
+  int token_start;
+  int part_offset;
+  int force_partials;
+  int prefix_chunk_tokens;  // prefix tokens per prefix-kernel CTA (cascade mode)
 };
+
+// Number of split-K partials of a sequence of length L (the prefix's ones
+// included) and the clamped length, shared by the decode and reduce kernels.
+__device__ __forceinline__ int clamp_context(const DecodeParams& p, int L) {
+  const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
+  const int cap = static_cast<int>(table_cap < p.max_context ? table_cap : p.max_context);
+  return L < 0 ? 0 : (L > cap ? cap : L);
+}
+__device__ __forceinline__ int suffix_partitions(const DecodeParams& p, int L) {
+  const int n = L - p.token_start;
+  return n > 0 ? (n + p.partition_tokens - 1) / p.partition_tokens : 0;
+}
 
 enum CacheKind { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
 
 // Block ids of one partition staged in shared memory (longer slices are read
 // from global memory row by row).
 constexpr int kBlockIdsInSmem = 1024;
+
+// Online softmax keeps a reference max per query and moves it only when a
+// tile's max exceeds it by more than this (log2 units): the exponentials stay
+// at most 2^8, exact in f16/bf16 and far from overflow in the fp32 sums, and
+// the accumulator is rescaled only when the reference moves. The reference
+// cancels in the final normalisation.
+constexpr float kRescaleLog2 = 8.f;
 
 template <int CK, int D>
 struct TileGeom {
@@ -99,14 +127,229 @@ struct DecodeSmem {
   // + block-table slice of the partition (int32), sized at launch
 };
 
+// ---- per-warp attention math shared by the decode and prefix kernels -------
+//
+// A warp owns NH blocks of 8 query columns. Thread (g = lane/4, t = lane%4)
+// holds the B-operand fragments of column 8*nh + g and the O^T accumulator
+// o[mt][nh] = {(channel row g, columns 2t, 2t+1), (channel row g+8, same)}.
+
+// Q^T fragments: qb[kk][nh] = {channels of k-slots 2t,2t+1 ; 2t+8,2t+9} of the
+// query row rows[nh] (nullptr: a padding column of zeros). For E4M3 the row
+// is first multiplied by the K scale (q' = q * k_scale) and split into f16
+// hi + lo; its channel order inside each 32-channel group gq (shared with the
+// K fragments of attend_tile): k-step 2gq + h holds channels 8t + 4h + {0,1}
+// in slots 2t, 2t+1 and 8t + 4h + {2,3} in slots 2t+8, 2t+9.
+template <typename TQ, int CK, int D, int NH>
+__device__ __forceinline__ void load_query_fragments(
+    const TQ* const (&rows)[NH], const float* k_scale_row, uint32_t (&qb)[D / 16][NH][2],
+    uint32_t (&qlo)[CK == kE4M3 ? D / 16 : 1][NH][2]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    const TQ* qr = rows[nh];
+    const bool ok = qr != nullptr;
+    if constexpr (CK != kE4M3) {
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qr);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qb[kk][nh][0] = ok ? q32[(kk * 16 + 2 * t) / 2] : 0u;
+        qb[kk][nh][1] = ok ? q32[(kk * 16 + 8 + 2 * t) / 2] : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int gq = 0; gq < D / 32; ++gq) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int kk = 2 * gq + h;
+          const int c = gq * 32 + 8 * t + 4 * h;
+          float x[4], hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[e] = ok ? to_f32<TQ>(qr[c + e]) * k_scale_row[c + e] : 0.f;
+            hi[e] = __half2float(__float2half_rn(x[e]));
+            lo[e] = x[e] - hi[e];
+          }
+          qb[kk][nh][0] = pack2<false>(hi[0], hi[1]);
+          qb[kk][nh][1] = pack2<false>(hi[2], hi[3]);
+          qlo[kk][nh][0] = pack2<false>(lo[0], lo[1]);
+          qlo[kk][nh][1] = pack2<false>(lo[2], lo[3]);
+        }
+      }
+    }
+  }
+}
+
+// Channels of O^T rows g and g + 8 in channel block mt.
+template <int CK, int D>
+__device__ __forceinline__ int2 accumulator_channels(int mt, int g) {
+  if constexpr (CK != kE4M3) return make_int2(16 * mt + g, 16 * mt + 8 + g);
+  return make_int2((D / 8) * g + 2 * mt, (D / 8) * g + 2 * mt + 1);
+}
+
+// One 16-token tile of K and V in shared memory (rows >= nvalid are zero and
+// masked) against the warp's query columns: S^T = K Q^T, online softmax
+// update of the per-column running max / sum (log2 domain), O^T += V^T P^T.
+template <int CK, int D, int NH>
+__device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nvalid,
+                                            float scale_log2,
+                                            const uint32_t (&qb)[D / 16][NH][2],
+                                            const uint32_t (&qlo)[CK == kE4M3 ? D / 16 : 1][NH][2],
+                                            float (&o)[D / 16][NH][4], float (&m_run)[NH][2],
+                                            float (&l_run)[NH][2]) {
+  using G = TileGeom<CK, D>;
+  constexpr bool kMmaBF16 = (CK == kBF16);  // MMA operand type (E4M3 widens to f16)
+  constexpr int KSTEPS = D / 16;
+  constexpr int MT = D / 16;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+
+  // S^T = K Q^T: s[nh] = {(token g, columns 2t, 2t+1), (token g+8, same)}
+  float s[NH][4];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
+  if constexpr (CK != kE4M3) {
+    const int mi = lane >> 3;
+    const int tok = (lane & 7) + 8 * (mi & 1);
+    const int chk = mi >> 1;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      uint32_t a[4];
+      ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(tok, 2 * kk + chk));
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(s[nh], a, qb[kk][nh][0], qb[kk][nh][1]);
+    }
+  } else {
+#pragma unroll
+    for (int gq = 0; gq < D / 32; ++gq) {
+      const int c = 2 * gq + (t >> 1);
+      const int bo = (t & 1) * 8;
+      const uint2 wl = lds64(sk_a + G::off(g, c) + bo);      // token g
+      const uint2 wh = lds64(sk_a + G::off(g + 8, c) + bo);  // token g + 8
+      uint32_t a0[4], a1[4];
+      e4m3x4_to_f16x2x2(wl.x, a0[0], a0[2]);
+      e4m3x4_to_f16x2x2(wh.x, a0[1], a0[3]);
+      e4m3x4_to_f16x2x2(wl.y, a1[0], a1[2]);
+      e4m3x4_to_f16x2x2(wh.y, a1[1], a1[3]);
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        mma_16816<false>(s[nh], a0, qb[2 * gq][nh][0], qb[2 * gq][nh][1]);
+        mma_16816<false>(s[nh], a0, qlo[2 * gq][nh][0], qlo[2 * gq][nh][1]);
+        mma_16816<false>(s[nh], a1, qb[2 * gq + 1][nh][0], qb[2 * gq + 1][nh][1]);
+        mma_16816<false>(s[nh], a1, qlo[2 * gq + 1][nh][0], qlo[2 * gq + 1][nh][1]);
+      }
+    }
+  }
+
+  // online softmax per column; the max is reduced over the 16 tokens
+  // (lanes with the same t, both row halves)
+  const bool va = g < nvalid;
+  const bool vb = g + 8 < nvalid;
+  uint32_t pb[NH][2];
+  bool grew = false;
+  float alpha[NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    float pr[2][2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float x0 = va ? s[nh][e] * scale_log2 : -INFINITY;
+      const float x1 = vb ? s[nh][2 + e] * scale_log2 : -INFINITY;
+      float mx = fmaxf(x0, x1);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      // mx is finite (token 0 of the tile exists), so the first tile always
+      // sets the reference
+      const bool up = mx > m_run[nh][e] + kRescaleLog2;
+      grew |= up;
+      const float m_ref = up ? mx : m_run[nh][e];
+      alpha[nh][e] = up ? ex2(m_run[nh][e] - m_ref) : 1.f;  // exactly 1 when unchanged
+      pr[0][e] = ex2(x0 - m_ref);
+      pr[1][e] = ex2(x1 - m_ref);
+      l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + (pr[0][e] + pr[1][e]);
+      m_run[nh][e] = m_ref;
+    }
+    // (token, column) 8x8 blocks -> transposed: column g, tokens 2t,2t+1 | 2t+8,2t+9
+    pb[nh][0] = movmatrix_trans(pack2<kMmaBF16>(pr[0][0], pr[0][1]));
+    pb[nh][1] = movmatrix_trans(pack2<kMmaBF16>(pr[1][0], pr[1][1]));
+  }
+  if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        o[mt][nh][0] *= alpha[nh][0];
+        o[mt][nh][1] *= alpha[nh][1];
+        o[mt][nh][2] *= alpha[nh][0];
+        o[mt][nh][3] *= alpha[nh][1];
+      }
+  }
+
+  // O^T += V^T P^T
+  if constexpr (CK != kE4M3) {
+    const int mi = lane >> 3;
+    const int tok = (lane & 7) + 8 * (mi >> 1);
+    const int chk = mi & 1;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a[0], a[1], a[2], a[3], sv_a + G::off(tok, 2 * mt + chk));
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(o[mt][nh], a, pb[nh][0], pb[nh][1]);
+    }
+  } else {
+    // Row m of O^T block mt is channel DPT*g + 2*mt (m = g) or that + 1
+    // (m = g + 8): this thread reads channels [DPT*g, DPT*g + DPT) of token
+    // rows 2t, 2t+1, 2t+8, 2t+9 and pairs tokens with byte permutes.
+    constexpr int DPT = D / 8;
+    constexpr int WORDS = DPT / 4;
+    uint32_t ra[4][WORDS];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int r = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
+      const int byte0 = DPT * g;
+      const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
+      if constexpr (WORDS == 4) {
+        const uint4 w = lds128(addr);
+        ra[q4][0] = w.x;
+        ra[q4][1] = w.y;
+        ra[q4][2] = w.z;
+        ra[q4][3] = w.w;
+      } else {
+        const uint2 w = lds64(addr);
+        ra[q4][0] = w.x;
+        ra[q4][1] = w.y;
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < WORDS; ++w) {
+      uint32_t f[4], e[4];
+      e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x5140), f[0], f[1]);
+      e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x7362), f[2], f[3]);
+      e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x5140), e[0], e[1]);
+      e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x7362), e[2], e[3]);
+      const uint32_t a0[4] = {f[0], f[1], e[0], e[1]};  // channel block 2w
+      const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        mma_16816<false>(o[2 * w][nh], a0, pb[nh][0], pb[nh][1]);
+        mma_16816<false>(o[2 * w + 1][nh], a1, pb[nh][0], pb[nh][1]);
+      }
+    }
+  }
+}
+
 // NH: 8-head column blocks per CTA (1 for groups of up to 8 query heads, 2
 // for 9..16).
+//
+// One decode CTA: partition `part` of sequence `b`, for KV head / head group
+// `by` (= kv_head * head_groups + head_group).
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH>
-__global__ void __launch_bounds__(NW * 32)
-    pa_decode_kernel(const DecodeParams p) {
+__device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part, const int by,
+                                           const int b) {
   using G = TileGeom<CK, D>;
   using S = DecodeSmem<CK, D, NW, NSTAGE>;
-  constexpr bool kMmaBF16 = (CK == kBF16);  // MMA operand type (E4M3 widens to f16)
   constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T
   constexpr int MT = D / 16;                // 16-channel row blocks of O^T
   constexpr int RPI = 32 / G::CPR;          // tile rows one load instruction covers
@@ -120,34 +363,37 @@ __global__ void __launch_bounds__(NW * 32)
   const int g = lane >> 2;  // MMA group id
   const int t = lane & 3;   // thread in group
 
-  const int b = blockIdx.z;
-  const int hk = blockIdx.y / p.head_groups;
-  const int hgrp = blockIdx.y - hk * p.head_groups;
-  const int part = blockIdx.x;
+  const int hk = by / p.head_groups;
+  const int hgrp = by - hk * p.head_groups;
   const int row0 = hgrp * 16;
   const int nrows = min(16, p.group - row0);  // query heads of this CTA
   const int hq0 = hk * p.group + row0;
 
   // ---- sequence length, checked against what the launch covers ----------
-  int L = p.context_lens[b];
-  const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
-  const int cap = static_cast<int>(table_cap < p.max_context ? table_cap : p.max_context);
-  if (L < 0 || L > cap) {
-    if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(PA_DEVERR_CONTEXT_LEN);
-    L = L < 0 ? 0 : cap;
+  const int L_in = p.context_lens[b];
+  const int L = clamp_context(p, L_in);
+  if (L != L_in && threadIdx.x == 0 && part == 0 && by == 0)
+    flag_error(PA_DEVERR_CONTEXT_LEN);
+  if (p.prefix_blocks > 0 && part == 0 && by == 0) {
+    // cascade mode: this sequence must start with the shared prefix blocks
+    const int32_t* row = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+    bool bad = L < p.token_start;
+    for (int i = threadIdx.x; i < p.prefix_blocks; i += NW * 32)
+      bad |= row[i] != p.block_tables[i];
+    if (bad) flag_error(PA_DEVERR_PREFIX);
   }
   const int PT = p.partition_tokens;
-  const int nparts = (L + PT - 1) / PT;
-  if (part >= (nparts > 0 ? nparts : 1)) return;
+  const int nparts = suffix_partitions(p, L);
+  if (part >= (nparts > 0 || p.force_partials ? nparts : 1)) return;
 
   TQ* out = reinterpret_cast<TQ*>(p.out);
-  if (L == 0) {
+  if (L == 0) {  // (plain mode only: a cascade launch has no partition here)
     for (int i = threadIdx.x; i < nrows * D; i += NW * 32)
       out[(static_cast<int64_t>(b) * p.num_q_heads + hq0 + i / D) * D + (i % D)] =
           from_f32<TQ>(0.f);
     return;
   }
-  const int t0 = part * PT;
+  const int t0 = p.token_start + part * PT;
   const int t1 = min(t0 + PT, L);
   const int ntiles = (t1 - t0 + 15) >> 4;
 
@@ -170,50 +416,17 @@ __global__ void __launch_bounds__(NW * 32)
   }
 
   // ---- Q^T fragments (B operand: k = channel, n = query head) -------------
-  // qb[kk][nh] = {channels of slots 2t,2t+1 ; slots 2t+8,2t+9} of head
-  // 8*nh + g.
   const TQ* qbase = reinterpret_cast<const TQ*>(p.q) +
                     (static_cast<int64_t>(b) * p.num_q_heads + hq0) * D;
   uint32_t qb[KSTEPS][NH][2];
   uint32_t qlo[CK == kE4M3 ? KSTEPS : 1][NH][2];
+  {
+    const TQ* rows[NH];
 #pragma unroll
-  for (int nh = 0; nh < NH; ++nh) {
-    const int hrow = 8 * nh + g;
-    const bool ok = hrow < nrows;
-    const TQ* qr = qbase + hrow * D;
-    if constexpr (CK != kE4M3) {
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qr);
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        qb[kk][nh][0] = ok ? q32[(kk * 16 + 2 * t) / 2] : 0u;
-        qb[kk][nh][1] = ok ? q32[(kk * 16 + 8 + 2 * t) / 2] : 0u;
-      }
-    } else {
-      // q' = q * k_scale[hk][:], as f16 hi + lo. Channel order inside each
-      // 32-channel group gq (shared with the K fragments below): k-step
-      // 2gq + h holds channels 8t + 4h + {0,1} in slots 2t, 2t+1 and
-      // 8t + 4h + {2,3} in slots 2t+8, 2t+9.
-      const float* ks = p.k_scale + static_cast<int64_t>(hk) * D;
-#pragma unroll
-      for (int gq = 0; gq < D / 32; ++gq) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int kk = 2 * gq + h;
-          const int c = gq * 32 + 8 * t + 4 * h;
-          float x[4], hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            x[e] = ok ? to_f32<TQ>(qr[c + e]) * ks[c + e] : 0.f;
-            hi[e] = __half2float(__float2half_rn(x[e]));
-            lo[e] = x[e] - hi[e];
-          }
-          qb[kk][nh][0] = pack2<false>(hi[0], hi[1]);
-          qb[kk][nh][1] = pack2<false>(hi[2], hi[3]);
-          qlo[kk][nh][0] = pack2<false>(lo[0], lo[1]);
-          qlo[kk][nh][1] = pack2<false>(lo[2], lo[3]);
-        }
-      }
-    }
+    for (int nh = 0; nh < NH; ++nh)
+      rows[nh] = 8 * nh + g < nrows ? qbase + (8 * nh + g) * D : nullptr;
+    load_query_fragments<TQ, CK, D, NH>(
+        rows, CK == kE4M3 ? p.k_scale + static_cast<int64_t>(hk) * D : nullptr, qb, qlo);
   }
   __syncthreads();  // s_bt ready
 
@@ -308,139 +521,7 @@ __global__ void __launch_bounds__(NW * 32)
     const uint32_t sv_a = sk_a + G::TB;
     const int tile = warp + it * NW;
     const int nvalid = t1 - (t0 + tile * 16);  // tokens of this tile that exist (>= 1)
-
-    // S^T = K Q^T: s[nh] = {(token g, heads 2t, 2t+1), (token g+8, heads 2t, 2t+1)}
-    float s[NH][4];
-#pragma unroll
-    for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
-    if constexpr (CK != kE4M3) {
-      const int mi = lane >> 3;
-      const int tok = (lane & 7) + 8 * (mi & 1);
-      const int chk = mi >> 1;
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        uint32_t a[4];
-        ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(tok, 2 * kk + chk));
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(s[nh], a, qb[kk][nh][0], qb[kk][nh][1]);
-      }
-    } else {
-#pragma unroll
-      for (int gq = 0; gq < D / 32; ++gq) {
-        const int c = 2 * gq + (t >> 1);
-        const int bo = (t & 1) * 8;
-        const uint2 wl = lds64(sk_a + G::off(g, c) + bo);      // token g
-        const uint2 wh = lds64(sk_a + G::off(g + 8, c) + bo);  // token g + 8
-        uint32_t a0[4], a1[4];
-        e4m3x4_to_f16x2x2(wl.x, a0[0], a0[2]);
-        e4m3x4_to_f16x2x2(wh.x, a0[1], a0[3]);
-        e4m3x4_to_f16x2x2(wl.y, a1[0], a1[2]);
-        e4m3x4_to_f16x2x2(wh.y, a1[1], a1[3]);
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh) {
-          mma_16816<false>(s[nh], a0, qb[2 * gq][nh][0], qb[2 * gq][nh][1]);
-          mma_16816<false>(s[nh], a0, qlo[2 * gq][nh][0], qlo[2 * gq][nh][1]);
-          mma_16816<false>(s[nh], a1, qb[2 * gq + 1][nh][0], qb[2 * gq + 1][nh][1]);
-          mma_16816<false>(s[nh], a1, qlo[2 * gq + 1][nh][0], qlo[2 * gq + 1][nh][1]);
-        }
-      }
-    }
-
-    // online softmax per query head (column), log2 domain; the max is
-    // reduced over the 16 tokens (lanes with the same t, both row halves)
-    const bool va = g < nvalid;
-    const bool vb = g + 8 < nvalid;
-    uint32_t pb[NH][2];
-    bool grew = false;
-    float alpha[NH][2];
-#pragma unroll
-    for (int nh = 0; nh < NH; ++nh) {
-      float pr[2][2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float x0 = va ? s[nh][e] * p.scale_log2 : -INFINITY;
-        const float x1 = vb ? s[nh][2 + e] * p.scale_log2 : -INFINITY;
-        float mx = fmaxf(x0, x1);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[nh][e], mx);  // finite: token 0 of the tile exists
-        const bool up = m_new > m_run[nh][e];
-        grew |= up;
-        alpha[nh][e] = up ? ex2(m_run[nh][e] - m_new) : 1.f;  // exactly 1 when unchanged
-        pr[0][e] = ex2(x0 - m_new);
-        pr[1][e] = ex2(x1 - m_new);
-        l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + (pr[0][e] + pr[1][e]);
-        m_run[nh][e] = m_new;
-      }
-      // (token, head) 8x8 blocks -> transposed: head g, tokens 2t,2t+1 | 2t+8,2t+9
-      pb[nh][0] = movmatrix_trans(pack2<kMmaBF16>(pr[0][0], pr[0][1]));
-      pb[nh][1] = movmatrix_trans(pack2<kMmaBF16>(pr[1][0], pr[1][1]));
-    }
-    if (__any_sync(0xffffffffu, grew)) {
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh) {
-          o[mt][nh][0] *= alpha[nh][0];
-          o[mt][nh][1] *= alpha[nh][1];
-          o[mt][nh][2] *= alpha[nh][0];
-          o[mt][nh][3] *= alpha[nh][1];
-        }
-    }
-
-    // O^T += V^T P^T
-    if constexpr (CK != kE4M3) {
-      const int mi = lane >> 3;
-      const int tok = (lane & 7) + 8 * (mi >> 1);
-      const int chk = mi & 1;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        uint32_t a[4];
-        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], sv_a + G::off(tok, 2 * mt + chk));
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(o[mt][nh], a, pb[nh][0], pb[nh][1]);
-      }
-    } else {
-      // Row m of O^T block mt is channel DPT*g + 2*mt (m = g) or that + 1
-      // (m = g + 8): this thread reads channels [DPT*g, DPT*g + DPT) of token
-      // rows 2t, 2t+1, 2t+8, 2t+9 and pairs tokens with byte permutes.
-      constexpr int DPT = D / 8;
-      constexpr int WORDS = DPT / 4;
-      uint32_t ra[4][WORDS];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int r = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
-        const int byte0 = DPT * g;
-        const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
-        if constexpr (WORDS == 4) {
-          const uint4 w = lds128(addr);
-          ra[q4][0] = w.x;
-          ra[q4][1] = w.y;
-          ra[q4][2] = w.z;
-          ra[q4][3] = w.w;
-        } else {
-          const uint2 w = lds64(addr);
-          ra[q4][0] = w.x;
-          ra[q4][1] = w.y;
-        }
-      }
-#pragma unroll
-      for (int w = 0; w < WORDS; ++w) {
-        uint32_t f[4], e[4];
-        e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x5140), f[0], f[1]);
-        e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x7362), f[2], f[3]);
-        e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x5140), e[0], e[1]);
-        e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x7362), e[2], e[3]);
-        const uint32_t a0[4] = {f[0], f[1], e[0], e[1]};  // channel block 2w
-        const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh) {
-          mma_16816<false>(o[2 * w][nh], a0, pb[nh][0], pb[nh][1]);
-          mma_16816<false>(o[2 * w + 1][nh], a1, pb[nh][0], pb[nh][1]);
-        }
-      }
-    }
+    attend_tile<CK, D, NH>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
     __syncwarp();  // this stage is reloaded by the next iteration
   }
   cp_async_wait<0>();
@@ -469,16 +550,9 @@ __global__ void __launch_bounds__(NW * 32)
         float* dst = w_o + (warp * 16 + head) * D;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          int c_lo, c_hi;
-          if constexpr (CK != kE4M3) {
-            c_lo = 16 * mt + g;
-            c_hi = c_lo + 8;
-          } else {
-            c_lo = (D / 8) * g + 2 * mt;
-            c_hi = c_lo + 1;
-          }
-          dst[c_lo] = o[mt][nh][e];
-          dst[c_hi] = o[mt][nh][2 + e];
+          const int2 ch = accumulator_channels<CK, D>(mt, g);
+          dst[ch.x] = o[mt][nh][e];
+          dst[ch.y] = o[mt][nh][2 + e];
         }
         if (g == 0) {
           w_m[warp * 16 + head] = m_run[nh][e];
@@ -503,7 +577,8 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncthreads();
 
-  const bool direct = nparts == 1;
+  const bool direct = nparts == 1 && !p.force_partials;
+  const int slot = p.part_offset + part;
   const float* vs = (CK == kE4M3) ? p.v_scale + static_cast<int64_t>(hk) * D : nullptr;
   for (int i = threadIdx.x; i < nrows * D; i += NW * 32) {
     const int row = i / D;
@@ -517,94 +592,112 @@ __global__ void __launch_bounds__(NW * 32)
     if (direct) {
       out[bh * D + c] = from_f32<TQ>(val);
     } else {
-      p.ws_o[(bh * p.num_partitions + part) * D + c] = val;
+      p.ws_o[(bh * p.num_partitions + slot) * D + c] = val;
       if (c == 0)
-        p.ws_ml[bh * p.num_partitions + part] =
+        p.ws_ml[bh * p.num_partitions + slot] =
             make_float2(r_stat[2 * row], r_stat[2 * row + 1]);
     }
   }
+}
+
+// grid: (partitions, num_kv_heads * head_groups, batch)
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH>
+__global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
+  decode_cta<TQ, CK, D, NW, NSTAGE, NH>(p, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
 // and normalised output o_p, out = sum_p w_p o_p / sum_p w_p where
 // w_p = l_p * 2^(m_p - max_p m_p).
 //
-// One CTA of kReduceWarps warps per (sequence, query head): the weights are
-// computed once per partition into shared memory, then each warp sums a
-// strided subset of the partitions with float4 loads (lane l owns channels
-// 4l .. 4l+3) and the warps' sums are added in shared memory.
+// A CTA has kReduceWarps warps; WPR warps merge one (sequence, query head)
+// row, so a CTA covers kReduceWarps / WPR rows (the host picks WPR from the
+// number of partials: few partials, several rows per CTA; many partials,
+// several warps per row). Within a warp, lanes read 32 partials' (max, sum)
+// at a time for the global max, then the warp walks its share of the
+// partials: lane l owns channels 4l .. 4l+3 (float4 loads of the partial
+// outputs); the WPR warps' sums are added in shared memory.
 constexpr int kReduceWarps = 8;
-constexpr int kReduceChunk = 1024;  // partitions weighted per pass
 
-template <typename TQ, int D>
+template <typename TQ, int D, int WPR>
 __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p) {
   static_assert(D % 4 == 0 && D <= 128, "one float4 per lane");
-  constexpr int NT = kReduceWarps * 32;
-  const int hq = blockIdx.x;
-  const int b = blockIdx.y;
+  static_assert(kReduceWarps % WPR == 0, "whole rows per CTA");
+  constexpr int RPC = kReduceWarps / WPR;  // rows per CTA
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  int L = p.context_lens[b];
-  const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
-  const int cap = static_cast<int>(table_cap < p.max_context ? table_cap : p.max_context);
-  L = L < 0 ? 0 : (L > cap ? cap : L);
-  const int nparts = (L + p.partition_tokens - 1) / p.partition_tokens;
-  if (nparts <= 1) return;
-  const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq;
-  const float2* ml = p.ws_ml + bh * p.num_partitions;
-  const float4* po = reinterpret_cast<const float4*>(p.ws_o + bh * p.num_partitions * D);
+  const int rloc = warp / WPR;
+  const int wsub = warp - rloc * WPR;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + rloc;  // b * Hq + head
+  const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
 
-  __shared__ float s_w[kReduceChunk];
-  __shared__ float s_red[kReduceWarps];
   __shared__ float4 s_acc[kReduceWarps][D / 4];
   __shared__ float s_wsum[kReduceWarps];
 
-  // max over partitions
-  float M = -INFINITY;
-  for (int i = threadIdx.x; i < nparts; i += NT) M = fmaxf(M, ml[i].x);
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) s_red[warp] = M;
-  __syncthreads();
-  M = s_red[0];
-#pragma unroll
-  for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, s_red[w]);
-
+  int nparts = 0;
+  if (row < rows) {
+    const int b = static_cast<int>(row / p.num_q_heads);
+    nparts = p.part_offset + suffix_partitions(p, clamp_context(p, p.context_lens[b]));
+  }
+  const bool work = nparts > 1 || (nparts == 1 && p.force_partials);
   const bool active = lane < D / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  for (int base = 0; base < nparts; base += kReduceChunk) {
-    const int n = min(kReduceChunk, nparts - base);
-    __syncthreads();  // previous chunk's weights consumed
-    for (int i = threadIdx.x; i < n; i += NT) {
-      const float2 v = ml[base + i];
-      s_w[i] = v.y * ex2(v.x - M);
-    }
-    __syncthreads();
+  if (work) {
+    const float2* ml = p.ws_ml + row * p.num_partitions;
+    const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
+    // global max over the row's partials (every warp of the row computes it)
+    float M = -INFINITY;
+    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    // this warp's partials: wsub, wsub + WPR, ...
 #pragma unroll 8
-    for (int i = warp; i < n; i += kReduceWarps) {
-      const float w = s_w[i];
+    for (int i = wsub; i < nparts; i += WPR) {
+      const float2 v = ml[i];  // the same address in every lane: one broadcast load
+      const float w = v.y * ex2(v.x - M);
       wsum += w;
       if (active) {
-        const float4 v = po[static_cast<int64_t>(base + i) * (D / 4) + lane];
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+        const float4 x = po[static_cast<int64_t>(i) * (D / 4) + lane];
+        acc.x += w * x.x;
+        acc.y += w * x.y;
+        acc.z += w * x.z;
+        acc.w += w * x.w;
       }
     }
+  }
+  if (WPR == 1) {
+    if (work && active) {
+      TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
+      const float inv = 1.f / wsum;
+      out[0] = from_f32<TQ>(acc.x * inv);
+      out[1] = from_f32<TQ>(acc.y * inv);
+      out[2] = from_f32<TQ>(acc.z * inv);
+      out[3] = from_f32<TQ>(acc.w * inv);
+    }
+    return;
   }
   if (active) s_acc[warp][lane] = acc;
   if (lane == 0) s_wsum[warp] = wsum;
   __syncthreads();
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
-    float a = 0.f, ws = 0.f;
+  if (work && wsub == 0 && active) {
+    float4 a = s_acc[warp][lane];
+    float ws = s_wsum[warp];
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) {
-      a += reinterpret_cast<const float*>(&s_acc[w][0])[c];
-      ws += s_wsum[w];
+    for (int k = 1; k < WPR; ++k) {
+      const float4 b4 = s_acc[warp + k][lane];
+      a.x += b4.x;
+      a.y += b4.y;
+      a.z += b4.z;
+      a.w += b4.w;
+      ws += s_wsum[warp + k];
     }
-    reinterpret_cast<TQ*>(p.out)[bh * D + c] = from_f32<TQ>(a / ws);
+    TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
+    const float inv = 1.f / ws;
+    out[0] = from_f32<TQ>(a.x * inv);
+    out[1] = from_f32<TQ>(a.y * inv);
+    out[2] = from_f32<TQ>(a.z * inv);
+    out[3] = from_f32<TQ>(a.w * inv);
   }
 }
 

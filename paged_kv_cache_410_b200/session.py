@@ -32,11 +32,16 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
 
 
 class DecodeStep:
-    def __init__(self, w, device="cuda", partition_tokens: int = 0, stream=None):
+    """`shared_prefix_blocks` > 0 decodes through pa_decode_shared_prefix (the
+    workload's tables must all start with those blocks)."""
+
+    def __init__(self, w, device="cuda", partition_tokens: int = 0, stream=None,
+                 shared_prefix_blocks: int = 0):
         self.w = w
         self.device = torch.device(device)
         self.stream = stream
         self.partition_tokens = partition_tokens
+        self.shared_prefix_blocks = shared_prefix_blocks
         dev = self.device
         cshape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         if w.cache_dtype == "e4m3":
@@ -63,8 +68,13 @@ class DecodeStep:
         self.out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=self.q.dtype,
                                device=dev)
         self.max_context = w.max_context
-        ws = B.pa_decode_workspace_size(w.batch, w.num_q_heads, self.max_context, self.cache,
-                                        partition_tokens)
+        if shared_prefix_blocks:
+            ws = B.pa_decode_shared_prefix_workspace_size(w.batch, w.num_q_heads,
+                                                          self.max_context, shared_prefix_blocks,
+                                                          self.cache, partition_tokens)
+        else:
+            ws = B.pa_decode_workspace_size(w.batch, w.num_q_heads, self.max_context,
+                                            self.cache, partition_tokens)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
         if w.cache_dtype == "e4m3" and w.fill_slots is not None and len(w.fill_slots):
             # history tokens are quantised into the pool by the library's append
@@ -84,6 +94,12 @@ class DecodeStep:
                        self.cache, self.stream)
 
     def decode(self):
+        if self.shared_prefix_blocks:
+            B.pa_decode_shared_prefix(self.q, self.k_cache, self.v_cache, self.block_tables,
+                                      self.context_lens, float(self.w.scale), self.out,
+                                      self.cache, self.max_context, self.shared_prefix_blocks,
+                                      self.partition_tokens, self.workspace, self.stream)
+            return
         B.pa_decode(self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                     float(self.w.scale), self.out, self.cache, self.max_context,
                     self.partition_tokens, self.workspace, self.stream)

@@ -230,7 +230,7 @@ def llama2_70b_prefix(batch=128, prefix_len=2000, max_suffix=2048, block_size=16
                          BS=block_size, NB=NB, dtype="bf16", lens=lens,
                          block_lists=block_lists,
                          meta={"prefix_len": prefix_len, "prefix_blocks": prefix_blocks,
-                               "refcount": batch})
+                               "shared_prefix_blocks": npre, "refcount": batch})
 
 
 def long_context(batch=1, context_len=131072, block_size=16, headroom=0.10,
@@ -360,8 +360,36 @@ def custom(lens, num_q_heads=8, num_kv_heads=8, head_dim=64, block_size=16, dtyp
                          block_lists=block_lists, meta={})
 
 
+def custom_shared_prefix(prefix_len, suffix_lens, num_q_heads=8, num_kv_heads=2, head_dim=64,
+                         block_size=16, dtype="f16", headroom=0.25, seed=SEED_BASE + 7):
+    """Sequences that all reference the same physical blocks for their first
+    ``prefix_len`` tokens (a multiple of the block size), followed by
+    ``suffix_lens[b]`` private tokens; the last suffix token is the one
+    appended this step. A suffix of 0 appends nothing (slot -1): such a
+    sequence ends exactly at the prefix."""
+    if prefix_len % block_size:
+        raise ValueError("the shared prefix must end on a block boundary")
+    rng = np.random.default_rng(seed)
+    suffix = np.asarray(suffix_lens, dtype=np.int64)
+    lens = prefix_len + suffix
+    npre = prefix_len // block_size
+    private = [-(-int(L) // block_size) - npre for L in lens]
+    NB = max(_pool_size(npre + sum(private), headroom), 1)
+    placer = _Placer(rng, NB)
+    prefix_blocks = placer.take(npre)
+    block_lists = [prefix_blocks + placer.take(p) for p in private]
+    w = _finish_16bit("custom_shared_prefix", rng, B=len(lens), Hq=num_q_heads,
+                      Hkv=num_kv_heads, D=head_dim, BS=block_size, NB=NB, dtype=dtype, lens=lens,
+                      block_lists=block_lists,
+                      meta={"prefix_len": prefix_len, "prefix_blocks": prefix_blocks,
+                            "shared_prefix_blocks": npre})
+    w.slot_mapping[suffix == 0] = -1
+    return w
+
+
 FAMILIES = {
     "custom": custom,
+    "custom_shared_prefix": custom_shared_prefix,
     "tiny_mha": tiny_mha,
     "llama2_7b": llama2_7b,
     "llama2_70b_prefix": llama2_70b_prefix,

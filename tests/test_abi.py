@@ -101,6 +101,33 @@ def test_decode_argument_checks(lib):
                          FAKE, 0, None, 0, None) == 1
 
 
+def test_shared_prefix_argument_checks(lib):
+    d = _desc()
+    call = lambda **kw: lib.pa_decode_shared_prefix(*[kw.get(k, v) for k, v in [
+        ("q", FAKE), ("q_dtype", 0), ("batch", 2), ("hq", 4), ("k", FAKE), ("v", FAKE),
+        ("desc", ctypes.byref(d)), ("bt", FAKE), ("mb", 4), ("lens", FAKE), ("maxc", 64),
+        ("pb", 2), ("scale", 0.1), ("out", FAKE), ("pt", 0), ("ws", None), ("wsb", 0),
+        ("s", None)]])
+    assert call(pb=5) == 1               # more shared blocks than table columns
+    assert call(pb=-1) == 1
+    assert call(pb=4, maxc=60) == 1      # prefix longer than max_context
+    assert call() == 4                   # a cascade always needs a workspace
+    need = lib.pa_decode_shared_prefix_workspace_size(2, 4, 64, 2, 0, ctypes.byref(d))
+    assert need > 0
+    assert call(ws=FAKE, wsb=need - 1) == 4
+    assert call(batch=0) == 0
+    # no shared blocks: the plain decode's workspace
+    assert (lib.pa_decode_shared_prefix_workspace_size(2, 4, 5000, 0, 64, ctypes.byref(d)) ==
+            lib.pa_decode_workspace_size(2, 4, 5000, 64, ctypes.byref(d)))
+    # partials: prefix chunks (up to 512 tokens each) + suffix partitions
+    ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 2048 + 256, 128, 64, ctypes.byref(d))
+    parts = 4 + 4
+    assert ws == -(-(3 * 4 * parts * 64 * 4) // 256) * 256 + -(-(3 * 4 * parts * 8) // 256) * 256
+    ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 8192 + 64, 512, 64, ctypes.byref(d))
+    parts = 16 + 1
+    assert ws == -(-(3 * 4 * parts * 64 * 4) // 256) * 256 + -(-(3 * 4 * parts * 8) // 256) * 256
+
+
 def test_append_argument_checks(lib):
     d = _desc()
     assert lib.pa_append_kv(FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, ctypes.byref(d), None) == 2

@@ -36,10 +36,14 @@ def sample(w, n, seed=0):
     return np.array(sorted(list(must) + rest[:max(0, n - len(must))]))
 
 
-@pytest.mark.parametrize("name,kw,n", FULL, ids=[f"{n}-{k}" for n, k, _ in FULL])
+@pytest.mark.parametrize("name,kw,n", FULL + [("llama2_70b_prefix", {"cascade": True}, 8)],
+                         ids=[f"{n}-{k}" for n, k, _ in FULL] + ["llama2_70b_prefix-cascade"])
 def test_full_size_step(name, kw, n):
+    kw = dict(kw)
+    cascade = kw.pop("cascade", False)
     w = W.make(name, **kw)
-    step = DecodeStep(w, "cuda")
+    step = DecodeStep(w, "cuda",
+                      shared_prefix_blocks=w.meta["shared_prefix_blocks"] if cascade else 0)
     step.run()
     torch.cuda.synchronize()
     assert step.device_errors() == 0
