@@ -187,9 +187,10 @@ __device__ __forceinline__ int2 accumulator_channels(int mt, int g) {
 }
 
 // One 16-token tile of K and V in shared memory (rows >= nvalid are zero and
-// masked) against the warp's query columns: S^T = K Q^T, online softmax
-// update of the per-column running max / sum (log2 domain), O^T += V^T P^T.
-template <int CK, int D, int NH>
+// masked; FULL: all 16 rows exist) against the warp's query columns:
+// S^T = K Q^T, online softmax update of the per-column running max / sum
+// (log2 domain), O^T += V^T P^T.
+template <int CK, int D, int NH, bool FULL>
 __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nvalid,
                                             float scale_log2,
                                             const uint32_t (&qb)[D / 16][NH][2],
@@ -242,9 +243,10 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
   }
 
   // online softmax per column; the max is reduced over the 16 tokens
-  // (lanes with the same t, both row halves)
-  const bool va = g < nvalid;
-  const bool vb = g + 8 < nvalid;
+  // (lanes with the same t, both row halves) on the raw scores (the scale is
+  // positive), and each exponent is one FFMA: s * scale_log2 - m_ref
+  const bool va = FULL || g < nvalid;
+  const bool vb = FULL || g + 8 < nvalid;
   uint32_t pb[NH][2];
   bool grew = false;
   float alpha[NH][2];
@@ -253,20 +255,21 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
     float pr[2][2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const float x0 = va ? s[nh][e] * scale_log2 : -INFINITY;
-      const float x1 = vb ? s[nh][2 + e] * scale_log2 : -INFINITY;
-      float mx = fmaxf(x0, x1);
+      float mx = fmaxf(va ? s[nh][e] : -INFINITY, vb ? s[nh][2 + e] : -INFINITY);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      mx *= scale_log2;
       // mx is finite (token 0 of the tile exists), so the first tile always
       // sets the reference
       const bool up = mx > m_run[nh][e] + kRescaleLog2;
       grew |= up;
       const float m_ref = up ? mx : m_run[nh][e];
       alpha[nh][e] = up ? ex2(m_run[nh][e] - m_ref) : 1.f;  // exactly 1 when unchanged
-      pr[0][e] = ex2(x0 - m_ref);
-      pr[1][e] = ex2(x1 - m_ref);
+      const float p0 = ex2(fmaf(s[nh][e], scale_log2, -m_ref));
+      const float p1 = ex2(fmaf(s[nh][2 + e], scale_log2, -m_ref));
+      pr[0][e] = va ? p0 : 0.f;
+      pr[1][e] = vb ? p1 : 0.f;
       l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + (pr[0][e] + pr[1][e]);
       m_run[nh][e] = m_ref;
     }
@@ -521,7 +524,10 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const uint32_t sv_a = sk_a + G::TB;
     const int tile = warp + it * NW;
     const int nvalid = t1 - (t0 + tile * 16);  // tokens of this tile that exist (>= 1)
-    attend_tile<CK, D, NH>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
+    if (nvalid >= 16)
+      attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
+    else
+      attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
     __syncwarp();  // this stage is reloaded by the next iteration
   }
   cp_async_wait<0>();

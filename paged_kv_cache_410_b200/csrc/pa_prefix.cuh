@@ -96,8 +96,8 @@ __device__ __forceinline__ int2 row_layout_channels(int i, int t) {
 }
 
 // One block of 16 * NSUB K/V rows against the warp's 16 query rows (row
-// layout), with one softmax round for the whole block.
-template <int CK, int D, int NSUB>
+// layout), with one softmax round for the whole block (FULL: all rows exist).
+template <int CK, int D, int NSUB, bool FULL>
 __device__ __forceinline__ void attend_block_rows(uint32_t sk_a, uint32_t sv_a, int nvalid,
                                                   float scale_log2,
                                                   const uint32_t (&qa)[D / 16][4],
@@ -148,8 +148,9 @@ __device__ __forceinline__ void attend_block_rows(uint32_t sk_a, uint32_t sv_a, 
   }
 
   // online softmax per row (log2 domain); the max is reduced over the 4
-  // threads of the row group. The reference max moves only when the block
-  // max exceeds it by more than kRescaleLog2, so P <= 2^kRescaleLog2 and the
+  // threads of the row group, on raw scores (the scale is positive), and each
+  // exponent is one FFMA. The reference max moves only when the block max
+  // exceeds it by more than kRescaleLog2, so P <= 2^kRescaleLog2 and the
   // accumulator is rarely rescaled.
   uint32_t pa[NSUB][4];
   bool grew = false;
@@ -161,13 +162,12 @@ __device__ __forceinline__ void attend_block_rows(uint32_t sk_a, uint32_t sv_a, 
     for (int n = 0; n < NS; ++n)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int tok = 8 * n + 2 * t + e;
-        const float x = tok < nvalid ? s[n][2 * rr + e] * scale_log2 : -INFINITY;
-        s[n][2 * rr + e] = x;
-        mx = fmaxf(mx, x);
+        const bool ok = FULL || 8 * n + 2 * t + e < nvalid;
+        mx = fmaxf(mx, ok ? s[n][2 * rr + e] : -INFINITY);
       }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx *= scale_log2;
     const bool up = mx > m_run[rr] + kRescaleLog2;  // the first block always moves it
     grew |= up;
     const float m_ref = up ? mx : m_run[rr];
@@ -175,8 +175,12 @@ __device__ __forceinline__ void attend_block_rows(uint32_t sk_a, uint32_t sv_a, 
     float sum = 0.f;
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
-      const float p0 = ex2(s[n][2 * rr] - m_ref);
-      const float p1 = ex2(s[n][2 * rr + 1] - m_ref);
+      float p0 = ex2(fmaf(s[n][2 * rr], scale_log2, -m_ref));
+      float p1 = ex2(fmaf(s[n][2 * rr + 1], scale_log2, -m_ref));
+      if constexpr (!FULL) {
+        p0 = 8 * n + 2 * t < nvalid ? p0 : 0.f;
+        p1 = 8 * n + 2 * t + 1 < nvalid ? p1 : 0.f;
+      }
       sum += p0 + p1;
       // A fragment of k-step n/2: rows g (rr=0) / g+8 (rr=1), tokens 2t,2t+1 (+8)
       pa[n >> 1][rr + 2 * (n & 1)] = pack2<kMmaBF16>(p0, p1);
@@ -355,8 +359,13 @@ __device__ __forceinline__ void prefix_cta(const DecodeParams& p, const int chun
     cp_async_wait<NSP - 1>();
     __syncthreads();  // tile `it` landed for every thread's copies
     const uint32_t sk_a = smem_addr(smem + (it % NSP) * S::kStageBytes);
-    attend_block_rows<CK, D, NSUB>(sk_a, sk_a + S::kKBytes, c1 - (c0 + it * BT), p.scale_log2,
-                                   qa, qalo, o, m_run, l_run);
+    const int nvalid = c1 - (c0 + it * BT);
+    if (nvalid >= BT)
+      attend_block_rows<CK, D, NSUB, true>(sk_a, sk_a + S::kKBytes, nvalid, p.scale_log2, qa,
+                                           qalo, o, m_run, l_run);
+    else
+      attend_block_rows<CK, D, NSUB, false>(sk_a, sk_a + S::kKBytes, nvalid, p.scale_log2, qa,
+                                            qalo, o, m_run, l_run);
     __syncthreads();  // every warp is done with the stage before it is refilled
   }
   cp_async_wait<0>();
@@ -407,9 +416,11 @@ struct CascadeGrid {
   int n_suffix_parts;
 };
 
+// Three CTAs per SM (the decode CTAs' shared-memory limit) for 16-bit caches;
+// two for E4M3, whose hi + lo query fragments need more registers.
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, int NWP, int NSP>
-__global__ void __launch_bounds__(NW * 32) pa_cascade_kernel(const DecodeParams p,
-                                                               const CascadeGrid cg) {
+__global__ void __launch_bounds__(NW * 32, CK == kE4M3 ? 2 : 3)
+    pa_cascade_kernel(const DecodeParams p, const CascadeGrid cg) {
   static_assert(NW == NWP, "one block size for both kinds of CTA");
   const int bid = blockIdx.x;
   const int j = bid / (cg.ratio + 1);
