@@ -64,7 +64,7 @@ def _load():
         lib.oracle_copy_blocks.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [P, ctypes.c_int, i32, i32, P, P, ctypes.c_int, i64,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, i32, P,
-                                      f32, P]
+                                      f32, i32, P]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -163,9 +163,9 @@ def copy_blocks(pairs, k_cache, v_cache, cache_dtype):
 
 
 def decode(q, q_dtype, k_cache, v_cache, cache_dtype, block_tables, context_lens, scale,
-           k_scale=None, v_scale=None) -> np.ndarray:
+           k_scale=None, v_scale=None, window=0) -> np.ndarray:
     """Float64 attention output [B, Hq, D] of one query per sequence over its
-    paged history."""
+    paged history (its last `window` tokens when window > 0)."""
     lib = _load()
     q = _c(q, np.uint16)
     block_tables = _c(block_tables, np.int32)
@@ -181,6 +181,6 @@ def decode(q, q_dtype, k_cache, v_cache, cache_dtype, block_tables, context_lens
     rc = lib.oracle_decode(_ptr(q), DTYPES[q_dtype], b, hq, _ptr(kc), _ptr(vc),
                            DTYPES[cache_dtype], nb, bs, hkv, d, _ptr(ks), _ptr(vs),
                            _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-                           float(np.float32(scale)), _ptr(out))
+                           float(np.float32(scale)), int(window), _ptr(out))
     _check(rc, "oracle_decode")
     return out

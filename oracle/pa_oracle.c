@@ -224,13 +224,17 @@ int oracle_copy_blocks(const int32_t* pairs, int32_t num_pairs, void* k_cache, v
  *  2. s_j = scale * sum_c q[c] * Kc[j][c];
  *  3. m = max_j s_j, w_j = exp(s_j - m) (subtracting m leaves the softmax
  *     unchanged), o = sum_j w_j Vc[j] / sum_j w_j.
+ * Sliding window ([KVA] section "再往后：压 KV 的三条路线", second route: each
+ * token attends only to the most recent window of tokens): with window > 0
+ * the sums run over j in [max(0, L - window), L) -- the window counts the
+ * new token itself -- and window == 0 means the whole history.
  * out: [B][Hq][D] doubles. */
 int oracle_decode(const void* q, int q_dtype, int32_t batch, int32_t num_q_heads,
                   const void* k_cache, const void* v_cache, int cache_dtype, int64_t num_blocks,
                   int block_size, int num_kv_heads, int head_dim, const float* k_scale,
                   const float* v_scale, const int32_t* block_tables,
                   int32_t max_blocks_per_seq, const int32_t* context_lens, float scale,
-                  double* out) {
+                  int32_t window, double* out) {
   if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return OR_ERR_ARG;
   if (cache_dtype == OR_E4M3 && (!k_scale || !v_scale)) return OR_ERR_ARG;
   const int group = num_q_heads / num_kv_heads;
@@ -252,12 +256,15 @@ int oracle_decode(const void* q, int q_dtype, int32_t batch, int32_t num_q_heads
     for (int32_t i = 0; i < num_q_heads; ++i) {
       const int h = i / group;
       const int32_t L = context_lens[b];
+      /* attended tokens: [j0, L), n of them */
+      const int32_t j0 = (window > 0 && L > window) ? L - window : 0;
+      const int32_t n = L - j0;
       double* o = out + ((int64_t)b * num_q_heads + i) * D;
       for (int c = 0; c < D; ++c) o[c] = 0.0;
-      if (L == 0) continue;
-      double* Kc = (double*)malloc(sizeof(double) * (size_t)L * D);
-      double* Vc = (double*)malloc(sizeof(double) * (size_t)L * D);
-      double* s = (double*)malloc(sizeof(double) * (size_t)L);
+      if (n == 0) continue;
+      double* Kc = (double*)malloc(sizeof(double) * (size_t)n * D);
+      double* Vc = (double*)malloc(sizeof(double) * (size_t)n * D);
+      double* s = (double*)malloc(sizeof(double) * (size_t)n);
       double* qd = (double*)malloc(sizeof(double) * (size_t)D);
       if (!Kc || !Vc || !s || !qd) {
 #pragma omp atomic write
@@ -269,7 +276,8 @@ int oracle_decode(const void* q, int q_dtype, int32_t batch, int32_t num_q_heads
         continue;
       }
       /* step 1: gather through the block table */
-      for (int32_t j = 0; j < L; ++j) {
+      for (int32_t k = 0; k < n; ++k) {
+        const int32_t j = j0 + k;
         int64_t blk = block_tables[(int64_t)b * max_blocks_per_seq + j / block_size];
         int64_t r = j % block_size;
         int64_t base = ((blk * block_size + r) * num_kv_heads + h) * D;
@@ -280,29 +288,29 @@ int oracle_decode(const void* q, int q_dtype, int32_t batch, int32_t num_q_heads
             kv *= (double)k_scale[h * D + c];
             vv *= (double)v_scale[h * D + c];
           }
-          Kc[(int64_t)j * D + c] = kv;
-          Vc[(int64_t)j * D + c] = vv;
+          Kc[(int64_t)k * D + c] = kv;
+          Vc[(int64_t)k * D + c] = vv;
         }
       }
       for (int c = 0; c < D; ++c)
         qd[c] = load_elem(q, ((int64_t)b * num_q_heads + i) * D + c, q_dtype);
       /* step 2: scores */
-      for (int32_t j = 0; j < L; ++j) {
+      for (int32_t k = 0; k < n; ++k) {
         double dot = 0.0;
-        for (int c = 0; c < D; ++c) dot += qd[c] * Kc[(int64_t)j * D + c];
-        s[j] = (double)scale * dot;
+        for (int c = 0; c < D; ++c) dot += qd[c] * Kc[(int64_t)k * D + c];
+        s[k] = (double)scale * dot;
       }
       /* step 3: softmax-weighted sum of values */
       double m = s[0];
-      for (int32_t j = 1; j < L; ++j)
-        if (s[j] > m) m = s[j];
+      for (int32_t k = 1; k < n; ++k)
+        if (s[k] > m) m = s[k];
       double denom = 0.0;
-      for (int32_t j = 0; j < L; ++j) {
-        s[j] = exp(s[j] - m);
-        denom += s[j];
+      for (int32_t k = 0; k < n; ++k) {
+        s[k] = exp(s[k] - m);
+        denom += s[k];
       }
-      for (int32_t j = 0; j < L; ++j)
-        for (int c = 0; c < D; ++c) o[c] += s[j] * Vc[(int64_t)j * D + c];
+      for (int32_t k = 0; k < n; ++k)
+        for (int c = 0; c < D; ++c) o[c] += s[k] * Vc[(int64_t)k * D + c];
       for (int c = 0; c < D; ++c) o[c] /= denom;
       free(Kc);
       free(Vc);

@@ -299,3 +299,49 @@ def test_empty_context_gives_zeros_and_bad_block_ids_are_rejected(oracle_mod):
     bad[1, 1] = kp.shape[0]
     with pytest.raises(oracle_mod.OracleError):
         oracle_mod.decode(q, "f16", kp, vp, "f16", bad, np.array([5, 20], np.int32), 0.5)
+
+
+# ---- sliding window (KV cache article, section '再往后：压 KV 的三条路线':
+# each token attends only to the most recent window of tokens) ------------------
+
+def test_window_at_least_the_length_changes_nothing(oracle_mod):
+    rng = np.random.default_rng(30)
+    lens = [1, 16, 37, 100]
+    q, ks, vs, kp, vp, tab = _case(rng, 4, 8, 2, 64, 16, lens, "f16")
+    L = np.array(lens, np.int32)
+    full = oracle_mod.decode(q, "f16", kp, vp, "f16", tab, L, 0.125)
+    for w in (100, 101, 5000):
+        assert np.array_equal(oracle_mod.decode(q, "f16", kp, vp, "f16", tab, L, 0.125,
+                                                window=w), full)
+
+
+def test_window_of_one_returns_the_newest_value(oracle_mod):
+    rng = np.random.default_rng(31)
+    lens = [1, 9, 40]
+    q, ks, vs, kp, vp, tab = _case(rng, 3, 4, 4, 32, 16, lens, "f16")
+    got = oracle_mod.decode(q, "f16", kp, vp, "f16", tab, np.array(lens, np.int32), 0.3,
+                            window=1)
+    for b, L in enumerate(lens):
+        assert np.array_equal(got[b], vs[b][L - 1].view(np.float16).astype(np.float64))
+
+
+@pytest.mark.parametrize("window", [2, 15, 16, 17, 33])
+def test_window_equals_attention_over_the_last_tokens(oracle_mod, window):
+    rng = np.random.default_rng(32 + window)
+    hq, hkv, d, bs = 8, 2, 64, 16
+    lens = [3, 16, 50, 129]
+    q, ks, vs, kp, vp, tab = _case(rng, len(lens), hq, hkv, d, bs, lens, "bf16")
+    scale = np.float32(0.2)
+    got = oracle_mod.decode(q, "bf16", kp, vp, "bf16", tab, np.array(lens, np.int32), scale,
+                            window=window)
+    # the same tokens laid out afresh as whole sequences of their own
+    ks_t = [k[max(0, L - window):] for k, L in zip(ks, lens)]
+    vs_t = [v[max(0, L - window):] for v, L in zip(vs, lens)]
+    nb = sum(-(-len(k) // bs) for k in ks_t) + 3
+    perm = rng.permutation(nb)
+    kp2, tab2 = scatter(ks_t, bs, nb, rng, hkv, d, "bf16", perm=perm)
+    vp2, _ = scatter(vs_t, bs, nb, rng, hkv, d, "bf16", perm=perm)
+    short = oracle_mod.decode(q, "bf16", kp2, vp2, "bf16", tab2,
+                              np.array([len(k) for k in ks_t], np.int32), scale)
+    assert np.array_equal(got, short)
+    np.testing.assert_allclose(got, sdpa_ref(q, ks_t, vs_t, scale, "bf16"), rtol=0, atol=1e-12)
