@@ -306,10 +306,19 @@ def run_ours(args):
 
     w = make_workload(args.workload, rank, args.batch)
     spb = w.meta.get("shared_prefix_blocks", 0) if args.cascade == "auto" else 0
-    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb)
+    if args.window:
+        spb = 0
+    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb,
+                      window=args.window)
     stream = torch.cuda.current_stream(dev)
-    sb = A.step_bytes(w)
-    if spb:
+    sb = A.step_bytes(w, window=args.window)
+    if args.window:
+        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
+            w.batch, min(w.max_context, args.window + 15), step.cache)
+        n_parts = max(1, math.ceil(min(w.max_context, args.window + 15) / plan_pt))
+        decode_launches = 1 + (1 if n_parts > 1 else 0)
+        decode_name = f"pa_decode_sliding_window (window {args.window}; main + split-K reduce)"
+    elif spb:
         prefix_len = spb * w.block_size
         plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
             w.batch, max(w.max_context - prefix_len, 0), step.cache)
@@ -442,6 +451,8 @@ def main(argv=None):
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding-window decode over the last WINDOW tokens (0: whole history)")
     ap.add_argument("--cascade", choices=["auto", "off"], default="auto",
                     help="decode a workload whose sequences share prefix blocks through "
                          "pa_decode_shared_prefix (auto) or plain pa_decode (off)")

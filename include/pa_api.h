@@ -141,6 +141,30 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* Workspace bytes for pa_decode_sliding_window. Pure host function. */
+size_t pa_decode_sliding_window_workspace_size(int32_t batch, int32_t num_q_heads,
+                                               int32_t max_context, int32_t window,
+                                               int32_t partition_tokens,
+                                               const pa_cache_desc* cache);
+
+/* pa_decode with sliding-window attention (KV cache article, section
+ * "再往后：压 KV 的三条路线": each token attends only to the most recent window
+ * of tokens, so the cache a sequence needs is bounded by the window): the
+ * query of sequence b attends to its tokens [max(0, L - window), L), L =
+ * context_lens[b], the new token included.
+ *   window  >= 1 tokens.
+ * Table entries for blocks that hold only tokens before the window are never
+ * read, so a caller may have freed those blocks (their entries may hold any
+ * value). Other arguments as for pa_decode; the workspace comes from
+ * pa_decode_sliding_window_workspace_size. */
+pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch,
+                                   int32_t num_q_heads, const void* k_cache, const void* v_cache,
+                                   const pa_cache_desc* cache, const int32_t* block_tables,
+                                   int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                   int32_t max_context, int32_t window, float scale, void* out,
+                                   int32_t partition_tokens, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Workspace bytes for pa_decode_shared_prefix (equals
  * pa_decode_workspace_size when prefix_blocks == 0). Pure host function. */
 size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads,

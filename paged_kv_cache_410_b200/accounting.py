@@ -15,33 +15,37 @@ import numpy as np
 ELEM_BYTES = {"f16": 2, "bf16": 2, "e4m3": 1}
 
 
-def _unique_slots(w) -> int:
-    """Distinct physical (block, row) slots read by all sequences: rows of a
-    block are filled from row 0, so a block contributes the largest row count
-    any sequence uses in it."""
-    rows = np.zeros(w.num_blocks, dtype=np.int64)
+def _attended(w, window: int):
+    """Per sequence, the first attended token and the count."""
+    lens = w.context_lens.astype(np.int64)
+    lo = np.maximum(lens - window, 0) if window > 0 else np.zeros_like(lens)
+    return lo, lens - lo
+
+
+def _unique_slots(w, window: int = 0) -> int:
+    """Distinct physical (block, row) slots read by all sequences."""
     bs = w.block_size
+    lo, n = _attended(w, window)
+    seen = np.zeros(w.num_blocks * bs, dtype=bool)
     for b in range(w.batch):
-        L = int(w.context_lens[b])
-        if L <= 0:
+        if n[b] <= 0:
             continue
-        n = -(-L // bs)
-        blocks = w.block_tables[b, :n].astype(np.int64)
-        used = np.full(n, bs, dtype=np.int64)
-        used[-1] = L - (n - 1) * bs
-        np.maximum.at(rows, blocks, used)
-    return int(rows.sum())
+        j = np.arange(lo[b], lo[b] + n[b], dtype=np.int64)
+        seen[w.block_tables[b, j // bs].astype(np.int64) * bs + j % bs] = True
+    return int(seen.sum())
 
 
-def decode_bytes(w) -> dict:
+def decode_bytes(w, window: int = 0) -> dict:
+    """`window` > 0: each sequence reads only its last `window` tokens."""
     eb = ELEM_BYTES[w.cache_dtype]
     io = ELEM_BYTES[w.io_dtype]
     per_token = 2 * w.num_kv_heads * w.head_dim * eb  # K and V of one token, one layer
-    lens = w.context_lens.astype(np.int64)
-    kv_logical = int(per_token * lens.sum())
-    kv_unique = int(per_token * _unique_slots(w))
+    lo, n = _attended(w, window)
+    kv_logical = int(per_token * n.sum())
+    kv_unique = int(per_token * _unique_slots(w, window))
     qo = 2 * w.batch * w.num_q_heads * w.head_dim * io
-    tables = int(4 * np.sum(-(-lens // w.block_size)))
+    bs = w.block_size
+    tables = int(4 * np.sum(np.where(n > 0, (lo + n - 1) // bs - lo // bs + 1, 0)))
     other = qo + tables + 4 * w.batch
     if w.cache_dtype == "e4m3":
         other += 2 * w.num_kv_heads * w.head_dim * 4
@@ -64,8 +68,8 @@ def copy_bytes(w) -> int:
     return int(len(w.copy_pairs) * block * 2 * 2)
 
 
-def step_bytes(w) -> dict:
-    d = decode_bytes(w)
+def step_bytes(w, window: int = 0) -> dict:
+    d = decode_bytes(w, window)
     a = append_bytes(w)
     c = copy_bytes(w)
     return {"decode": d["total_unique"], "decode_logical": d["total_logical"],

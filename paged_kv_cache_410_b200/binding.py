@@ -28,7 +28,8 @@ DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_PREFIX = 0x1, 0x2, 0x4,
 EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tokens",
             "pa_decode", "pa_copy_blocks", "pa_get_device_error", "pa_status_string",
             "pa_version", "pa_decode_static_workspace",
-            "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix"]
+            "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
+            "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -84,6 +85,11 @@ def load_library(path: str = LIB_PATH):
     lib.pa_decode_shared_prefix.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, i32,
                                             ctypes.c_float, P, i32, P, ctypes.c_size_t, P]
     lib.pa_decode_shared_prefix.restype = ctypes.c_int
+    lib.pa_decode_sliding_window_workspace_size.argtypes = [i32, i32, i32, i32, i32, D]
+    lib.pa_decode_sliding_window_workspace_size.restype = ctypes.c_size_t
+    lib.pa_decode_sliding_window.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, i32,
+                                             ctypes.c_float, P, i32, P, ctypes.c_size_t, P]
+    lib.pa_decode_sliding_window.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -204,6 +210,32 @@ def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, sca
                                      int(partition_tokens), _ptr(workspace), ws_bytes,
                                      _stream(stream))
     _check(rc, "pa_decode_shared_prefix")
+
+
+def pa_decode_sliding_window_workspace_size(batch, num_q_heads, max_context, window,
+                                            cache: PagedCache, partition_tokens=0) -> int:
+    lib = load_library()
+    d = cache.desc()
+    return int(lib.pa_decode_sliding_window_workspace_size(batch, num_q_heads, max_context,
+                                                           window, partition_tokens,
+                                                           ctypes.byref(d)))
+
+
+def pa_decode_sliding_window(q, k_cache, v_cache, block_tables, context_lens, scale, out,
+                             cache: PagedCache, max_context: int, window: int,
+                             partition_tokens: int = 0, workspace=None, stream=None):
+    """pa_decode attending only to each sequence's last `window` tokens."""
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.pa_decode_sliding_window(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache),
+                                      _ptr(v_cache), ctypes.byref(d), _ptr(block_tables),
+                                      block_tables.shape[1], _ptr(context_lens),
+                                      int(max_context), int(window), float(scale), _ptr(out),
+                                      int(partition_tokens), _ptr(workspace), ws_bytes,
+                                      _stream(stream))
+    _check(rc, "pa_decode_sliding_window")
 
 
 def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, scale, out,

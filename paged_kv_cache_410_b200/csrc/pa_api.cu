@@ -81,7 +81,10 @@ struct Plan {
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int partition_tokens,
-               const pa_cache_desc* cd) {
+               const pa_cache_desc* cd, int window = 0) {
+  // with a sliding window a sequence spans at most window + 15 tokens from
+  // its first (16-aligned) partition start
+  if (window > 0) max_context = std::min<int64_t>(max_context, window + 15);
   Plan pl{};
   pl.partition_tokens = partition_tokens > 0
                             ? partition_tokens
@@ -421,6 +424,50 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                 : nullptr;
   p.partition_tokens = pl.partition_tokens;
   p.num_partitions = pl.num_partitions;
+  return launch_decode(p, q_dtype, cache, as_stream(stream));
+}
+
+size_t pa_decode_sliding_window_workspace_size(int32_t batch, int32_t num_q_heads,
+                                               int32_t max_context, int32_t window,
+                                               int32_t partition_tokens,
+                                               const pa_cache_desc* cache) {
+  int bs_log2 = 0;
+  if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || num_q_heads <= 0 ||
+      max_context < 0 || partition_tokens < 0 || window <= 0)
+    return 0;
+  return make_plan(batch, num_q_heads, max_context, partition_tokens, cache, window).ws_bytes;
+}
+
+pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch,
+                                   int32_t num_q_heads, const void* k_cache, const void* v_cache,
+                                   const pa_cache_desc* cache, const int32_t* block_tables,
+                                   int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                   int32_t max_context, int32_t window, float scale, void* out,
+                                   int32_t partition_tokens, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  int bs_log2 = 0;
+  bool nothing = false;
+  pa_status st = check_decode_args(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, out, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK) return st;
+  if (window <= 0) return PA_ERR_INVALID_ARG;
+  if (nothing) return PA_OK;
+  const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache, window);
+  if (pl.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
+  }
+  pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
+                                     block_tables, max_blocks_per_seq, context_lens, max_context,
+                                     scale, out, bs_log2);
+  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
+  p.ws_ml = pl.ws_bytes
+                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
+                : nullptr;
+  p.partition_tokens = pl.partition_tokens;
+  p.num_partitions = pl.num_partitions;
+  p.window = window;
   return launch_decode(p, q_dtype, cache, as_stream(stream));
 }
 

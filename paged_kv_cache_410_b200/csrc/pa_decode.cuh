@@ -68,18 +68,42 @@ struct DecodeParams {
   int part_offset;
   int force_partials;
   int prefix_chunk_tokens;  // prefix tokens per prefix-kernel CTA (cascade mode)
+  // Sliding window (0: none): a sequence of length L attends to its tokens
+  // [L - window, L) only.
+  int window;
 };
 
-// Number of split-K partials of a sequence of length L (the prefix's ones
-// included) and the clamped length, shared by the decode and reduce kernels.
 __device__ __forceinline__ int clamp_context(const DecodeParams& p, int L) {
   const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
   const int cap = static_cast<int>(table_cap < p.max_context ? table_cap : p.max_context);
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
+
+// Tokens a CTA of this launch covers for a sequence of length L: it attends
+// to [lo, L); partitions start at `base` (lo rounded down to 16 for a sliding
+// window, so that tiles stay block aligned; the tokens in [base, lo) are
+// masked and never read).
+struct SeqSpan {
+  int lo;
+  int base;
+};
+__device__ __forceinline__ SeqSpan seq_span(const DecodeParams& p, int L) {
+  SeqSpan s;
+  s.lo = p.token_start;
+  s.base = p.token_start;
+  if (p.window > 0 && L - p.window > s.lo) {
+    s.lo = L - p.window;
+    s.base = s.lo & ~15;
+  }
+  return s;
+}
+
+// Number of split-K partials of a sequence of length L after the prefix's
+// (cascade mode) ones, shared by the decode and reduce kernels.
 __device__ __forceinline__ int suffix_partitions(const DecodeParams& p, int L) {
-  const int n = L - p.token_start;
-  return n > 0 ? (n + p.partition_tokens - 1) / p.partition_tokens : 0;
+  const SeqSpan s = seq_span(p, L);
+  const int n = L - s.base;
+  return L > s.lo ? (n + p.partition_tokens - 1) / p.partition_tokens : 0;
 }
 
 enum CacheKind { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
@@ -186,12 +210,12 @@ __device__ __forceinline__ int2 accumulator_channels(int mt, int g) {
   return make_int2((D / 8) * g + 2 * mt, (D / 8) * g + 2 * mt + 1);
 }
 
-// One 16-token tile of K and V in shared memory (rows >= nvalid are zero and
-// masked; FULL: all 16 rows exist) against the warp's query columns:
-// S^T = K Q^T, online softmax update of the per-column running max / sum
-// (log2 domain), O^T += V^T P^T.
+// One 16-token tile of K and V in shared memory (rows < nskip or >= nvalid
+// are zero and masked; FULL: all 16 rows count) against the warp's query
+// columns: S^T = K Q^T, online softmax update of the per-column running max /
+// sum (log2 domain), O^T += V^T P^T.
 template <int CK, int D, int NH, bool FULL>
-__device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nvalid,
+__device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nvalid, int nskip,
                                             float scale_log2,
                                             const uint32_t (&qb)[D / 16][NH][2],
                                             const uint32_t (&qlo)[CK == kE4M3 ? D / 16 : 1][NH][2],
@@ -245,8 +269,8 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
   // online softmax per column; the max is reduced over the 16 tokens
   // (lanes with the same t, both row halves) on the raw scores (the scale is
   // positive), and each exponent is one FFMA: s * scale_log2 - m_ref
-  const bool va = FULL || g < nvalid;
-  const bool vb = FULL || g + 8 < nvalid;
+  const bool va = FULL || (g < nvalid && g >= nskip);
+  const bool vb = FULL || (g + 8 < nvalid && g + 8 >= nskip);
   uint32_t pb[NH][2];
   bool grew = false;
   float alpha[NH][2];
@@ -396,14 +420,17 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
           from_f32<TQ>(0.f);
     return;
   }
-  const int t0 = p.token_start + part * PT;
+  const SeqSpan span = seq_span(p, L);
+  const int lo = span.lo;  // first attended token
+  const int t0 = span.base + part * PT;
   const int t1 = min(t0 + PT, L);
   const int ntiles = (t1 - t0 + 15) >> 4;
 
   // ---- block ids of this partition -> shared memory ----------------------
   // (up to kBlockIdsInSmem of them; a longer slice is read from global
-  // memory per row instead)
-  const int bt0 = t0 >> p.bs_log2;
+  // memory per row instead). Blocks before `lo` are never looked up: a
+  // sliding-window caller may have freed them.
+  const int bt0 = max(t0, lo) >> p.bs_log2;
   const int nbt = ((t1 - 1) >> p.bs_log2) - bt0 + 1;
   const bool bt_in_smem = nbt <= kBlockIdsInSmem;
   const int32_t* gbt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + bt0;
@@ -467,7 +494,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 #pragma unroll
       for (int i = 0; i < LITERS; ++i) {
         const int r = lrow + i * RPI;
-        const bool ok = blk >= 0 && tb + r < t1;
+        const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
         const int64_t off = ok ? base + static_cast<int64_t>(i * RPI) * slot_stride : 0;
         const uint32_t so = G::off(r, lch);
         cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
@@ -478,7 +505,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
       for (int i = 0; i < LITERS; ++i) {
         const int r = lrow + i * RPI;
         const int j = tb + r;
-        const int blk = j < t1 ? block_id((j >> p.bs_log2) - bt0) : -1;
+        const int blk = (j < t1 && j >= lo) ? block_id((j >> p.bs_log2) - bt0) : -1;
         const bool ok = blk >= 0;
         const int64_t off =
             ok ? ((static_cast<int64_t>(blk) << p.bs_log2) + (j & bs_mask)) * slot_stride +
@@ -523,11 +550,15 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
     const int tile = warp + it * NW;
-    const int nvalid = t1 - (t0 + tile * 16);  // tokens of this tile that exist (>= 1)
-    if (nvalid >= 16)
-      attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
+    const int ts = t0 + tile * 16;
+    const int nvalid = t1 - ts;                // rows of the tile below the end (>= 1)
+    const int nskip = max(lo - ts, 0);         // rows before the window (first tile only)
+    if (nvalid >= 16 && nskip == 0)
+      attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, 0, p.scale_log2, qb, qlo, o, m_run,
+                                   l_run);
     else
-      attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, p.scale_log2, qb, qlo, o, m_run, l_run);
+      attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, nskip, p.scale_log2, qb, qlo, o, m_run,
+                                    l_run);
     __syncwarp();  // this stage is reloaded by the next iteration
   }
   cp_async_wait<0>();

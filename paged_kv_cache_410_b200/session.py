@@ -33,15 +33,19 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
 
 class DecodeStep:
     """`shared_prefix_blocks` > 0 decodes through pa_decode_shared_prefix (the
-    workload's tables must all start with those blocks)."""
+    workload's tables must all start with those blocks); `window` > 0 through
+    pa_decode_sliding_window."""
 
     def __init__(self, w, device="cuda", partition_tokens: int = 0, stream=None,
-                 shared_prefix_blocks: int = 0):
+                 shared_prefix_blocks: int = 0, window: int = 0):
+        if shared_prefix_blocks and window:
+            raise ValueError("a shared prefix and a sliding window are separate decode paths")
         self.w = w
         self.device = torch.device(device)
         self.stream = stream
         self.partition_tokens = partition_tokens
         self.shared_prefix_blocks = shared_prefix_blocks
+        self.window = window
         dev = self.device
         cshape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         if w.cache_dtype == "e4m3":
@@ -72,6 +76,10 @@ class DecodeStep:
             ws = B.pa_decode_shared_prefix_workspace_size(w.batch, w.num_q_heads,
                                                           self.max_context, shared_prefix_blocks,
                                                           self.cache, partition_tokens)
+        elif window:
+            ws = B.pa_decode_sliding_window_workspace_size(w.batch, w.num_q_heads,
+                                                           self.max_context, window, self.cache,
+                                                           partition_tokens)
         else:
             ws = B.pa_decode_workspace_size(w.batch, w.num_q_heads, self.max_context,
                                             self.cache, partition_tokens)
@@ -99,6 +107,12 @@ class DecodeStep:
                                       self.context_lens, float(self.w.scale), self.out,
                                       self.cache, self.max_context, self.shared_prefix_blocks,
                                       self.partition_tokens, self.workspace, self.stream)
+            return
+        if self.window:
+            B.pa_decode_sliding_window(self.q, self.k_cache, self.v_cache, self.block_tables,
+                                       self.context_lens, float(self.w.scale), self.out,
+                                       self.cache, self.max_context, self.window,
+                                       self.partition_tokens, self.workspace, self.stream)
             return
         B.pa_decode(self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                     float(self.w.scale), self.out, self.cache, self.max_context,

@@ -26,7 +26,7 @@ def oracle_caches(w):
     return w.k_pool.copy(), w.v_pool.copy()
 
 
-def oracle_step(w, seqs=None):
+def oracle_step(w, seqs=None, window=0):
     """copy_blocks -> append -> decode on the CPU; returns (k_cache, v_cache,
     out) with out float64 [len(seqs), Hq, D]."""
     kc, vc = oracle_caches(w)
@@ -36,7 +36,7 @@ def oracle_step(w, seqs=None):
                      w.block_size, w.k_inv_scale, w.v_inv_scale)
     sel = np.arange(w.batch) if seqs is None else np.asarray(seqs)
     out = oracle.decode(w.q[sel], w.io_dtype, kc, vc, w.cache_dtype, w.block_tables[sel],
-                        w.context_lens[sel], w.scale, w.k_scale, w.v_scale)
+                        w.context_lens[sel], w.scale, w.k_scale, w.v_scale, window=window)
     return kc, vc, out
 
 
