@@ -1,7 +1,8 @@
 """Build libpagedattn.so in-tree with nvcc for sm_100a (B200).
 
-The whole library is one translation unit (csrc/pa_api.cu includes the
-kernel headers), so the build is a single nvcc call. The result lands next to
+The kernels and their C ABI are one translation unit (csrc/pa_api.cu
+includes the kernel headers); the host block manager is a second, plain C++
+one. One nvcc call compiles and links both. The result lands next to
 this file, where the binding loads it from.
 """
 from __future__ import annotations
@@ -14,7 +15,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libpagedattn.so")
-SOURCES = [os.path.join(HERE, "csrc", "pa_api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "pa_api.cu"),
+           os.path.join(HERE, "csrc", "pa_block_manager.cpp")]
 DEPS = sorted(glob.glob(os.path.join(HERE, "csrc", "*")) +
               glob.glob(os.path.join(ROOT, "include", "*.h")))
 

@@ -1,0 +1,194 @@
+"""Host block manager (include/pa_block_manager.h) on the CPU.
+
+What the pages fix and these tests check: blocks of a fixed size, taken on
+demand -- a sequence gets its second block only when token BS+1 arrives (page
+'AI 陪读顶会论文（三）：KV Cache 显存占用计算与 PagedAttention 原理拆解',
+section 'PagedAttention 的破局哲学'); a shared prefix is stored once and
+reference-counted, and branches copy a block only where they diverge (KV cache
+article, section 'PagedAttention：把操作系统的老智慧搬进推理引擎'); a radix tree
+of token ids lets later requests reuse a cached prefix (chapter '第2章 KV
+Cache：模型内部的显存复用')."""
+import re
+import os
+
+import numpy as np
+import pytest
+
+from paged_kv_cache_410_b200 import block_manager as BM
+from paged_kv_cache_410_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def test_header_symbols_are_exported():
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "pa_block_manager.h")).read(),
+                  flags=re.S)
+    names = sorted(set(re.findall(r"\b(pa_bm_[a-z_]+)\s*\(", text)))
+    assert names == sorted(BM.EXPORTED)
+    lib = BM._lib()
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_blocks_are_taken_on_demand():
+    bm = BM.BlockManager(10, 16)
+    bm.add_sequence(1, range(16))                    # 16 tokens: one block
+    assert bm.num_free_blocks == 9
+    slot, cow = bm.append_token(1, 99)               # token 17: the second block
+    assert cow is None and bm.num_free_blocks == 8
+    tables, lens = bm.block_tables([1], 4)
+    assert lens.tolist() == [17]
+    assert slot == tables[0, 1] * 16 + 0
+    for k in range(15):                              # tokens 18..32 fill it
+        bm.append_token(1, k)
+    assert bm.num_free_blocks == 8
+    bm.append_token(1, 0)                            # token 33: the third block
+    assert bm.num_free_blocks == 7
+
+
+def test_slots_follow_the_block_table():
+    bm = BM.BlockManager(50, 8)
+    bm.add_sequence(7, range(29))
+    tables, lens = bm.block_tables([7], 6)
+    slots = bm.slots(7, 0, 29)
+    j = np.arange(29)
+    assert np.array_equal(slots, tables[0, j // 8].astype(np.int64) * 8 + j % 8)
+    assert len(set(tables[0, :4].tolist())) == 4 and tables[0, 4:].tolist() == [0, 0]
+
+
+def test_fork_shares_blocks_and_copies_only_the_partial_last_block():
+    bm = BM.BlockManager(20, 16)
+    bm.add_sequence(0, range(40))                    # 2 full blocks + 8 tokens in a third
+    for c in (1, 2, 3):
+        bm.fork(0, c)
+    t, _ = bm.block_tables([0, 1, 2, 3], 4)
+    assert (t == t[0]).all()                         # the beams share every block
+    assert [bm.refcount(b) for b in t[0, :3]] == [4, 4, 4]
+    free0 = bm.num_free_blocks
+    copies = []
+    for s in (0, 1, 2, 3):
+        slot, cow = bm.append_token(s, 1000 + s)
+        if cow:
+            copies.append(cow)
+    # three beams copy the shared partial block; the last one writes in place
+    assert len(copies) == 3 and {c[0] for c in copies} == {int(t[0, 2])}
+    assert bm.num_free_blocks == free0 - 3
+    t2, lens = bm.block_tables([0, 1, 2, 3], 4)
+    assert lens.tolist() == [41] * 4
+    assert (t2[:, :2] == t[0, :2]).all()             # full blocks still shared
+    assert len(set(t2[:, 2].tolist())) == 4          # last blocks now private
+    assert [bm.refcount(b) for b in t2[0, :2]] == [4, 4]
+
+
+def test_fork_at_a_block_boundary_needs_no_copy():
+    bm = BM.BlockManager(20, 16)
+    bm.add_sequence(0, range(32))
+    bm.fork(0, 1)
+    for s in (0, 1):
+        _, cow = bm.append_token(s, 5)
+        assert cow is None
+
+
+def test_freeing_drops_references_not_shared_blocks():
+    bm = BM.BlockManager(12, 4)
+    bm.add_sequence(0, range(10))                    # 3 blocks
+    bm.fork(0, 1)
+    bm.free_sequence(0)
+    assert bm.num_free_blocks == 9                   # the child still holds all three
+    t, _ = bm.block_tables([1], 3)
+    assert [bm.refcount(b) for b in t[0]] == [1, 1, 1]
+    bm.free_sequence(1)
+    assert bm.num_free_blocks == 12
+
+
+def test_prefix_cache_reuses_full_prompt_blocks():
+    bm = BM.BlockManager(40, 16, prefix_cache=True)
+    system = list(range(100, 132))                   # a 32-token system prompt
+    assert bm.add_sequence(1, system + [1, 2, 3]) == 0
+    assert bm.add_sequence(2, system + [7, 8]) == 32
+    assert bm.add_sequence(3, [5] + system) == 0     # different first block: no reuse
+    t, _ = bm.block_tables([1, 2, 3], 3)
+    assert (t[0, :2] == t[1, :2]).all() and t[0, 2] != t[1, 2]
+    assert not set(t[2, :2].tolist()) & set(t[0, :2].tolist())
+    # the cached blocks outlive the requests that made them
+    bm.free_sequence(1)
+    bm.free_sequence(2)
+    assert bm.num_cached_blocks >= 2
+    assert bm.add_sequence(4, system + [9]) == 32
+    t4, _ = bm.block_tables([4], 3)
+    assert (t4[0, :2] == t[0, :2]).all()
+
+
+def test_partial_prefix_match_stops_at_the_first_different_block():
+    bm = BM.BlockManager(40, 4, prefix_cache=True)
+    bm.add_sequence(1, [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12])
+    assert bm.add_sequence(2, [1, 2, 3, 4, 5, 6, 7, 0, 9, 10, 11, 12]) == 4
+    assert bm.add_sequence(3, [1, 2, 3, 4, 5, 6, 7, 8, 9]) == 8
+
+
+def test_blocks_filled_by_decoding_join_the_cache():
+    bm = BM.BlockManager(20, 8, prefix_cache=True)
+    bm.add_sequence(1, [3] * 5)
+    for k in range(3):
+        bm.append_token(1, 3)                        # the first block fills with token 8
+    assert bm.add_sequence(2, [3] * 8 + [4]) == 8
+
+
+def test_lru_eviction_of_cached_blocks():
+    bm = BM.BlockManager(4, 2, prefix_cache=True)
+    bm.add_sequence(1, [1, 1])                       # cached block A
+    bm.free_sequence(1)
+    bm.add_sequence(2, [2, 2])                       # cached block B
+    bm.free_sequence(2)
+    assert bm.num_free_blocks == 2 and bm.num_cached_blocks == 2
+    assert bm.add_sequence(3, [1, 1]) == 2           # touches A: B is now least recent
+    bm.free_sequence(3)
+    bm.add_sequence(4, [9, 9, 9, 9, 9, 9])           # 3 blocks: 2 free + 1 evicted (B)
+    assert bm.num_free_blocks == 0
+    bm.free_sequence(4)
+    assert bm.add_sequence(5, [1, 1]) == 2           # A survived
+    assert bm.add_sequence(6, [2, 2]) == 0           # B did not
+
+
+def test_out_of_blocks_leaves_the_manager_unchanged():
+    bm = BM.BlockManager(3, 4)
+    bm.add_sequence(1, range(8))
+    with pytest.raises(BM.BlockManagerError) as e:
+        bm.add_sequence(2, range(8))
+    assert e.value.code == BM.ERR_NO_BLOCKS
+    assert bm.num_free_blocks == 1
+    with pytest.raises(BM.BlockManagerError):
+        bm.length(2)
+
+
+def test_release_before_frees_blocks_outside_a_window():
+    bm = BM.BlockManager(10, 4)
+    bm.add_sequence(1, range(18))                    # 5 blocks
+    bm.release_before(1, 9)                          # blocks 0 and 1 hold only tokens < 8
+    assert bm.num_free_blocks == 7
+    bm.slots(1, 8, 10)
+    with pytest.raises(BM.BlockManagerError):
+        bm.slots(1, 7, 2)
+    bm.free_sequence(1)
+    assert bm.num_free_blocks == 10
+
+
+def test_invalid_calls():
+    bm = BM.BlockManager(5, 4)
+    bm.add_sequence(1, range(3))
+    for fn in (lambda: bm.add_sequence(1, [1]), lambda: bm.append_token(9),
+               lambda: bm.fork(9, 10), lambda: bm.fork(1, 1), lambda: bm.free_sequence(9),
+               lambda: bm.slots(1, 2, 5), lambda: bm.block_tables([1, 9], 2)):
+        with pytest.raises(BM.BlockManagerError):
+            fn()
+    with pytest.raises(BM.BlockManagerError) as e:
+        bm.block_tables([1], 0)
+    bm.add_sequence(2, range(9))
+    with pytest.raises(BM.BlockManagerError) as e:
+        bm.block_tables([2], 2)
+    assert e.value.code == BM.ERR_CAPACITY
