@@ -306,12 +306,12 @@ def run_ours(args):
 
     w = make_workload(args.workload, rank, args.batch)
     spb = w.meta.get("shared_prefix_blocks", 0) if args.cascade == "auto" else 0
-    if args.window:
+    if args.window or args.fused:
         spb = 0
     step = DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb,
-                      window=args.window)
+                      window=args.window, fused=args.fused)
     stream = torch.cuda.current_stream(dev)
-    sb = A.step_bytes(w, window=args.window)
+    sb = A.step_bytes(w, window=args.window, fused=args.fused)
     if args.window:
         plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
             w.batch, min(w.max_context, args.window + 15), step.cache)
@@ -331,7 +331,12 @@ def run_ours(args):
         n_parts = max(1, math.ceil(w.max_context / plan_pt))
         decode_launches = 1 + (1 if n_parts > 1 else 0)
         decode_name = "pa_decode (main + split-K reduce)"
-    launches_per_step = 1 + decode_launches + math.ceil(len(w.copy_pairs) / 256)
+    if args.fused:
+        decode_name = "pa_append_decode (append fused into decode; main + split-K reduce)"
+    launches_per_step = (0 if args.fused else 1) + decode_launches + math.ceil(
+        len(w.copy_pairs) / 256)
+    timed_call = step.append_decode if args.fused else step.decode
+    timed_bytes = sb["append_decode"] if args.fused else sb["decode"]
 
     for _ in range(args.warmup):
         step.run()
@@ -353,9 +358,10 @@ def run_ours(args):
     t_start.record(stream)
     for i in range(args.steps):
         step.copy()
-        step.append()
+        if not args.fused:
+            step.append()
         ev[i][0].record(stream)
-        step.decode()
+        timed_call()
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -406,10 +412,15 @@ def run_ours(args):
     else:
         peak, peak_src = FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
     dec_ms = statistics.mean(decode_ms)
-    achieved = sb["decode"] / (dec_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(w.name)
+    achieved = timed_bytes / (dec_ms * 1e-3) / 1e9
+    # the committed ncu counters cover the plain whole-history decode only
+    traffic = None if (args.window or args.fused or spb) else recorded_traffic(w.name)
 
     line = base_line(args, w, world)
+    line["config"]["decode"] = ("append fused into decode" if args.fused else
+                                f"sliding window {args.window}" if args.window else
+                                f"shared-prefix cascade ({spb} blocks)" if spb else
+                                "whole history")
     line.update({
         "value": value, "ms_per_step": ms_per_step,
         "tokens_per_s_per_layer": tokens_per_s,
@@ -419,7 +430,7 @@ def run_ours(args):
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
-                     "algorithmic_bytes_per_launch": sb["decode"],
+                     "algorithmic_bytes_per_launch": timed_bytes,
                      "decode_ms_mean": dec_ms, "decode_ms_median": statistics.median(decode_ms),
                      "partition_tokens": plan_pt, "partitions": n_parts},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -453,6 +464,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--window", type=int, default=0,
                     help="sliding-window decode over the last WINDOW tokens (0: whole history)")
+    ap.add_argument("--fused", action="store_true",
+                    help="append each sequence's new token inside the decode launch "
+                         "(pa_append_decode) instead of a separate pa_append_kv")
     ap.add_argument("--cascade", choices=["auto", "off"], default="auto",
                     help="decode a workload whose sequences share prefix blocks through "
                          "pa_decode_shared_prefix (auto) or plain pa_decode (off)")

@@ -9,6 +9,11 @@
  *                   whole cached history, gathered through its block table;
  *   pa_copy_blocks  duplicate whole blocks (copy-on-write at a fork).
  *
+ * Variants: pa_append_decode (append fused into the decode launch),
+ * pa_decode_sliding_window, pa_decode_shared_prefix (a shared prefix attended
+ * once for the whole batch), pa_copy_blocks_layers (every layer's caches in
+ * one call) and pa_decode_static_workspace (no caller workspace).
+ *
  * Sources of the definitions (page titles and sections):
  *  - "AI 陪读顶会论文（三）：KV Cache 显存占用计算与 PagedAttention 原理拆解",
  *    section "为什么自回归解码必须使用 KV Cache？": the attention equation
@@ -72,7 +77,8 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
 /* Bits of the device error word (pa_get_device_error). */
 #define PA_DEVERR_BLOCK_ID 0x1u    /* a block-table entry outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT_LEN 0x2u /* context_len < 0, > max_context, or beyond the table */
-#define PA_DEVERR_SLOT 0x4u        /* append slot >= num_blocks * block_size */
+#define PA_DEVERR_SLOT 0x4u        /* append slot >= num_blocks * block_size, or (fused
+                                      append) not the slot of position context_len - 1 */
 #define PA_DEVERR_PREFIX 0x8u      /* pa_decode_shared_prefix: a sequence does not start
                                       with the shared prefix blocks, or is shorter */
 
@@ -141,6 +147,34 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                     int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* pa_append_kv followed by pa_decode in one launch, for a batch with one new
+ * token per sequence ("AI 陪读顶会论文（三）：...", section "为什么自回归解码必须
+ * 使用 KV Cache？": each step computes the new token's k_t, v_t, appends them and
+ * attends over the whole cache). The new token of sequence b is the token at
+ * position context_lens[b] - 1: the decode reads its K/V from k / v directly
+ * (quantised exactly as pa_append_kv would for an E4M3 cache) and the CTA of
+ * the sequence's last partition stores it at slot_mapping[b]. Caches and
+ * output equal those of the two separate calls.
+ *   q             [batch][num_q_heads][head_dim] in dtype.
+ *   k, v          [batch][num_kv_heads][head_dim] in dtype (PA_F16 / PA_BF16;
+ *                 for a 16-bit cache, the cache dtype).
+ *   slot_mapping  [batch] int64; slot_mapping[b] must be the slot of position
+ *                 context_lens[b] - 1 in sequence b's table (else the device
+ *                 error word gets PA_DEVERR_SLOT, nothing is stored and that
+ *                 sequence's result is not meaningful); < 0: no new token for
+ *                 b (plain decode). The slot must not lie in another
+ *                 sequence's context in this batch (copy-on-write has run).
+ *   k_cache, v_cache  written at the new slots (the same as pa_decode's
+ *                 caches otherwise).
+ * Other arguments as for pa_decode (same workspace size). */
+pa_status pa_append_decode(const void* q, const void* k, const void* v, int32_t dtype,
+                           int32_t batch, int32_t num_q_heads, const int64_t* slot_mapping,
+                           void* k_cache, void* v_cache, const pa_cache_desc* cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t max_context, float scale,
+                           void* out, int32_t partition_tokens, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Workspace bytes for pa_decode_sliding_window. Pure host function. */
 size_t pa_decode_sliding_window_workspace_size(int32_t batch, int32_t num_q_heads,
                                                int32_t max_context, int32_t window,
@@ -207,6 +241,20 @@ pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
  * matter); otherwise PA_ERR_INVALID_ARG. num_pairs == 0 is a no-op. */
 pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_cache,
                          void* v_cache, const pa_cache_desc* cache, void* stream);
+
+/* pa_copy_blocks applied to every layer of a model in one call (one launch
+ * per 32 layers and 256 pairs). Copy-on-write is decided per sequence, not
+ * per layer, so a step's block copies are the same for all layers and can
+ * run before any layer does; a layer's append and decode cannot be batched
+ * this way, since they need that layer's input.
+ *   k_caches, v_caches  HOST arrays of num_layers DEVICE pointers, one K and
+ *                 one V cache per layer, all described by `cache`; every
+ *                 pointer non-null and 16-byte aligned.
+ * Pair rules as for pa_copy_blocks; num_pairs == 0 or num_layers == 0 is a
+ * no-op. */
+pa_status pa_copy_blocks_layers(const int32_t* pairs_host, int32_t num_pairs,
+                                void* const* k_caches, void* const* v_caches, int32_t num_layers,
+                                const pa_cache_desc* cache, void* stream);
 
 /* Synchronise `stream`, then read and clear the current device's error
  * word into *flags (PA_DEVERR_* bits). Returns PA_ERR_DEVICE_BOUNDS when

@@ -68,10 +68,25 @@ def copy_bytes(w) -> int:
     return int(len(w.copy_pairs) * block * 2 * 2)
 
 
-def step_bytes(w, window: int = 0) -> dict:
+def fused_bytes(w) -> int:
+    """Append and decode as one pass: the decode's bytes and the append's,
+    less the cache read of each new token's row (the pass takes that row from
+    the appended input instead; it lies in a block no other sequence reads)."""
+    eb = ELEM_BYTES[w.cache_dtype]
+    T = int(np.sum(w.slot_mapping >= 0))
+    new_rows = 2 * T * w.num_kv_heads * w.head_dim * eb
+    return decode_bytes(w)["total_unique"] + append_bytes(w) - new_rows
+
+
+def step_bytes(w, window: int = 0, fused: bool = False) -> dict:
+    """`fused`: append and decode counted as one pass (fused_bytes)."""
     d = decode_bytes(w, window)
     a = append_bytes(w)
     c = copy_bytes(w)
-    return {"decode": d["total_unique"], "decode_logical": d["total_logical"],
-            "kv_unique": d["kv_unique"], "append": a, "copy": c,
-            "total": d["total_unique"] + a + c}
+    out = {"decode": d["total_unique"], "decode_logical": d["total_logical"],
+           "kv_unique": d["kv_unique"], "append": a, "copy": c,
+           "total": d["total_unique"] + a + c}
+    if fused:
+        out["append_decode"] = fused_bytes(w)
+        out["total"] = out["append_decode"] + c
+    return out

@@ -29,7 +29,8 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_decode", "pa_copy_blocks", "pa_get_device_error", "pa_status_string",
             "pa_version", "pa_decode_static_workspace",
             "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
-            "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window"]
+            "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
+            "pa_append_decode", "pa_copy_blocks_layers"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -90,6 +91,12 @@ def load_library(path: str = LIB_PATH):
     lib.pa_decode_sliding_window.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, i32,
                                              ctypes.c_float, P, i32, P, ctypes.c_size_t, P]
     lib.pa_decode_sliding_window.restype = ctypes.c_int
+    lib.pa_append_decode.argtypes = [P, P, P, i32, i32, i32, P, P, P, D, P, i32, P, i32,
+                                     ctypes.c_float, P, i32, P, ctypes.c_size_t, P]
+    lib.pa_append_decode.restype = ctypes.c_int
+    lib.pa_copy_blocks_layers.argtypes = [P, i32, ctypes.POINTER(P), ctypes.POINTER(P), i32, D,
+                                          P]
+    lib.pa_copy_blocks_layers.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -184,6 +191,27 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache
     _check(rc, "pa_decode")
 
 
+def pa_append_decode(q, k, v, slot_mapping, k_cache, v_cache, block_tables, context_lens,
+                     scale, out, cache: PagedCache, max_context: int, partition_tokens: int = 0,
+                     workspace=None, stream=None):
+    """pa_append_kv of one new token per sequence (k, v: [batch, Hkv, D];
+    slot_mapping: [batch] int64, the slot of position context_lens[b] - 1,
+    or -1 for none) and pa_decode over the updated history, in one launch.
+    The workspace is sized by pa_decode_workspace_size."""
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("pa_append_decode: q, k and v share one dtype")
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.pa_append_decode(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), batch, hq,
+                              _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+                              _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                              int(max_context), float(scale), _ptr(out), int(partition_tokens),
+                              _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "pa_append_decode")
+
+
 def pa_decode_shared_prefix_workspace_size(batch, num_q_heads, max_context, prefix_blocks,
                                            cache: PagedCache, partition_tokens=0) -> int:
     lib = load_library()
@@ -264,6 +292,22 @@ def pa_copy_blocks(pairs, k_cache, v_cache, cache: PagedCache, stream=None):
     rc = lib.pa_copy_blocks(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], _ptr(k_cache),
                             _ptr(v_cache), ctypes.byref(d), _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def pa_copy_blocks_layers(pairs, k_caches, v_caches, cache: PagedCache, stream=None):
+    """pa_copy_blocks on every layer's K and V cache (sequences of device
+    tensors, one per layer, all of `cache`'s shape) in one call."""
+    if len(k_caches) != len(v_caches):
+        raise ValueError("one K and one V cache per layer")
+    lib = load_library()
+    d = cache.desc()
+    arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    n = len(k_caches)
+    kp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in k_caches])
+    vp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in v_caches])
+    rc = lib.pa_copy_blocks_layers(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], kp, vp, n,
+                                   ctypes.byref(d), _stream(stream))
+    _check(rc, "pa_copy_blocks_layers")
 
 
 def pa_get_device_error(stream=None) -> int:

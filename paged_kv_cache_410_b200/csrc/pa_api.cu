@@ -141,7 +141,8 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
 template <typename TQ, int CK, int D, int NH>
 pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
-  auto kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH>;
+  auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
+                      : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
   const int bt_entries =
       std::min((p.partition_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
   const int smem = S::kMainBytes + bt_entries * 4;
@@ -427,6 +428,46 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
   return launch_decode(p, q_dtype, cache, as_stream(stream));
 }
 
+pa_status pa_append_decode(const void* q, const void* k, const void* v, int32_t dtype,
+                           int32_t batch, int32_t num_q_heads, const int64_t* slot_mapping,
+                           void* k_cache, void* v_cache, const pa_cache_desc* cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t max_context, float scale,
+                           void* out, int32_t partition_tokens, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  int bs_log2 = 0;
+  bool nothing = false;
+  pa_status st = check_decode_args(q, dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, out, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK || nothing) return st;
+  if (!k || !v || !slot_mapping || !aligned16(k) || !aligned16(v)) return PA_ERR_INVALID_ARG;
+  if (cache->cache_dtype == PA_E4M3 &&
+      (!cache->k_inv_scale || !cache->v_inv_scale || !aligned16(cache->k_inv_scale) ||
+       !aligned16(cache->v_inv_scale)))
+    return PA_ERR_INVALID_ARG;
+  const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (pl.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
+  }
+  pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
+                                     block_tables, max_blocks_per_seq, context_lens, max_context,
+                                     scale, out, bs_log2);
+  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
+  p.ws_ml = pl.ws_bytes
+                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
+                : nullptr;
+  p.partition_tokens = pl.partition_tokens;
+  p.num_partitions = pl.num_partitions;
+  p.k_new = k;
+  p.v_new = v;
+  p.slot_mapping = slot_mapping;
+  p.k_inv_scale = cache->k_inv_scale;
+  p.v_inv_scale = cache->v_inv_scale;
+  return launch_decode(p, dtype, cache, as_stream(stream));
+}
+
 size_t pa_decode_sliding_window_workspace_size(int32_t batch, int32_t num_q_heads,
                                                int32_t max_context, int32_t window,
                                                int32_t partition_tokens,
@@ -539,15 +580,18 @@ pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
   }
 }
 
-pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_cache,
-                         void* v_cache, const pa_cache_desc* cache, void* stream) {
+pa_status pa_copy_blocks_layers(const int32_t* pairs_host, int32_t num_pairs,
+                                void* const* k_caches, void* const* v_caches, int32_t num_layers,
+                                const pa_cache_desc* cache, void* stream) {
   int bs_log2 = 0;
   pa_status st = check_cache(cache, &bs_log2);
   if (st != PA_OK) return st;
-  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
-  if (num_pairs == 0) return PA_OK;
-  if (!pairs_host || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+  if (num_pairs < 0 || num_layers < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0 || num_layers == 0) return PA_OK;
+  if (!pairs_host || !k_caches || !v_caches) return PA_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < num_layers; ++l)
+    if (!k_caches[l] || !v_caches[l] || !aligned16(k_caches[l]) || !aligned16(v_caches[l]))
+      return PA_ERR_INVALID_ARG;
   std::unordered_set<int32_t> srcs, dsts;
   for (int32_t i = 0; i < num_pairs; ++i) {
     const int32_t s = pairs_host[2 * i], d = pairs_host[2 * i + 1];
@@ -562,20 +606,30 @@ pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_c
   const int64_t block_bytes = static_cast<int64_t>(cache->block_size) * cache->num_kv_heads *
                               cache->head_dim * elem_bytes(cache->cache_dtype);
   pa::CopyParams p{};
-  p.k_cache = k_cache;
-  p.v_cache = v_cache;
   p.block_vec16 = block_bytes / 16;
   const int64_t slices = std::min<int64_t>(std::max<int64_t>(p.block_vec16 / (256 * 4), 1), 64);
   const cudaStream_t s = as_stream(stream);
-  for (int32_t base = 0; base < num_pairs; base += pa::kCopyPairsPerLaunch) {
-    const int n = std::min(num_pairs - base, pa::kCopyPairsPerLaunch);
-    p.num_pairs = n;
-    for (int i = 0; i < n; ++i)
-      p.pairs[i] = make_int2(pairs_host[2 * (base + i)], pairs_host[2 * (base + i) + 1]);
-    pa::pa_copy_blocks_kernel<<<dim3(n, static_cast<unsigned>(slices)), 256, 0, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  for (int32_t l0 = 0; l0 < num_layers; l0 += pa::kCopyLayersPerLaunch) {
+    const int nl = std::min(num_layers - l0, pa::kCopyLayersPerLaunch);
+    for (int l = 0; l < nl; ++l) {
+      p.k_cache[l] = k_caches[l0 + l];
+      p.v_cache[l] = v_caches[l0 + l];
+    }
+    for (int32_t base = 0; base < num_pairs; base += pa::kCopyPairsPerLaunch) {
+      const int n = std::min(num_pairs - base, pa::kCopyPairsPerLaunch);
+      p.num_pairs = n;
+      for (int i = 0; i < n; ++i)
+        p.pairs[i] = make_int2(pairs_host[2 * (base + i)], pairs_host[2 * (base + i) + 1]);
+      pa::pa_copy_blocks_kernel<<<dim3(n, static_cast<unsigned>(slices), nl), 256, 0, s>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    }
   }
   return PA_OK;
+}
+
+pa_status pa_copy_blocks(const int32_t* pairs_host, int32_t num_pairs, void* k_cache,
+                         void* v_cache, const pa_cache_desc* cache, void* stream) {
+  return pa_copy_blocks_layers(pairs_host, num_pairs, &k_cache, &v_cache, 1, cache, stream);
 }
 
 pa_status pa_get_device_error(void* stream, uint32_t* flags) {

@@ -83,22 +83,25 @@ __global__ void __launch_bounds__(128) pa_append_kernel(const AppendParams p) {
 }
 
 constexpr int kCopyPairsPerLaunch = 256;
+constexpr int kCopyLayersPerLaunch = 32;
 
 struct CopyParams {
-  void* k_cache;
-  void* v_cache;
+  void* k_cache[kCopyLayersPerLaunch];  // one K and one V cache per layer of this launch
+  void* v_cache[kCopyLayersPerLaunch];
   int64_t block_vec16;  // 16-byte vectors per block
   int num_pairs;
   int2 pairs[kCopyPairsPerLaunch];  // (src, dst), checked on the host
 };
 
-// grid.x = pair, grid.y = slices of the block; each thread moves 16 B at a time.
+// grid.x = pair, grid.y = slices of the block, grid.z = layer; each thread
+// moves 16 B of K and 16 B of V at a time.
 __global__ void __launch_bounds__(256) pa_copy_blocks_kernel(const CopyParams p) {
   const int2 pr = p.pairs[blockIdx.x];
-  const uint4* ks = reinterpret_cast<const uint4*>(p.k_cache) + pr.x * p.block_vec16;
-  const uint4* vs = reinterpret_cast<const uint4*>(p.v_cache) + pr.x * p.block_vec16;
-  uint4* kd = reinterpret_cast<uint4*>(p.k_cache) + pr.y * p.block_vec16;
-  uint4* vd = reinterpret_cast<uint4*>(p.v_cache) + pr.y * p.block_vec16;
+  const int layer = blockIdx.z;
+  const uint4* ks = reinterpret_cast<const uint4*>(p.k_cache[layer]) + pr.x * p.block_vec16;
+  const uint4* vs = reinterpret_cast<const uint4*>(p.v_cache[layer]) + pr.x * p.block_vec16;
+  uint4* kd = reinterpret_cast<uint4*>(p.k_cache[layer]) + pr.y * p.block_vec16;
+  uint4* vd = reinterpret_cast<uint4*>(p.v_cache[layer]) + pr.y * p.block_vec16;
   const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; i < p.block_vec16;
        i += stride) {

@@ -71,7 +71,38 @@ struct DecodeParams {
   // Sliding window (0: none): a sequence of length L attends to its tokens
   // [L - window, L) only.
   int window;
+  // Fused append (null k_new: none): sequence b's new token, at position
+  // L - 1, comes from k_new / v_new [batch][num_kv_heads][head_dim] (in the
+  // query dtype); it is read from there, not from the cache, and the CTA of
+  // the sequence's last partition stores it at slot_mapping[b].
+  const void* k_new;
+  const void* v_new;
+  const int64_t* slot_mapping;
+  const float* k_inv_scale;  // E4M3 caches
+  const float* v_inv_scale;
 };
+
+// 16 consecutive channels of a 16-bit input row -> 16 E4M3 codes, each
+// e4m3_rn_satfinite(fp32(x) * inv_scale) (the append kernel's rounding).
+template <typename TIn>
+__device__ __forceinline__ uint4 quantize16(const TIn* x, const float* inv) {
+  const uint4 a = *reinterpret_cast<const uint4*>(x);
+  const uint4 b = *reinterpret_cast<const uint4*>(x + 8);
+  const TIn* ea = reinterpret_cast<const TIn*>(&a);
+  const TIn* eb = reinterpret_cast<const TIn*>(&b);
+  float y[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    y[j] = __fmul_rn(to_f32<TIn>(ea[j]), inv[j]);
+    y[8 + j] = __fmul_rn(to_f32<TIn>(eb[j]), inv[8 + j]);
+  }
+  uint4 r;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    w[k] = f32x2_to_e4m3x2(y[4 * k], y[4 * k + 1]) | (f32x2_to_e4m3x2(y[4 * k + 2], y[4 * k + 3]) << 16);
+  return r;
+}
 
 __device__ __forceinline__ int clamp_context(const DecodeParams& p, int L) {
   const int64_t table_cap = static_cast<int64_t>(p.max_blocks_per_seq) << p.bs_log2;
@@ -372,7 +403,8 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
 //
 // One decode CTA: partition `part` of sequence `b`, for KV head / head group
 // `by` (= kv_head * head_groups + head_group).
-template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH>
+// FUSED: the launch also appends each sequence's new token (pa_append_decode).
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED = false>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part, const int by,
                                            const int b) {
   using G = TileGeom<CK, D>;
@@ -482,6 +514,70 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     return id;
   };
 
+  // ---- fused append: the new token (position L - 1) comes from the input --
+  const bool has_new = FUSED && p.slot_mapping[b] >= 0;
+  const int jnew = has_new ? L - 1 : -1;
+  const int64_t new_row = (static_cast<int64_t>(b) * p.num_kv_heads + hk) * D;  // elements
+  const TQ* knew = has_new ? reinterpret_cast<const TQ*>(p.k_new) + new_row : nullptr;
+  const TQ* vnew = has_new ? reinterpret_cast<const TQ*>(p.v_new) + new_row : nullptr;
+  if (has_new && part == nparts - 1 && hgrp == 0) {
+    // store it in the cache, as pa_append_kv would; the slot must be the one
+    // the table gives position L - 1
+    const int64_t slot = p.slot_mapping[b];
+    const int64_t expect =
+        (static_cast<int64_t>(p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq +
+                                             (jnew >> p.bs_log2)])
+         << p.bs_log2) +
+        (jnew & ((1 << p.bs_log2) - 1));
+    if (slot != expect || slot >= (static_cast<int64_t>(p.num_blocks) << p.bs_log2)) {
+      if (threadIdx.x == 0) flag_error(PA_DEVERR_SLOT);
+    } else if (threadIdx.x < 2 * G::CPR) {
+      const bool is_v = threadIdx.x >= G::CPR;
+      const int ch = threadIdx.x - (is_v ? G::CPR : 0);
+      // (the fused entry point passes writable caches)
+      uint8_t* dst = static_cast<uint8_t*>(const_cast<void*>(is_v ? p.v_cache : p.k_cache)) +
+                     (slot * p.num_kv_heads + hk) * G::RB + ch * 16;
+      const TQ* src = is_v ? vnew : knew;
+      if constexpr (CK == kE4M3) {
+        const float* inv = (is_v ? p.v_inv_scale : p.k_inv_scale) + hk * D + 16 * ch;
+        *reinterpret_cast<uint4*>(dst) = quantize16<TQ>(src + 16 * ch, inv);
+      } else {
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src + 8 * ch);
+      }
+    }
+  }
+
+  // One 16-byte chunk of row r: from the cache at `off`, or from the fused
+  // new token (16-bit: the same bytes by cp.async; E4M3: no copy here, the
+  // tile's new-token fix-up below stores the quantised row).
+  auto load_chunk = [&](uint32_t sk_a, uint32_t sv_a, int r, int j, bool ok, int64_t off) {
+    const uint32_t so = G::off(r, lch);
+    if (FUSED && j == jnew) {
+      if constexpr (CK != kE4M3) {
+        cp_async_16(sk_a + so, knew + 8 * lch, 16u);
+        cp_async_16(sv_a + so, vnew + 8 * lch, 16u);
+      }
+      return;
+    }
+    cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
+    cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
+  };
+  // E4M3 fused: the new token's row of the tile starting at tb, quantised
+  // once per tile by lanes 0 .. 2*CPR-1 (K chunks, then V chunks).
+  auto store_new_row = [&](uint32_t sk_a, uint32_t sv_a, int tb) {
+    if constexpr (FUSED && CK == kE4M3) {
+      if (jnew >= tb && jnew < tb + 16 && lane < 2 * G::CPR) {
+        const bool is_v = lane >= G::CPR;
+        const int ch = lane - (is_v ? G::CPR : 0);
+        const uint4 qv = quantize16<TQ>((is_v ? vnew : knew) + 16 * ch,
+                                        (is_v ? p.v_inv_scale : p.k_inv_scale) + hk * D + 16 * ch);
+        const uint32_t a = (is_v ? sv_a : sk_a) + G::off(jnew - tb, ch);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(qv.x),
+                     "r"(qv.y), "r"(qv.z), "r"(qv.w));
+      }
+    }
+  };
+
   auto load_tile = [&](int tile, int stage) {
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
@@ -496,26 +592,23 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
         const int r = lrow + i * RPI;
         const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
         const int64_t off = ok ? base + static_cast<int64_t>(i * RPI) * slot_stride : 0;
-        const uint32_t so = G::off(r, lch);
-        cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
-        cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
+        load_chunk(sk_a, sv_a, r, tb + r, ok, off);
       }
     } else {
 #pragma unroll
       for (int i = 0; i < LITERS; ++i) {
         const int r = lrow + i * RPI;
         const int j = tb + r;
-        const int blk = (j < t1 && j >= lo) ? block_id((j >> p.bs_log2) - bt0) : -1;
+        const int blk = (j < t1 && j >= lo && j != jnew) ? block_id((j >> p.bs_log2) - bt0) : -1;
         const bool ok = blk >= 0;
         const int64_t off =
             ok ? ((static_cast<int64_t>(blk) << p.bs_log2) + (j & bs_mask)) * slot_stride +
                      lane_goff
                : 0;
-        const uint32_t so = G::off(r, lch);
-        cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
-        cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
+        load_chunk(sk_a, sv_a, r, j, ok, off);
       }
     }
+    store_new_row(sk_a, sv_a, tb);
   };
 
   float o[MT][NH][4];
@@ -638,9 +731,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 }
 
 // grid: (partitions, num_kv_heads * head_groups, batch)
-template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH>
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
 __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
-  decode_cta<TQ, CK, D, NW, NSTAGE, NH>(p, blockIdx.x, blockIdx.y, blockIdx.z);
+  decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p

@@ -34,18 +34,20 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
 class DecodeStep:
     """`shared_prefix_blocks` > 0 decodes through pa_decode_shared_prefix (the
     workload's tables must all start with those blocks); `window` > 0 through
-    pa_decode_sliding_window."""
+    pa_decode_sliding_window; `fused` runs append and decode as one
+    pa_append_decode launch."""
 
     def __init__(self, w, device="cuda", partition_tokens: int = 0, stream=None,
-                 shared_prefix_blocks: int = 0, window: int = 0):
-        if shared_prefix_blocks and window:
-            raise ValueError("a shared prefix and a sliding window are separate decode paths")
+                 shared_prefix_blocks: int = 0, window: int = 0, fused: bool = False):
+        if sum(map(bool, (shared_prefix_blocks, window, fused))) > 1:
+            raise ValueError("shared prefix, sliding window and fused append are separate paths")
         self.w = w
         self.device = torch.device(device)
         self.stream = stream
         self.partition_tokens = partition_tokens
         self.shared_prefix_blocks = shared_prefix_blocks
         self.window = window
+        self.fused = fused
         dev = self.device
         cshape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
         if w.cache_dtype == "e4m3":
@@ -118,8 +120,17 @@ class DecodeStep:
                     float(self.w.scale), self.out, self.cache, self.max_context,
                     self.partition_tokens, self.workspace, self.stream)
 
+    def append_decode(self):
+        B.pa_append_decode(self.q, self.k_new, self.v_new, self.slot_mapping, self.k_cache,
+                           self.v_cache, self.block_tables, self.context_lens,
+                           float(self.w.scale), self.out, self.cache, self.max_context,
+                           self.partition_tokens, self.workspace, self.stream)
+
     def run(self):
         self.copy()
+        if self.fused:
+            self.append_decode()
+            return
         self.append()
         self.decode()
 

@@ -158,3 +158,42 @@ def test_workspace_plan(lib):
     assert lib.pa_decode_partition_tokens(256, 8192, ctypes.byref(d8)) == 1024
     assert lib.pa_decode_partition_tokens(1, 4096, ctypes.byref(d)) == 64
     assert lib.pa_decode_partition_tokens(1, 100, ctypes.byref(d)) == 64
+
+
+def test_append_decode_argument_checks(lib):
+    d = _desc()
+    call = lambda desc=d, **kw: lib.pa_append_decode(*[kw.get(k, v) for k, v in [
+        ("q", FAKE), ("k", FAKE), ("v", FAKE), ("dtype", 0), ("batch", 2), ("hq", 4),
+        ("slots", FAKE), ("kc", FAKE), ("vc", FAKE), ("desc", ctypes.byref(desc)), ("bt", FAKE),
+        ("mb", 4), ("lens", FAKE), ("maxc", 64), ("scale", 0.1), ("out", FAKE), ("pt", 0),
+        ("ws", None), ("wsb", 0), ("s", None)]])
+    assert call(k=None) == 1                  # the new token's K is required
+    assert call(slots=None) == 1
+    assert call(v=FAKE + 8) == 1              # misaligned
+    assert call(dtype=1) == 2                 # bf16 input on an fp16 cache
+    assert call(hq=3) == 1
+    assert call(batch=0) == 0                 # nothing to do
+    need = lib.pa_decode_workspace_size(2, 4, 5000, 64, ctypes.byref(d))
+    assert call(maxc=5000, pt=64) == 4        # same workspace rule as pa_decode
+    assert call(maxc=5000, pt=64, ws=FAKE, wsb=need - 1) == 4
+    # an E4M3 cache needs the inverse scales to quantise the new token
+    d8 = _desc(cache_dtype=B.PA_E4M3, k_scale=FAKE, v_scale=FAKE)
+    assert call(desc=d8) == 1
+    d8 = _desc(cache_dtype=B.PA_E4M3, k_scale=FAKE, v_scale=FAKE, k_inv_scale=FAKE,
+               v_inv_scale=FAKE + 4)
+    assert call(desc=d8) == 1
+
+
+def test_copy_blocks_layers_argument_checks(lib):
+    d = _desc()
+    arr = np.asarray([[1, 2], [3, 4]], np.int32)
+    ptrs = lambda *xs: (ctypes.c_void_p * len(xs))(*xs)
+    call = lambda ks, vs, n, pairs=arr: lib.pa_copy_blocks_layers(
+        pairs.ctypes.data_as(ctypes.c_void_p), len(pairs), ks, vs, n, ctypes.byref(d), None)
+    assert call(ptrs(FAKE, None), ptrs(FAKE, FAKE), 2) == 1        # a null layer
+    assert call(ptrs(FAKE, FAKE + 8), ptrs(FAKE, FAKE), 2) == 1    # misaligned layer
+    assert call(ptrs(FAKE), ptrs(FAKE), -1) == 1
+    assert call(ptrs(FAKE), ptrs(FAKE), 0) == 0                    # no layers: no-op
+    assert call(None, None, 2) == 1
+    bad = np.asarray([[1, 2], [2, 5]], np.int32)                   # destination is a source
+    assert call(ptrs(FAKE, FAKE), ptrs(FAKE, FAKE), 2, bad) == 1
