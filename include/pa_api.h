@@ -81,6 +81,8 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_E4M3 = 2 } pa_dtype;
                                       append) not the slot of position context_len - 1 */
 #define PA_DEVERR_PREFIX 0x8u      /* pa_decode_shared_prefix: a sequence does not start
                                       with the shared prefix blocks, or is shorter */
+#define PA_DEVERR_TIMEOUT 0x10u    /* a kernel's bounded wait for its own tensor-core
+                                      work gave up (1 s); its results are not written */
 
 /* Describes one paged KV cache (one layer's K cache and V cache). */
 typedef struct pa_cache_desc {

@@ -2,6 +2,7 @@
 // split-K planning, template dispatch and launches. All kernels of the
 // library live in this one translation unit (they share the device error
 // word).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -19,6 +20,7 @@
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
 #include "pa_prefix.cuh"
+#include "pa_prefix_umma.cuh"
 
 namespace {
 
@@ -249,7 +251,10 @@ pa::DecodeParams decode_params(const void* q, int32_t batch, int32_t num_q_heads
 // ---- shared-prefix (cascade) decode -----------------------------------------
 constexpr int kPrefixWarps = 4;   // 16 query columns per warp
 constexpr int kPrefixStages = 2;  // CTA-wide cp.async stages of one 32/64-token block
-constexpr int kPrefixChunkMax = 512;
+#ifndef PA_PREFIX_CHUNK_MAX
+#define PA_PREFIX_CHUNK_MAX 512
+#endif
+constexpr int kPrefixChunkMax = PA_PREFIX_CHUNK_MAX;  // a multiple of 64
 
 struct CascadePlan {
   int prefix_len;
@@ -262,12 +267,70 @@ struct CascadePlan {
   size_t ws_bytes;
 };
 
+// 16-bit caches with blocks of >= 8 tokens (whole 1024-byte swizzle atoms
+// per TMA box) and groups of <= 128 query heads run the prefix on the
+// tcgen05 kernel (pa_prefix_umma.cuh); the rest on the mma.sync prefix CTAs
+// of pa_cascade_kernel.
+bool cascade_uses_umma(const pa_cache_desc* cd, int64_t group) {
+  return cd->cache_dtype != PA_E4M3 && cd->block_size >= 8 && group <= pa::kUmmaRows &&
+         cd->num_blocks * cd->block_size < (int64_t{1} << 31);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// A 3-D map of 16-bit elements, 128-byte swizzle, zeros out of range.
+bool make_map_3d(CUtensorMap* m, bool bf16, const void* base, const uint64_t (&dims)[3],
+                 const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t b[3] = {box[0], box[1], box[2]};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+            const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kUmmaMaxChunks = 64;
+
 CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_context,
                               int prefix_blocks, int partition_tokens, const pa_cache_desc* cd) {
   CascadePlan pl{};
   pl.prefix_len = prefix_blocks * cd->block_size;
-  // prefix tokens per prefix CTA: the whole prefix up to kPrefixChunkMax
-  pl.chunk_tokens = std::min((pl.prefix_len + 15) / 16 * 16, kPrefixChunkMax);
+  const int64_t group = num_q_heads / cd->num_kv_heads;
+  if (cascade_uses_umma(cd, group)) {
+    // row tiles (128 / group sequences each) x KV heads x chunks of 64-token
+    // steps, about two CTAs per SM (the kernel's occupancy)
+    const int64_t seqs = pa::kUmmaRows / group;
+    const int64_t tiles = (batch + seqs - 1) / seqs * cd->num_kv_heads;
+    const int64_t steps = (pl.prefix_len + pa::kUmmaTokens - 1) / pa::kUmmaTokens;
+    const int64_t want = std::max<int64_t>(1, 2 * kNumSMs / tiles);
+    const int64_t chunks = std::min<int64_t>(std::min<int64_t>(want, steps), kUmmaMaxChunks);
+    pl.chunk_tokens = static_cast<int>((steps + chunks - 1) / chunks) * pa::kUmmaTokens;
+  } else {
+    // prefix tokens per prefix CTA: the whole prefix up to kPrefixChunkMax
+    pl.chunk_tokens = std::min((pl.prefix_len + 15) / 16 * 16, kPrefixChunkMax);
+  }
   pl.num_chunks = (pl.prefix_len + pl.chunk_tokens - 1) / pl.chunk_tokens;
   const int64_t suffix_max = std::max<int64_t>(max_context - pl.prefix_len, 0);
   pl.suffix_partition_tokens =
@@ -314,15 +377,65 @@ pa_status launch_cascade_t(const pa::DecodeParams& p, const CascadePlan& pl, cud
   return launch_reduce<TQ, D>(p, st);
 }
 
+// 16-bit caches: the tcgen05 prefix kernel, then the suffix decode in
+// cascade mode and the merge.
+template <typename TQ, int CK, int D>
+pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl,
+                                cudaStream_t st) {
+  using S = pa::UmmaSmem<D>;
+  constexpr bool kBF16 = std::is_same<TQ, __nv_bfloat16>::value;
+  auto kern = pa::pa_prefix_umma_kernel<TQ, D>;
+  if (ensure_smem(reinterpret_cast<const void*>(kern), S::kRequest) != cudaSuccess)
+    return PA_ERR_CUDA;
+  pa::UmmaGrid ug{};
+  ug.n_chunks = pl.num_chunks;
+  ug.seqs_per_tile = pa::kUmmaRows / p.group;
+  ug.n_rowtiles = (p.batch + ug.seqs_per_tile - 1) / ug.seqs_per_tile;
+  const int bs = 1 << p.bs_log2;
+  ug.unit_tokens = std::min(bs, pa::kUmmaTokens);
+  ug.num_slots = static_cast<int>(p.num_blocks * bs);
+  // q [batch][Hq][D]: box of 64 channels x the group's heads x the tile's
+  // sequences; caches [slot][Hkv][D]: box of 64 channels x 1 head x a unit
+  CUtensorMap tq, tk, tv;
+  const uint64_t row = static_cast<uint64_t>(D) * 2;
+  if (!make_map_3d(&tq, kBF16, p.q,
+                   {static_cast<uint64_t>(D), static_cast<uint64_t>(p.num_q_heads),
+                    static_cast<uint64_t>(p.batch)},
+                   {row, row * p.num_q_heads},
+                   {64u, static_cast<uint32_t>(p.group), static_cast<uint32_t>(ug.seqs_per_tile)}) ||
+      !make_map_3d(&tk, kBF16, p.k_cache,
+                   {static_cast<uint64_t>(D), static_cast<uint64_t>(p.num_kv_heads),
+                    static_cast<uint64_t>(ug.num_slots)},
+                   {row, row * p.num_kv_heads}, {64u, 1u, static_cast<uint32_t>(ug.unit_tokens)}) ||
+      !make_map_3d(&tv, kBF16, p.v_cache,
+                   {static_cast<uint64_t>(D), static_cast<uint64_t>(p.num_kv_heads),
+                    static_cast<uint64_t>(ug.num_slots)},
+                   {row, row * p.num_kv_heads}, {64u, 1u, static_cast<uint32_t>(ug.unit_tokens)}))
+    return PA_ERR_CUDA;
+  const int64_t ctas = static_cast<int64_t>(ug.n_chunks) * ug.n_rowtiles * p.num_kv_heads;
+  if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  kern<<<static_cast<unsigned>(ctas), pa::kUmmaThreads, S::kRequest, st>>>(p, ug, tq, tk, tv);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  return launch_decode_d<TQ, CK>(p, D, std::max(pl.suffix_partitions, 1), st);
+}
+
 template <typename TQ, int CK>
-pa_status launch_cascade_d(const pa::DecodeParams& p, const CascadePlan& pl, int head_dim,
-                           cudaStream_t st) {
-  const bool two = std::min(p.group, 16) > 8;
-  if (head_dim == 64)
-    return two ? launch_cascade_t<TQ, CK, 64, 2>(p, pl, st)
-               : launch_cascade_t<TQ, CK, 64, 1>(p, pl, st);
-  return two ? launch_cascade_t<TQ, CK, 128, 2>(p, pl, st)
-             : launch_cascade_t<TQ, CK, 128, 1>(p, pl, st);
+pa_status launch_cascade_d(const pa::DecodeParams& p, const CascadePlan& pl,
+                           const pa_cache_desc* cd, cudaStream_t st) {
+  const int head_dim = cd->head_dim;
+  if constexpr (CK != pa::kE4M3) {
+    if (cascade_uses_umma(cd, p.group))
+      return head_dim == 64 ? launch_cascade_umma_t<TQ, CK, 64>(p, pl, st)
+                            : launch_cascade_umma_t<TQ, CK, 128>(p, pl, st);
+  }
+  {
+    const bool two = std::min(p.group, 16) > 8;
+    if (head_dim == 64)
+      return two ? launch_cascade_t<TQ, CK, 64, 2>(p, pl, st)
+                 : launch_cascade_t<TQ, CK, 64, 1>(p, pl, st);
+    return two ? launch_cascade_t<TQ, CK, 128, 2>(p, pl, st)
+               : launch_cascade_t<TQ, CK, 128, 1>(p, pl, st);
+  }
 }
 
 }  // namespace
@@ -571,12 +684,11 @@ pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
   // sequence's table is checked against the shared prefix); then the merge.
   const cudaStream_t s = as_stream(stream);
   switch (cache->cache_dtype) {
-    case PA_F16: return launch_cascade_d<__half, pa::kF16>(p, pl, cache->head_dim, s);
-    case PA_BF16: return launch_cascade_d<__nv_bfloat16, pa::kBF16>(p, pl, cache->head_dim, s);
+    case PA_F16: return launch_cascade_d<__half, pa::kF16>(p, pl, cache, s);
+    case PA_BF16: return launch_cascade_d<__nv_bfloat16, pa::kBF16>(p, pl, cache, s);
     default:
-      return q_dtype == PA_F16
-                 ? launch_cascade_d<__half, pa::kE4M3>(p, pl, cache->head_dim, s)
-                 : launch_cascade_d<__nv_bfloat16, pa::kE4M3>(p, pl, cache->head_dim, s);
+      return q_dtype == PA_F16 ? launch_cascade_d<__half, pa::kE4M3>(p, pl, cache, s)
+                               : launch_cascade_d<__nv_bfloat16, pa::kE4M3>(p, pl, cache, s);
   }
 }
 

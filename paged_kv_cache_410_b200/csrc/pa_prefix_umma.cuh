@@ -1,0 +1,584 @@
+// Shared-prefix attention on the 5th-generation tensor cores (tcgen05 MMA,
+// accumulators in tensor memory), for 16-bit caches.
+//
+// Every sequence of the batch references the same physical blocks for the
+// first token_start tokens (KV cache article, section
+// "PagedAttention：把操作系统的老智慧搬进推理引擎": a common prompt is stored
+// once and shared). For one KV head the batch's query rows against those
+// tokens are one dense problem, so a CTA takes 128 query rows (of any
+// sequences) and one chunk of prefix tokens, 64 tokens per step:
+//   S (128 x 64, f32, TMEM)  = Q (128 x D, smem) . K_tile^T (64 x D, smem)
+//   P (128 x 64, 16-bit, smem) = 2^(S * scale * log2(e) - m)     [one row per thread]
+//   O (128 x D, f32, TMEM)  += P . V_tile (64 x D, smem)
+// and writes, per query row, the normalised partial (O / l, m, l) that the
+// split-K merge combines with the row's suffix partials.
+//
+// Shared-memory tiles use the 128-byte swizzle (rows of 128 bytes, 16-byte
+// chunk c of row r stored at chunk c ^ (r % 8), 8-row atoms of 1024 bytes);
+// a D-channel row is split into D/64 slabs of 64 channels. Q, K and P are
+// K-major operands (channels or tokens contiguous); V is read MN-major
+// straight from its token-major tile. One thread moves the tiles with TMA
+// (3-D tensor maps over q [batch][Hq][D] and the caches [slot][Hkv][D], one
+// box per cache block of >= 8 tokens, no multicast) and issues the MMAs;
+// every wait on a copy or an MMA is bounded in time.
+#pragma once
+
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "pa_decode.cuh"
+
+namespace pa {
+
+constexpr int kUmmaRows = 128;    // query rows per CTA (MMA M)
+constexpr int kUmmaTokens = 64;   // prefix tokens per step (N of S, K of P.V)
+constexpr int kUmmaSoftmaxThreads = 128;  // warps 0-3: one query row (TMEM lane) each
+constexpr int kUmmaProducerWarp = 4;      // TMA loads
+constexpr int kUmmaMmaWarp = 5;           // MMA issue
+constexpr int kUmmaThreads = 192;
+constexpr int kUmmaTmemCols = 256;  // S: 2 x 64 columns, O: up to 128 columns
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+template <int D>
+struct UmmaSmem {
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kQBytes = kSlabs * kUmmaRows * 128;
+  static constexpr int kTileSlab = kUmmaTokens * 128;  // one 64-channel slab of a K/V tile
+  static constexpr int kTileBytes = kSlabs * kTileSlab;
+  static constexpr int kPBytes = kUmmaRows * 128;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kQBytes;          // 2 stages
+  static constexpr int kV = kK + 2 * kTileBytes;   // 2 stages
+  static constexpr int kP = kV + 2 * kTileBytes;
+  static constexpr int kBytes = kP + kPBytes;      // all 1024-byte aligned pieces
+  static constexpr int kSmall = 192;               // mbarriers, TMEM address, abort flag
+  // requested: the tiles, plus slack to align them to 1024 bytes (the small
+  // items live in the slack when it has room, else after the tiles)
+  static constexpr int kRequest = kBytes + 1024;
+};
+
+struct UmmaGrid {
+  int n_chunks;
+  int n_rowtiles;
+  int seqs_per_tile;  // a tile holds seqs_per_tile x group query rows (<= 128)
+  int unit_tokens;    // tokens per TMA box: min(block_size, 64)
+  int num_slots;      // num_blocks * block_size (an out-of-range slot loads zeros)
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "  selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+// Wait for the phase with parity `parity` to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+
+// As mbar_wait, but also gives up as soon as the CTA's abort flag (shared
+// u32 at `abort`) is set, and sets it on a timeout, so that after one
+// failed wait every role drains at once.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                   uint32_t abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    uint32_t a;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];\n" : "=r"(a) : "r"(abort));
+    if (a) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      asm volatile("st.volatile.shared.u32 [%0], %1;\n" ::"r"(abort), "r"(1u) : "memory");
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// 3-D tiled TMA load of one box at coordinates (x, y, z) into shared memory,
+// completing `bar`'s transaction bytes.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%3, %4, %5}], [%2];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+// Make this thread's generic-proxy shared-memory writes (st.shared,
+// cp.async) visible to the tensor core's reads.
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+// D (TMEM) (+)= A (smem) . B (smem)^T, 16-bit inputs, f32 accumulate.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  setp.ne.b32 p, %4, 0;\n"
+      "  tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+      : "memory");
+}
+
+#define PA_R32(X)                                                                             \
+  X(0), X(1), X(2), X(3), X(4), X(5), X(6), X(7), X(8), X(9), X(10), X(11), X(12), X(13),   \
+      X(14), X(15), X(16), X(17), X(18), X(19), X(20), X(21), X(22), X(23), X(24), X(25),   \
+      X(26), X(27), X(28), X(29), X(30), X(31)
+#define PA_OUT(i) "=r"(r[i])
+#define PA_IN(i) "r"(r[i])
+
+// This warp's 32 TMEM lanes, 32 consecutive 32-bit columns from `taddr`:
+// v[j] = column j of the calling thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];\n"
+      : PA_R32(PA_OUT)
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  uint32_t r[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};\n" ::"r"(taddr),
+      PA_R32(PA_IN)
+      : "memory");
+}
+#undef PA_R32
+#undef PA_OUT
+#undef PA_IN
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading
+// and stride byte offsets (16-byte units), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of a kind::f16 MMA with f32 accumulation, M = 128:
+// A K-major, B K-major or MN-major, N columns.
+template <bool BF16, int N, bool B_MN>
+__host__ __device__ constexpr uint32_t umma_idesc() {
+  return (1u << 4) | ((BF16 ? 1u : 0u) << 7) | ((BF16 ? 1u : 0u) << 10) |
+         ((B_MN ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(kUmmaRows >> 4) << 24);
+}
+// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled slab.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// ---- the kernel ---------------------------------------------------------------
+
+// Grid: n_chunks * n_rowtiles * num_kv_heads CTAs (chunk fastest, then the
+// row tile, then the KV head) of six warps:
+//   warps 0-3  softmax: thread i owns query row i of the tile (TMEM lane i):
+//              sequence rt * seqs_per_tile + i / group, head i % group;
+//   warp 4     producer: TMA loads of Q and of the K and V tiles, two stages
+//              each, refilled as soon as the MMA that read a stage is done;
+//   warp 5     MMA issue: S(it+1) is issued before P.V(it), so the tensor
+//              core computes the next scores while the softmax warps work.
+// The roles meet only at mbarriers (full / free per stage, S full / S read,
+// P written, P.V done); every wait is bounded and a timeout aborts all roles.
+template <typename TQ, int D>
+__global__ void __launch_bounds__(kUmmaThreads, 2)
+    pa_prefix_umma_kernel(const DecodeParams p, const UmmaGrid ug,
+                          const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v) {
+  constexpr bool BF16 = std::is_same<TQ, __nv_bfloat16>::value;
+  using S = UmmaSmem<D>;
+  constexpr int SLABS = D / 64;
+  constexpr uint32_t kIdescS = umma_idesc<BF16, kUmmaTokens, false>();
+  constexpr uint32_t kIdescPV = umma_idesc<BF16, D, true>();
+
+  extern __shared__ __align__(128) uint8_t smem[];  // tiles aligned to 1024 below
+  const uint32_t raw = smem_addr(smem);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  // barriers, the TMEM address, the abort flag and the chunk's block ids: in
+  // the alignment slack when it holds the fixed part, else after the tiles
+  const uint32_t small = (base - raw >= static_cast<uint32_t>(S::kSmall)) ? raw : base + S::kBytes;
+  const uint32_t small_end = small == raw ? base : raw + S::kRequest;
+  const uint32_t bar_q = small;
+  const uint32_t bar_kfull = small + 8;    // + 8 * stage
+  const uint32_t bar_vfull = small + 24;   // + 8 * stage
+  const uint32_t bar_kfree = small + 40;   // + 8 * stage
+  const uint32_t bar_vfree = small + 56;   // + 8 * stage
+  const uint32_t bar_sfull = small + 72;   // + 8 * S buffer
+  const uint32_t bar_sfree = small + 88;   // + 8 * S buffer
+  const uint32_t bar_pfull = small + 104;
+  const uint32_t bar_pv = small + 112;
+  const uint32_t bar_done = small + 120;
+  const uint32_t tmem_slot = small + 128;
+  const uint32_t abort = small + 132;
+  const uint32_t s_bt = small + S::kSmall;
+  const uint32_t sQ = base + S::kQ;
+  const uint32_t sK = base + S::kK;
+  const uint32_t sV = base + S::kV;
+  const uint32_t sP = base + S::kP;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int chunk = blockIdx.x % ug.n_chunks;
+  const int rt = (blockIdx.x / ug.n_chunks) % ug.n_rowtiles;
+  const int hk = blockIdx.x / (ug.n_chunks * ug.n_rowtiles);
+  const int c0 = chunk * p.prefix_chunk_tokens;
+  const int c1 = min(c0 + p.prefix_chunk_tokens, p.token_start);
+  if (c0 >= c1) return;  // uniform over the CTA, before anything is allocated
+  const int nsteps = (c1 - c0 + kUmmaTokens - 1) / kUmmaTokens;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kUmmaTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == kUmmaMmaWarp * 32) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_kfull + 8 * i, 1);
+      mbar_init(bar_vfull + 8 * i, 1);
+      mbar_init(bar_kfree + 8 * i, 1);
+      mbar_init(bar_vfree + 8 * i, 1);
+      mbar_init(bar_sfull + 8 * i, 1);
+      mbar_init(bar_sfree + 8 * i, kUmmaSoftmaxThreads);
+    }
+    mbar_init(bar_pfull, kUmmaSoftmaxThreads);
+    mbar_init(bar_pv, 1);
+    mbar_init(bar_done, 1);
+    asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(abort), "r"(0u) : "memory");
+    mbar_init_fence();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  uint32_t tmem;
+  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(tmem) : "r"(tmem_slot));
+  const uint32_t tO = tmem + 2 * kUmmaTokens;
+  bool ok = true;
+
+  if (warp == kUmmaProducerWarp) {
+    // ---- producer ---------------------------------------------------------
+    // block ids of the chunk (prefix entries of sequence 0's table): staged
+    // in shared memory when they fit in the space left, else read when used
+    const int bt0 = c0 >> p.bs_log2;
+    const int nbt = ((c1 - 1) >> p.bs_log2) - bt0 + 1;
+    const bool bt_in_smem = s_bt + 4u * static_cast<uint32_t>(nbt) <= small_end;
+    if (bt_in_smem) {
+      for (int i = lane; i < nbt; i += 32) {
+        int id = __ldg(p.block_tables + bt0 + i);
+        if (id < 0 || id >= p.num_blocks) {
+          flag_error(PA_DEVERR_BLOCK_ID);
+          id = -1;
+        }
+        asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(s_bt + 4u * i), "r"(id) : "memory");
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      auto block_id = [&](int j) -> int {
+        const int bi = (j >> p.bs_log2) - bt0;
+        int id;
+        if (bt_in_smem) {
+          asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(id) : "r"(s_bt + 4u * bi));
+          return id;
+        }
+        id = __ldg(p.block_tables + bt0 + bi);
+        if (id < 0 || id >= p.num_blocks) {
+          flag_error(PA_DEVERR_BLOCK_ID);
+          id = -1;
+        }
+        return id;
+      };
+      // one tile: a box of unit_tokens rows per slab; units past the chunk
+      // (and blocks with a bad id) are read at an out-of-range slot: zeros
+      const int bs_mask = (1 << p.bs_log2) - 1;
+      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int it) {
+        mbar_arrive_expect_tx(bar, S::kTileBytes);
+        const int tb = c0 + it * kUmmaTokens;
+        for (int u0 = 0; u0 < kUmmaTokens; u0 += ug.unit_tokens) {
+          const int j = tb + u0;
+          int slot = ug.num_slots;
+          if (j < c1) {
+            const int blk = block_id(j);
+            if (blk >= 0) slot = (blk << p.bs_log2) + (j & bs_mask);
+          }
+#pragma unroll
+          for (int sl = 0; sl < SLABS; ++sl)
+            tma_load_3d(dst + sl * S::kTileSlab + u0 * 128, map, bar, sl * 64, hk, slot);
+        }
+      };
+      const int qrows = ug.seqs_per_tile * p.group;
+      mbar_arrive_expect_tx(bar_q, SLABS * qrows * 128);
+#pragma unroll
+      for (int sl = 0; sl < SLABS; ++sl)
+        tma_load_3d(sQ + sl * (kUmmaRows * 128), &tm_q, bar_q, sl * 64, hk * p.group,
+                    rt * ug.seqs_per_tile);
+      int issued = 0;  // tiles (K and V) issued so far
+      for (int it = 0; it < nsteps; ++it) {
+        const int st = it & 1;
+        const uint32_t par = static_cast<uint32_t>(((it - 2) >> 1) & 1);
+        if (it >= 2 && !mbar_wait_or_abort(bar_kfree + 8 * st, par, abort)) break;
+        load_tile(&tm_k, sK + st * S::kTileBytes, bar_kfull + 8 * st, it);
+        if (it >= 2 && !mbar_wait_or_abort(bar_vfree + 8 * st, par, abort)) {
+          issued = 2 * it + 1;
+          break;
+        }
+        load_tile(&tm_v, sV + st * S::kTileBytes, bar_vfull + 8 * st, it);
+        issued = 2 * it + 2;
+      }
+      // every issued copy has landed before the CTA can exit (normally the
+      // MMA warp has waited for all of them already)
+      for (int i = issued - 4 > 0 ? issued - 4 : 0; i < issued; ++i) {
+        const int it = i >> 1;
+        const uint32_t bar = ((i & 1) ? bar_vfull : bar_kfull) + 8 * (it & 1);
+        mbar_wait(bar, static_cast<uint32_t>((it >> 1) & 1));
+      }
+      mbar_wait(bar_q, 0);
+    }
+  } else if (warp == kUmmaMmaWarp) {
+    // ---- MMA issue --------------------------------------------------------
+    if (lane == 0) {
+      auto issue_s = [&](int i) -> bool {
+        if (!mbar_wait_or_abort(bar_kfull + 8 * (i & 1), static_cast<uint32_t>((i >> 1) & 1),
+                                abort))
+          return false;
+        if (i >= 2 && !mbar_wait_or_abort(bar_sfree + 8 * (i & 1),
+                                          static_cast<uint32_t>(((i - 2) >> 1) & 1), abort))
+          return false;
+        tc_fence_after();
+        const uint32_t kst = sK + (i & 1) * S::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a =
+              sw128_desc(sQ + (kk >> 2) * (kUmmaRows * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sw128_desc(kst + (kk >> 2) * S::kTileSlab + (kk & 3) * 32, 16, 1024);
+          umma_f16(tmem + (i & 1) * kUmmaTokens, a, b, kIdescS, kk > 0);
+        }
+        umma_commit(bar_sfull + 8 * (i & 1));
+        umma_commit(bar_kfree + 8 * (i & 1));
+        return true;
+      };
+      ok = mbar_wait_or_abort(bar_q, 0, abort) && issue_s(0);
+      for (int it = 0; ok && it < nsteps; ++it) {
+        if (it + 1 < nsteps && !issue_s(it + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_or_abort(bar_pfull, static_cast<uint32_t>(it & 1), abort) ||
+            !mbar_wait_or_abort(bar_vfull + 8 * (it & 1), static_cast<uint32_t>((it >> 1) & 1),
+                                abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t vst = sV + (it & 1) * S::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kUmmaTokens / 16; ++kk) {
+          const uint64_t a = sw128_desc(sP + kk * 32, 16, 1024);
+          const uint64_t b = sw128_desc(vst + kk * 16 * 128, S::kTileSlab, 1024);
+          umma_f16(tO, a, b, kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_pv);
+        umma_commit(bar_vfree + 8 * (it & 1));
+      }
+      // every issued MMA has completed before TMEM is released
+      umma_commit(bar_done);
+      mbar_wait(bar_done, 0);
+    }
+  } else {
+    // ---- softmax warps --------------------------------------------------------
+    const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
+    const int my_row = tid;
+    float m_run = -INFINITY;
+    float l_run = 0.f;
+    for (int it = 0; it < nsteps; ++it) {
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(bar_sfull + 8 * (it & 1),
+                                                      static_cast<uint32_t>((it >> 1) & 1), abort));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kUmmaTokens];
+      {
+        float h[32];
+        tmem_ld32(tmem + t_lane + (it & 1) * kUmmaTokens, h);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = h[j];
+        tmem_ld32(tmem + t_lane + (it & 1) * kUmmaTokens + 32, h);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[32 + j] = h[j];
+        tmem_ld_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(bar_sfree + 8 * (it & 1));
+
+      const int nvalid = c1 - (c0 + it * kUmmaTokens);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, j < nvalid ? s[j] : -INFINITY);
+      mx *= p.scale_log2;
+      const bool up = mx > m_run + kRescaleLog2;  // the first step always moves it
+      const float m_ref = up ? mx : m_run;
+      const float alpha = up ? ex2(m_run - m_ref) : 1.f;
+
+      if (it > 0) {  // P.V(it-1) done: the P tile and O are free
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_or_abort(bar_pv, static_cast<uint32_t>((it - 1) & 1), abort));
+        if (!ok) break;
+        tc_fence_after();
+        // rows whose reference max moved rescale their O row
+        if (__any_sync(0xffffffffu, up)) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            float o[32];
+            tmem_ld32(tO + t_lane + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tO + t_lane + c, o);
+          }
+          tmem_st_wait();
+        }
+      }
+
+      // P row: 64 tokens -> 8 chunks of 8 16-bit values
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 8 * c + 2 * e;
+          float p0 = ex2(fmaf(s[j], p.scale_log2, -m_ref));
+          float p1 = ex2(fmaf(s[j + 1], p.scale_log2, -m_ref));
+          p0 = j < nvalid ? p0 : 0.f;
+          p1 = j + 1 < nvalid ? p1 : 0.f;
+          sum += p0 + p1;
+          w[e] = pack2<BF16>(p0, p1);
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + sw128_off(my_row, c)),
+                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                     : "memory");
+      }
+      l_run = l_run * alpha + sum;
+      m_run = m_ref;
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_pfull);
+    }
+    if (ok) {  // the last P.V
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_or_abort(bar_pv, static_cast<uint32_t>((nsteps - 1) & 1), abort));
+      tc_fence_after();
+    }
+
+    // ---- one partial per query row -------------------------------------------
+    const int si = my_row / p.group;
+    const int bq = rt * ug.seqs_per_tile + si;
+    const bool write = ok && si < ug.seqs_per_tile && bq < p.batch;
+    const int64_t bh =
+        static_cast<int64_t>(bq) * p.num_q_heads + hk * p.group + (my_row - si * p.group);
+    const float inv = 1.f / l_run;
+    if (ok) {
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        tmem_ld32(tO + t_lane + c, o);
+        tmem_ld_wait();
+        if (write) {
+          float4* dst =
+              reinterpret_cast<float4*>(p.ws_o + (bh * p.num_partitions + chunk) * D + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(o[4 * e] * inv, o[4 * e + 1] * inv, o[4 * e + 2] * inv,
+                                 o[4 * e + 3] * inv);
+        }
+      }
+    }
+    if (write) p.ws_ml[bh * p.num_partitions + chunk] = make_float2(m_run, l_run);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  uint32_t aborted;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];\n" : "=r"(aborted) : "r"(abort));
+  if (aborted && tid == 0) flag_error(PA_DEVERR_TIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kUmmaTmemCols);
+  }
+}
+
+}  // namespace pa

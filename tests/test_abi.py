@@ -119,13 +119,21 @@ def test_shared_prefix_argument_checks(lib):
     # no shared blocks: the plain decode's workspace
     assert (lib.pa_decode_shared_prefix_workspace_size(2, 4, 5000, 0, 64, ctypes.byref(d)) ==
             lib.pa_decode_workspace_size(2, 4, 5000, 64, ctypes.byref(d)))
-    # partials: prefix chunks (up to 512 tokens each) + suffix partitions
+    # partials: prefix chunks + suffix partitions. 16-bit caches (tcgen05
+    # prefix kernel): 64-token steps split into chunks so that 128-row tiles
+    # x KV heads x chunks is about 2 CTAs per SM (296), at most 64 chunks.
+    wsz = lambda parts: (-(-(3 * 4 * parts * 64 * 4) // 256) * 256 +
+                         -(-(3 * 4 * parts * 8) // 256) * 256)
     ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 2048 + 256, 128, 64, ctypes.byref(d))
-    parts = 4 + 4
-    assert ws == -(-(3 * 4 * parts * 64 * 4) // 256) * 256 + -(-(3 * 4 * parts * 8) // 256) * 256
+    assert ws == wsz(32 + 4)    # 2 tiles -> 148 wanted, 32 steps -> 32 chunks of 64 tokens
     ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 8192 + 64, 512, 64, ctypes.byref(d))
-    parts = 16 + 1
-    assert ws == -(-(3 * 4 * parts * 64 * 4) // 256) * 256 + -(-(3 * 4 * parts * 8) // 256) * 256
+    assert ws == wsz(64 + 1)    # 128 steps, capped at 64 chunks of 128 tokens
+    # E4M3 caches (mma.sync prefix CTAs): chunks of up to 512 tokens
+    d8 = _desc(cache_dtype=B.PA_E4M3, k_scale=FAKE, v_scale=FAKE)
+    ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 2048 + 256, 128, 64, ctypes.byref(d8))
+    assert ws == wsz(4 + 4)
+    ws = lib.pa_decode_shared_prefix_workspace_size(3, 4, 8192 + 64, 512, 64, ctypes.byref(d8))
+    assert ws == wsz(16 + 1)
 
 
 def test_append_argument_checks(lib):

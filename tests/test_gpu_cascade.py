@@ -35,6 +35,13 @@ def test_70b_shaped_prefix_batch():
     run_cascade(w, w.meta["shared_prefix_blocks"])
 
 
+def test_many_row_tiles():
+    # 44 sequences x group 8 = 352 query rows per KV head: three 128-row
+    # tiles of the tensor-core prefix kernel, the last one ragged
+    w = W.llama2_70b_prefix(batch=44, prefix_len=640, max_suffix=300)
+    run_cascade(w, w.meta["shared_prefix_blocks"], check_caches=False)
+
+
 @pytest.mark.parametrize("pt", [16, 128, 0])
 def test_suffix_partitions(pt):
     w = W.llama2_70b_prefix(batch=4, max_suffix=900)
