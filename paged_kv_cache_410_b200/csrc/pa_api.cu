@@ -141,7 +141,8 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
 // Decode kernel over `grid_x` partition columns, then the split-K merge when
 // the plan has more than one partial per sequence (or always, in cascade mode).
 template <typename TQ, int CK, int D, int NH>
-pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st) {
+pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st,
+                          bool with_reduce = true) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
                       : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
@@ -153,7 +154,7 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
   dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
   kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (p.num_partitions > 1 || p.force_partials) {
+  if (with_reduce && (p.num_partitions > 1 || p.force_partials)) {
     const pa_status rs = launch_reduce<TQ, D>(p, st);
     if (rs != PA_OK) return rs;
   }
@@ -162,14 +163,14 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
 
 template <typename TQ, int CK>
 pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, int grid_x,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool with_reduce = true) {
   // query heads per CTA: the whole group up to 16; 8-head column blocks
   const bool two = std::min(p.group, 16) > 8;
   if (head_dim == 64)
-    return two ? launch_decode_t<TQ, CK, 64, 2>(p, grid_x, st)
-               : launch_decode_t<TQ, CK, 64, 1>(p, grid_x, st);
-  return two ? launch_decode_t<TQ, CK, 128, 2>(p, grid_x, st)
-             : launch_decode_t<TQ, CK, 128, 1>(p, grid_x, st);
+    return two ? launch_decode_t<TQ, CK, 64, 2>(p, grid_x, st, with_reduce)
+               : launch_decode_t<TQ, CK, 64, 1>(p, grid_x, st, with_reduce);
+  return two ? launch_decode_t<TQ, CK, 128, 2>(p, grid_x, st, with_reduce)
+             : launch_decode_t<TQ, CK, 128, 1>(p, grid_x, st, with_reduce);
 }
 
 pa_status launch_decode(const pa::DecodeParams& p, int q_dtype, const pa_cache_desc* cache,
@@ -312,6 +313,19 @@ bool make_map_3d(CUtensorMap* m, bool bf16, const void* base, const uint64_t (&d
 }
 
 constexpr int kUmmaMaxChunks = 64;
+// Row tiles of 128 query rows per prefix CTA, and K / V stages.
+#ifndef PA_UMMA_TILES
+#define PA_UMMA_TILES 2
+#endif
+#ifndef PA_UMMA_STAGES
+#define PA_UMMA_STAGES 2
+#endif
+constexpr int kUmmaTiles = PA_UMMA_TILES;
+constexpr int kUmmaStages = PA_UMMA_STAGES;
+#ifndef PA_UMMA_TARGET_CTAS
+#define PA_UMMA_TARGET_CTAS (148 * (kUmmaTiles == 1 ? 2 : 1))
+#endif
+constexpr int kUmmaTargetCtas = PA_UMMA_TARGET_CTAS;  // prefix CTAs the chunk plan aims at
 
 CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_context,
                               int prefix_blocks, int partition_tokens, const pa_cache_desc* cd) {
@@ -319,12 +333,13 @@ CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_co
   pl.prefix_len = prefix_blocks * cd->block_size;
   const int64_t group = num_q_heads / cd->num_kv_heads;
   if (cascade_uses_umma(cd, group)) {
-    // row tiles (128 / group sequences each) x KV heads x chunks of 64-token
-    // steps, about two CTAs per SM (the kernel's occupancy)
-    const int64_t seqs = pa::kUmmaRows / group;
+    // row blocks (kUmmaTiles x 128 / group sequences each) x KV heads x
+    // chunks of 64-token steps, about kUmmaTargetCtas CTAs (the kernel's
+    // occupancy on 148 SMs)
+    const int64_t seqs = kUmmaTiles * (pa::kUmmaRows / group);  // sequences per CTA
     const int64_t tiles = (batch + seqs - 1) / seqs * cd->num_kv_heads;
     const int64_t steps = (pl.prefix_len + pa::kUmmaTokens - 1) / pa::kUmmaTokens;
-    const int64_t want = std::max<int64_t>(1, 2 * kNumSMs / tiles);
+    const int64_t want = std::max<int64_t>(1, kUmmaTargetCtas / tiles);
     const int64_t chunks = std::min<int64_t>(std::min<int64_t>(want, steps), kUmmaMaxChunks);
     pl.chunk_tokens = static_cast<int>((steps + chunks - 1) / chunks) * pa::kUmmaTokens;
   } else {
@@ -377,20 +392,49 @@ pa_status launch_cascade_t(const pa::DecodeParams& p, const CascadePlan& pl, cud
   return launch_reduce<TQ, D>(p, st);
 }
 
-// 16-bit caches: the tcgen05 prefix kernel, then the suffix decode in
-// cascade mode and the merge.
+// A side stream per device on which the prefix kernel runs next to the
+// suffix decode, with the events that fork it from and join it back to the
+// caller's stream. The mutex keeps each fork / join pair together when
+// several host threads call at once.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  SideStream& ss = g_side[dev & 63];
+  if (!ss.stream) {
+    if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
+      return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
+// 16-bit caches: the tcgen05 prefix kernel on the side stream, concurrently
+// with the suffix decode (cascade mode) on the caller's stream; the merge
+// after both.
 template <typename TQ, int CK, int D>
 pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl,
                                 cudaStream_t st) {
-  using S = pa::UmmaSmem<D>;
+  using C = pa::UmmaCfg<D, kUmmaTiles, kUmmaStages>;
   constexpr bool kBF16 = std::is_same<TQ, __nv_bfloat16>::value;
-  auto kern = pa::pa_prefix_umma_kernel<TQ, D>;
-  if (ensure_smem(reinterpret_cast<const void*>(kern), S::kRequest) != cudaSuccess)
+  auto kern = pa::pa_prefix_umma_kernel<TQ, D, kUmmaTiles, kUmmaStages>;
+  if (ensure_smem(reinterpret_cast<const void*>(kern), C::kRequest) != cudaSuccess)
     return PA_ERR_CUDA;
   pa::UmmaGrid ug{};
   ug.n_chunks = pl.num_chunks;
   ug.seqs_per_tile = pa::kUmmaRows / p.group;
-  ug.n_rowtiles = (p.batch + ug.seqs_per_tile - 1) / ug.seqs_per_tile;
+  const int seqs_per_cta = kUmmaTiles * ug.seqs_per_tile;
+  ug.n_rowtiles = (p.batch + seqs_per_cta - 1) / seqs_per_cta;
   const int bs = 1 << p.bs_log2;
   ug.unit_tokens = std::min(bs, pa::kUmmaTokens);
   ug.num_slots = static_cast<int>(p.num_blocks * bs);
@@ -414,9 +458,20 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
     return PA_ERR_CUDA;
   const int64_t ctas = static_cast<int64_t>(ug.n_chunks) * ug.n_rowtiles * p.num_kv_heads;
   if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-  kern<<<static_cast<unsigned>(ctas), pa::kUmmaThreads, S::kRequest, st>>>(p, ug, tq, tk, tv);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = nullptr;
+  if (side_stream(&ss) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+    return PA_ERR_CUDA;
+  kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kRequest, ss->stream>>>(p, ug, tq, tk, tv);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  return launch_decode_d<TQ, CK>(p, D, std::max(pl.suffix_partitions, 1), st);
+  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return PA_ERR_CUDA;
+  const pa_status rs = launch_decode_d<TQ, CK>(p, D, std::max(pl.suffix_partitions, 1), st,
+                                               /*with_reduce=*/false);
+  if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return PA_ERR_CUDA;
+  if (rs != PA_OK) return rs;
+  return launch_reduce<TQ, D>(p, st);
 }
 
 template <typename TQ, int CK>

@@ -773,6 +773,48 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
   const bool active = lane < D / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
+  if (WPR == 1) {
+    // at most 16 partials (the launch picks WPR = 1 only then): every load
+    // is issued before any is used, so a row costs one memory round trip
+    // after its length
+    if (work) {
+      const float2* ml = p.ws_ml + row * p.num_partitions;
+      const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
+      const float2 mine = lane < nparts ? ml[lane] : make_float2(-INFINITY, 0.f);
+      // unconditional loads (indexes clamped to the row's partials and to
+      // the row's D / 4 lanes; the clamped copies get weight 0 or are not
+      // stored), so that they are all issued together
+      const int lc = active ? lane : D / 4 - 1;
+      float4 x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        x[i] = po[static_cast<int64_t>(min(i, nparts - 1)) * (D / 4) + lc];
+      float M = mine.x;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float wl = lane < nparts ? mine.y * ex2(mine.x - M) : 0.f;
+      wsum = wl;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float w = __shfl_sync(0xffffffffu, wl, i);
+        acc.x += w * x[i].x;
+        acc.y += w * x[i].y;
+        acc.z += w * x[i].z;
+        acc.w += w * x[i].w;
+      }
+      if (active) {
+        TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
+        const float inv = 1.f / wsum;
+        out[0] = from_f32<TQ>(acc.x * inv);
+        out[1] = from_f32<TQ>(acc.y * inv);
+        out[2] = from_f32<TQ>(acc.z * inv);
+        out[3] = from_f32<TQ>(acc.w * inv);
+      }
+    }
+    return;
+  }
   if (work) {
     const float2* ml = p.ws_ml + row * p.num_partitions;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
@@ -795,17 +837,6 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
         acc.w += w * x.w;
       }
     }
-  }
-  if (WPR == 1) {
-    if (work && active) {
-      TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
-      const float inv = 1.f / wsum;
-      out[0] = from_f32<TQ>(acc.x * inv);
-      out[1] = from_f32<TQ>(acc.y * inv);
-      out[2] = from_f32<TQ>(acc.z * inv);
-      out[3] = from_f32<TQ>(acc.w * inv);
-    }
-    return;
   }
   if (active) s_acc[warp][lane] = acc;
   if (lane == 0) s_wsum[warp] = wsum;

@@ -31,37 +31,48 @@
 
 namespace pa {
 
-constexpr int kUmmaRows = 128;    // query rows per CTA (MMA M)
+constexpr int kUmmaRows = 128;    // query rows per MMA tile (M)
 constexpr int kUmmaTokens = 64;   // prefix tokens per step (N of S, K of P.V)
-constexpr int kUmmaSoftmaxThreads = 128;  // warps 0-3: one query row (TMEM lane) each
-constexpr int kUmmaProducerWarp = 4;      // TMA loads
-constexpr int kUmmaMmaWarp = 5;           // MMA issue
-constexpr int kUmmaThreads = 192;
-constexpr int kUmmaTmemCols = 256;  // S: 2 x 64 columns, O: up to 128 columns
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
-template <int D>
-struct UmmaSmem {
+// A CTA holds NT row tiles of 128 query rows, all against the same K / V
+// stages (so that each stage serves NT * 128 rows), NSTAGE stages deep.
+// Warps 0 .. 4*NT-1 run the softmax (warp w: tile w / 4, TMEM lanes
+// 32 * (w % 4) ..), then one TMA producer warp and one MMA warp.
+template <int D, int NT, int NSTAGE>
+struct UmmaCfg {
+  static constexpr int kSoftmaxWarps = 4 * NT;
+  static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  // TMEM columns: S of tile t, buffer b at t*128 + b*64; O of tile t at
+  // NT*128 + t*D; allocated as a power of two
+  static constexpr int kOCol = NT * 2 * kUmmaTokens;
+  static constexpr int kColsUsed = kOCol + NT * D;
+  static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
+  // shared memory: 1024-byte aligned pieces
   static constexpr int kSlabs = D / 64;
-  static constexpr int kQBytes = kSlabs * kUmmaRows * 128;
-  static constexpr int kTileSlab = kUmmaTokens * 128;  // one 64-channel slab of a K/V tile
-  static constexpr int kTileBytes = kSlabs * kTileSlab;
-  static constexpr int kPBytes = kUmmaRows * 128;
+  static constexpr int kQTile = kSlabs * kUmmaRows * 128;     // one row tile of Q
+  static constexpr int kTileSlab = kUmmaTokens * 128;          // one slab of a K/V stage
+  static constexpr int kTileBytes = kSlabs * kTileSlab;        // one K or V stage
+  static constexpr int kPTile = kUmmaRows * 128;               // P of one row tile
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;          // 2 stages
-  static constexpr int kV = kK + 2 * kTileBytes;   // 2 stages
-  static constexpr int kP = kV + 2 * kTileBytes;
-  static constexpr int kBytes = kP + kPBytes;      // all 1024-byte aligned pieces
-  static constexpr int kSmall = 192;               // mbarriers, TMEM address, abort flag
-  // requested: the tiles, plus slack to align them to 1024 bytes (the small
+  static constexpr int kK = kQ + NT * kQTile;
+  static constexpr int kV = kK + NSTAGE * kTileBytes;
+  static constexpr int kP = kV + NSTAGE * kTileBytes;
+  static constexpr int kBytes = kP + NT * kPTile;
+  static constexpr int kSmall = 256;  // mbarriers, TMEM address, abort flag
+  // requested: the tiles plus slack to align them to 1024 bytes (the small
   // items live in the slack when it has room, else after the tiles)
   static constexpr int kRequest = kBytes + 1024;
+  static_assert(kColsUsed <= 512, "TMEM holds 512 columns");
 };
 
 struct UmmaGrid {
   int n_chunks;
-  int n_rowtiles;
-  int seqs_per_tile;  // a tile holds seqs_per_tile x group query rows (<= 128)
+  int n_rowtiles;     // CTAs per (KV head, chunk): NT row tiles each
+  int seqs_per_tile;  // a row tile holds seqs_per_tile x group query rows (<= 128)
   int unit_tokens;    // tokens per TMA box: min(block_size, 64)
   int num_slots;      // num_blocks * block_size (an out-of-range slot loads zeros)
 };
@@ -245,24 +256,25 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 // ---- the kernel ---------------------------------------------------------------
 
 // Grid: n_chunks * n_rowtiles * num_kv_heads CTAs (chunk fastest, then the
-// row tile, then the KV head) of six warps:
-//   warps 0-3  softmax: thread i owns query row i of the tile (TMEM lane i):
-//              sequence rt * seqs_per_tile + i / group, head i % group;
-//   warp 4     producer: TMA loads of Q and of the K and V tiles, two stages
-//              each, refilled as soon as the MMA that read a stage is done;
-//   warp 5     MMA issue: S(it+1) is issued before P.V(it), so the tensor
+// row block, then the KV head). Roles (UmmaCfg):
+//   softmax warps: thread i of tile t owns query row i of the tile (TMEM
+//              lane i): sequence (rt * NT + t) * seqs_per_tile + i / group,
+//              head i % group of the KV head's group;
+//   producer:  TMA loads of Q and of the K and V stages, each stage refilled
+//              as soon as the MMAs that read it are done;
+//   MMA warp:  S(it+1) of all tiles is issued before P.V(it), so the tensor
 //              core computes the next scores while the softmax warps work.
 // The roles meet only at mbarriers (full / free per stage, S full / S read,
 // P written, P.V done); every wait is bounded and a timeout aborts all roles.
-template <typename TQ, int D>
-__global__ void __launch_bounds__(kUmmaThreads, 2)
+template <typename TQ, int D, int NT, int NSTAGE>
+__global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     pa_prefix_umma_kernel(const DecodeParams p, const UmmaGrid ug,
                           const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v) {
   constexpr bool BF16 = std::is_same<TQ, __nv_bfloat16>::value;
-  using S = UmmaSmem<D>;
-  constexpr int SLABS = D / 64;
+  using C = UmmaCfg<D, NT, NSTAGE>;
+  constexpr int SLABS = C::kSlabs;
   constexpr uint32_t kIdescS = umma_idesc<BF16, kUmmaTokens, false>();
   constexpr uint32_t kIdescPV = umma_idesc<BF16, D, true>();
 
@@ -271,25 +283,26 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   const uint32_t base = (raw + 1023u) & ~1023u;
   // barriers, the TMEM address, the abort flag and the chunk's block ids: in
   // the alignment slack when it holds the fixed part, else after the tiles
-  const uint32_t small = (base - raw >= static_cast<uint32_t>(S::kSmall)) ? raw : base + S::kBytes;
-  const uint32_t small_end = small == raw ? base : raw + S::kRequest;
+  const uint32_t small = (base - raw >= static_cast<uint32_t>(C::kSmall)) ? raw : base + C::kBytes;
+  const uint32_t small_end = small == raw ? base : raw + C::kRequest;
   const uint32_t bar_q = small;
-  const uint32_t bar_kfull = small + 8;    // + 8 * stage
-  const uint32_t bar_vfull = small + 24;   // + 8 * stage
-  const uint32_t bar_kfree = small + 40;   // + 8 * stage
-  const uint32_t bar_vfree = small + 56;   // + 8 * stage
-  const uint32_t bar_sfull = small + 72;   // + 8 * S buffer
-  const uint32_t bar_sfree = small + 88;   // + 8 * S buffer
-  const uint32_t bar_pfull = small + 104;
-  const uint32_t bar_pv = small + 112;
-  const uint32_t bar_done = small + 120;
-  const uint32_t tmem_slot = small + 128;
-  const uint32_t abort = small + 132;
-  const uint32_t s_bt = small + S::kSmall;
-  const uint32_t sQ = base + S::kQ;
-  const uint32_t sK = base + S::kK;
-  const uint32_t sV = base + S::kV;
-  const uint32_t sP = base + S::kP;
+  const uint32_t bar_kfull = small + 8;      // + 8 * stage (<= 4 stages)
+  const uint32_t bar_vfull = small + 40;     // + 8 * stage
+  const uint32_t bar_kfree = small + 72;     // + 8 * stage
+  const uint32_t bar_vfree = small + 104;    // + 8 * stage
+  const uint32_t bar_sfull = small + 136;    // + 8 * S buffer
+  const uint32_t bar_sfree = small + 152;    // + 8 * S buffer
+  const uint32_t bar_pfull = small + 168;
+  const uint32_t bar_pv = small + 176;
+  const uint32_t bar_done = small + 184;
+  const uint32_t tmem_slot = small + 192;
+  const uint32_t abort = small + 196;
+  const uint32_t s_bt = small + C::kSmall;
+  const uint32_t sQ = base + C::kQ;
+  const uint32_t sK = base + C::kK;
+  const uint32_t sV = base + C::kV;
+  const uint32_t sP = base + C::kP;
+  static_assert(NSTAGE >= 2 && NSTAGE <= 4, "stages");
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -301,22 +314,26 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   const int c1 = min(c0 + p.prefix_chunk_tokens, p.token_start);
   if (c0 >= c1) return;  // uniform over the CTA, before anything is allocated
   const int nsteps = (c1 - c0 + kUmmaTokens - 1) / kUmmaTokens;
+  // use i of a stage-indexed barrier completes once per NSTAGE steps
+  auto stage_parity = [](int it) { return static_cast<uint32_t>((it / NSTAGE) & 1); };
 
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kUmmaTmemCols);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  if (tid == kUmmaMmaWarp * 32) {
+  if (tid == C::kMmaWarp * 32) {
     mbar_init(bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(bar_kfull + 8 * i, 1);
       mbar_init(bar_vfull + 8 * i, 1);
       mbar_init(bar_kfree + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
-      mbar_init(bar_sfull + 8 * i, 1);
-      mbar_init(bar_sfree + 8 * i, kUmmaSoftmaxThreads);
     }
-    mbar_init(bar_pfull, kUmmaSoftmaxThreads);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull + 8 * i, 1);
+      mbar_init(bar_sfree + 8 * i, C::kSoftmaxThreads);
+    }
+    mbar_init(bar_pfull, C::kSoftmaxThreads);
     mbar_init(bar_pv, 1);
     mbar_init(bar_done, 1);
     asm volatile("st.shared.u32 [%0], %1;\n" ::"r"(abort), "r"(0u) : "memory");
@@ -327,10 +344,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   tc_fence_after();
   uint32_t tmem;
   asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(tmem) : "r"(tmem_slot));
-  const uint32_t tO = tmem + 2 * kUmmaTokens;
   bool ok = true;
 
-  if (warp == kUmmaProducerWarp) {
+  if (warp == C::kProducerWarp) {
     // ---- producer ---------------------------------------------------------
     // block ids of the chunk (prefix entries of sequence 0's table): staged
     // in shared memory when they fit in the space left, else read when used
@@ -349,6 +365,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
     }
     __syncwarp();
     if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
       auto block_id = [&](int j) -> int {
         const int bi = (j >> p.bs_log2) - bt0;
         int id;
@@ -367,7 +385,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       // (and blocks with a bad id) are read at an out-of-range slot: zeros
       const int bs_mask = (1 << p.bs_log2) - 1;
       auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int it) {
-        mbar_arrive_expect_tx(bar, S::kTileBytes);
+        mbar_arrive_expect_tx(bar, C::kTileBytes);
         const int tb = c0 + it * kUmmaTokens;
         for (int u0 = 0; u0 < kUmmaTokens; u0 += ug.unit_tokens) {
           const int j = tb + u0;
@@ -378,58 +396,62 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
           }
 #pragma unroll
           for (int sl = 0; sl < SLABS; ++sl)
-            tma_load_3d(dst + sl * S::kTileSlab + u0 * 128, map, bar, sl * 64, hk, slot);
+            tma_load_3d(dst + sl * C::kTileSlab + u0 * 128, map, bar, sl * 64, hk, slot);
         }
       };
       const int qrows = ug.seqs_per_tile * p.group;
-      mbar_arrive_expect_tx(bar_q, SLABS * qrows * 128);
+      mbar_arrive_expect_tx(bar_q, NT * SLABS * qrows * 128);
 #pragma unroll
-      for (int sl = 0; sl < SLABS; ++sl)
-        tma_load_3d(sQ + sl * (kUmmaRows * 128), &tm_q, bar_q, sl * 64, hk * p.group,
-                    rt * ug.seqs_per_tile);
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int sl = 0; sl < SLABS; ++sl)
+          tma_load_3d(sQ + t * C::kQTile + sl * (kUmmaRows * 128), &tm_q, bar_q, sl * 64,
+                      hk * p.group, (rt * NT + t) * ug.seqs_per_tile);
       int issued = 0;  // tiles (K and V) issued so far
       for (int it = 0; it < nsteps; ++it) {
-        const int st = it & 1;
-        const uint32_t par = static_cast<uint32_t>(((it - 2) >> 1) & 1);
-        if (it >= 2 && !mbar_wait_or_abort(bar_kfree + 8 * st, par, abort)) break;
-        load_tile(&tm_k, sK + st * S::kTileBytes, bar_kfull + 8 * st, it);
-        if (it >= 2 && !mbar_wait_or_abort(bar_vfree + 8 * st, par, abort)) {
+        const int st = it % NSTAGE;
+        const uint32_t par = stage_parity(it - NSTAGE);
+        if (it >= NSTAGE && !mbar_wait_or_abort(bar_kfree + 8 * st, par, abort)) break;
+        load_tile(&tm_k, sK + st * C::kTileBytes, bar_kfull + 8 * st, it);
+        if (it >= NSTAGE && !mbar_wait_or_abort(bar_vfree + 8 * st, par, abort)) {
           issued = 2 * it + 1;
           break;
         }
-        load_tile(&tm_v, sV + st * S::kTileBytes, bar_vfull + 8 * st, it);
+        load_tile(&tm_v, sV + st * C::kTileBytes, bar_vfull + 8 * st, it);
         issued = 2 * it + 2;
       }
       // every issued copy has landed before the CTA can exit (normally the
       // MMA warp has waited for all of them already)
-      for (int i = issued - 4 > 0 ? issued - 4 : 0; i < issued; ++i) {
+      for (int i = issued - 2 * NSTAGE > 0 ? issued - 2 * NSTAGE : 0; i < issued; ++i) {
         const int it = i >> 1;
-        const uint32_t bar = ((i & 1) ? bar_vfull : bar_kfull) + 8 * (it & 1);
-        mbar_wait(bar, static_cast<uint32_t>((it >> 1) & 1));
+        const uint32_t bar = ((i & 1) ? bar_vfull : bar_kfull) + 8 * (it % NSTAGE);
+        mbar_wait(bar, stage_parity(it));
       }
       mbar_wait(bar_q, 0);
     }
-  } else if (warp == kUmmaMmaWarp) {
+  } else if (warp == C::kMmaWarp) {
     // ---- MMA issue --------------------------------------------------------
     if (lane == 0) {
       auto issue_s = [&](int i) -> bool {
-        if (!mbar_wait_or_abort(bar_kfull + 8 * (i & 1), static_cast<uint32_t>((i >> 1) & 1),
-                                abort))
+        if (!mbar_wait_or_abort(bar_kfull + 8 * (i % NSTAGE), stage_parity(i), abort))
           return false;
         if (i >= 2 && !mbar_wait_or_abort(bar_sfree + 8 * (i & 1),
                                           static_cast<uint32_t>(((i - 2) >> 1) & 1), abort))
           return false;
         tc_fence_after();
-        const uint32_t kst = sK + (i & 1) * S::kTileBytes;
+        const uint32_t kst = sK + (i % NSTAGE) * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a =
-              sw128_desc(sQ + (kk >> 2) * (kUmmaRows * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sw128_desc(kst + (kk >> 2) * S::kTileSlab + (kk & 3) * 32, 16, 1024);
-          umma_f16(tmem + (i & 1) * kUmmaTokens, a, b, kIdescS, kk > 0);
-        }
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sw128_desc(
+                sQ + t * C::kQTile + (kk >> 2) * (kUmmaRows * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t b =
+                sw128_desc(kst + (kk >> 2) * C::kTileSlab + (kk & 3) * 32, 16, 1024);
+            umma_f16(tmem + t * 2 * kUmmaTokens + (i & 1) * kUmmaTokens, a, b, kIdescS, kk > 0);
+          }
         umma_commit(bar_sfull + 8 * (i & 1));
-        umma_commit(bar_kfree + 8 * (i & 1));
+        umma_commit(bar_kfree + 8 * (i % NSTAGE));
         return true;
       };
       ok = mbar_wait_or_abort(bar_q, 0, abort) && issue_s(0);
@@ -439,21 +461,22 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
           break;
         }
         if (!mbar_wait_or_abort(bar_pfull, static_cast<uint32_t>(it & 1), abort) ||
-            !mbar_wait_or_abort(bar_vfull + 8 * (it & 1), static_cast<uint32_t>((it >> 1) & 1),
-                                abort)) {
+            !mbar_wait_or_abort(bar_vfull + 8 * (it % NSTAGE), stage_parity(it), abort)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t vst = sV + (it & 1) * S::kTileBytes;
+        const uint32_t vst = sV + (it % NSTAGE) * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kUmmaTokens / 16; ++kk) {
-          const uint64_t a = sw128_desc(sP + kk * 32, 16, 1024);
-          const uint64_t b = sw128_desc(vst + kk * 16 * 128, S::kTileSlab, 1024);
-          umma_f16(tO, a, b, kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+          for (int kk = 0; kk < kUmmaTokens / 16; ++kk) {
+            const uint64_t a = sw128_desc(sP + t * C::kPTile + kk * 32, 16, 1024);
+            const uint64_t b = sw128_desc(vst + kk * 16 * 128, C::kTileSlab, 1024);
+            umma_f16(tmem + C::kOCol + t * D, a, b, kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
+          }
         umma_commit(bar_pv);
-        umma_commit(bar_vfree + 8 * (it & 1));
+        umma_commit(bar_vfree + 8 * (it % NSTAGE));
       }
       // every issued MMA has completed before TMEM is released
       umma_commit(bar_done);
@@ -461,8 +484,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
     }
   } else {
     // ---- softmax warps --------------------------------------------------------
-    const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-    const int my_row = tid;
+    const int tile = warp >> 2;
+    const int my_row = tid & (kUmmaRows - 1);  // row within the tile = TMEM lane
+    const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t_lane + tile * 2 * kUmmaTokens;
+    const uint32_t tO = tmem + t_lane + C::kOCol + tile * D;
+    const uint32_t sPt = sP + tile * C::kPTile;
     float m_run = -INFINITY;
     float l_run = 0.f;
     for (int it = 0; it < nsteps; ++it) {
@@ -473,10 +500,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       float s[kUmmaTokens];
       {
         float h[32];
-        tmem_ld32(tmem + t_lane + (it & 1) * kUmmaTokens, h);
+        tmem_ld32(tS + (it & 1) * kUmmaTokens, h);
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = h[j];
-        tmem_ld32(tmem + t_lane + (it & 1) * kUmmaTokens + 32, h);
+        tmem_ld32(tS + (it & 1) * kUmmaTokens + 32, h);
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[32 + j] = h[j];
         tmem_ld_wait();
@@ -493,6 +520,22 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
       const float m_ref = up ? mx : m_run;
       const float alpha = up ? ex2(m_run - m_ref) : 1.f;
 
+      // P row (64 tokens, packed in pairs), computed while P.V(it-1) may
+      // still be running
+      uint32_t pw[kUmmaTokens / 2];
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kUmmaTokens; j += 2) {
+        float p0 = ex2(fmaf(s[j], p.scale_log2, -m_ref));
+        float p1 = ex2(fmaf(s[j + 1], p.scale_log2, -m_ref));
+        p0 = j < nvalid ? p0 : 0.f;
+        p1 = j + 1 < nvalid ? p1 : 0.f;
+        sum += p0 + p1;
+        pw[j / 2] = pack2<BF16>(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      m_run = m_ref;
+
       if (it > 0) {  // P.V(it-1) done: the P tile and O are free
         ok = __all_sync(0xffffffffu,
                         mbar_wait_or_abort(bar_pv, static_cast<uint32_t>((it - 1) & 1), abort));
@@ -503,37 +546,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
             float o[32];
-            tmem_ld32(tO + t_lane + c, o);
+            tmem_ld32(tO + c, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tO + t_lane + c, o);
+            tmem_st32(tO + c, o);
           }
           tmem_st_wait();
         }
       }
-
-      // P row: 64 tokens -> 8 chunks of 8 16-bit values
-      float sum = 0.f;
+      // P tile (128-byte swizzled, K-major): 8 chunks of 8 values
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 8 * c + 2 * e;
-          float p0 = ex2(fmaf(s[j], p.scale_log2, -m_ref));
-          float p1 = ex2(fmaf(s[j + 1], p.scale_log2, -m_ref));
-          p0 = j < nvalid ? p0 : 0.f;
-          p1 = j + 1 < nvalid ? p1 : 0.f;
-          sum += p0 + p1;
-          w[e] = pack2<BF16>(p0, p1);
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sP + sw128_off(my_row, c)),
-                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+      for (int c = 0; c < 8; ++c)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sPt + sw128_off(my_row, c)),
+                     "r"(pw[4 * c]), "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3])
                      : "memory");
-      }
-      l_run = l_run * alpha + sum;
-      m_run = m_ref;
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar_pfull);
@@ -546,7 +573,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 
     // ---- one partial per query row -------------------------------------------
     const int si = my_row / p.group;
-    const int bq = rt * ug.seqs_per_tile + si;
+    const int bq = (rt * NT + tile) * ug.seqs_per_tile + si;
     const bool write = ok && si < ug.seqs_per_tile && bq < p.batch;
     const int64_t bh =
         static_cast<int64_t>(bq) * p.num_q_heads + hk * p.group + (my_row - si * p.group);
@@ -555,7 +582,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         float o[32];
-        tmem_ld32(tO + t_lane + c, o);
+        tmem_ld32(tO + c, o);
         tmem_ld_wait();
         if (write) {
           float4* dst =
@@ -577,7 +604,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 2)
   if (aborted && tid == 0) flag_error(PA_DEVERR_TIMEOUT);
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kUmmaTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
