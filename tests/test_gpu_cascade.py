@@ -93,3 +93,17 @@ def test_sequences_not_starting_with_the_prefix_are_flagged():
                               step.context_lens, float(w.scale), step.out, step.cache,
                               step.max_context, 4, workspace=step.workspace)
     assert step.device_errors() == 0
+
+
+def test_dirty_workspace_and_repeat():
+    # the prefix and suffix partials live in the caller's workspace: garbage
+    # left in it changes nothing, and repeated calls agree bit for bit
+    w = W.llama2_70b_prefix(batch=20, prefix_len=512, max_suffix=700)
+    step, got = run_cascade(w, w.meta["shared_prefix_blocks"], check_caches=False)
+    first = step.out.clone()
+    for fill in (0x00, 0x5A, 0xFF):
+        step.workspace.fill_(fill)
+        step.decode()
+        torch.cuda.synchronize()
+        assert step.device_errors() == 0
+        assert torch.equal(step.out, first)

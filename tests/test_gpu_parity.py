@@ -176,3 +176,22 @@ def test_device_bounds_are_reported_not_faulted():
     after_other[s1] = before.reshape(-1, 4, 64)[s1]
     assert np.array_equal(after_other, before.reshape(-1, 4, 64))  # only the valid token landed
     assert step.device_errors() == 0  # the word was cleared
+
+
+def test_split_k_merge_with_a_dirty_workspace():
+    # the split-K partials live in the caller's workspace: a reused workspace
+    # full of garbage must give the same result as a fresh one
+    w = W.llama2_7b(batch=3, min_len=2000, max_len=3000)
+    step = DecodeStep(w, "cuda", partition_tokens=64)
+    assert step.workspace is not None
+    step.workspace.fill_(0xA5)
+    step.run()
+    torch.cuda.synchronize()
+    assert step.device_errors() == 0
+    first = step.out.clone()
+    step.workspace.fill_(0xFF)
+    step.decode()
+    torch.cuda.synchronize()
+    assert torch.equal(step.out, first)
+    _, _, want = oracle_step(w)
+    assert max_abs_err(step.out_f64(), want) <= TOL["f16"]
