@@ -367,61 +367,68 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
       asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
-      auto block_id = [&](int j) -> int {
-        const int bi = (j >> p.bs_log2) - bt0;
-        int id;
-        if (bt_in_smem) {
-          asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(id) : "r"(s_bt + 4u * bi));
-          return id;
-        }
-        id = __ldg(p.block_tables + bt0 + bi);
-        if (id < 0 || id >= p.num_blocks) {
-          flag_error(PA_DEVERR_BLOCK_ID);
-          id = -1;
-        }
+    }
+    auto block_id = [&](int j) -> int {
+      const int bi = (j >> p.bs_log2) - bt0;
+      int id;
+      if (bt_in_smem) {
+        asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(id) : "r"(s_bt + 4u * bi));
         return id;
-      };
-      // one tile: a box of unit_tokens rows per slab; units past the chunk
-      // (and blocks with a bad id) are read at an out-of-range slot: zeros
-      const int bs_mask = (1 << p.bs_log2) - 1;
-      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int it) {
-        mbar_arrive_expect_tx(bar, C::kTileBytes);
-        const int tb = c0 + it * kUmmaTokens;
-        for (int u0 = 0; u0 < kUmmaTokens; u0 += ug.unit_tokens) {
-          const int j = tb + u0;
-          int slot = ug.num_slots;
-          if (j < c1) {
-            const int blk = block_id(j);
-            if (blk >= 0) slot = (blk << p.bs_log2) + (j & bs_mask);
-          }
-#pragma unroll
-          for (int sl = 0; sl < SLABS; ++sl)
-            tma_load_3d(dst + sl * C::kTileSlab + u0 * 128, map, bar, sl * 64, hk, slot);
-        }
-      };
-      const int qrows = ug.seqs_per_tile * p.group;
-      mbar_arrive_expect_tx(bar_q, NT * SLABS * qrows * 128);
-#pragma unroll
-      for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int sl = 0; sl < SLABS; ++sl)
-          tma_load_3d(sQ + t * C::kQTile + sl * (kUmmaRows * 128), &tm_q, bar_q, sl * 64,
-                      hk * p.group, (rt * NT + t) * ug.seqs_per_tile);
-      int issued = 0;  // tiles (K and V) issued so far
-      for (int it = 0; it < nsteps; ++it) {
-        const int st = it % NSTAGE;
-        const uint32_t par = stage_parity(it - NSTAGE);
-        if (it >= NSTAGE && !mbar_wait_or_abort(bar_kfree + 8 * st, par, abort)) break;
-        load_tile(&tm_k, sK + st * C::kTileBytes, bar_kfull + 8 * st, it);
-        if (it >= NSTAGE && !mbar_wait_or_abort(bar_vfree + 8 * st, par, abort)) {
-          issued = 2 * it + 1;
-          break;
-        }
-        load_tile(&tm_v, sV + st * C::kTileBytes, bar_vfull + 8 * st, it);
-        issued = 2 * it + 2;
       }
-      // every issued copy has landed before the CTA can exit (normally the
-      // MMA warp has waited for all of them already)
+      id = __ldg(p.block_tables + bt0 + bi);
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PA_DEVERR_BLOCK_ID);
+        id = -1;
+      }
+      return id;
+    };
+    // One tile: a box of unit_tokens rows per (unit, slab); the warp's lanes
+    // issue the boxes together, lane i the box (unit i / SLABS, slab
+    // i % SLABS). Units past the chunk (and blocks with a bad id) are read at
+    // an out-of-range slot: zeros.
+    const int bs_mask = (1 << p.bs_log2) - 1;
+    const int nbox = (kUmmaTokens / ug.unit_tokens) * SLABS;  // <= 16
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int it) {
+      if (lane == 0) mbar_arrive_expect_tx(bar, C::kTileBytes);
+      if (lane < nbox) {
+        const int u0 = (lane / SLABS) * ug.unit_tokens;
+        const int sl = lane % SLABS;
+        const int j = c0 + it * kUmmaTokens + u0;
+        int slot = ug.num_slots;
+        if (j < c1) {
+          const int blk = block_id(j);
+          if (blk >= 0) slot = (blk << p.bs_log2) + (j & bs_mask);
+        }
+        tma_load_3d(dst + sl * C::kTileSlab + u0 * 128, map, bar, sl * 64, hk, slot);
+      }
+    };
+    const int qrows = ug.seqs_per_tile * p.group;
+    if (lane == 0) mbar_arrive_expect_tx(bar_q, NT * SLABS * qrows * 128);
+    if (lane < NT * SLABS) {
+      const int t = lane / SLABS;
+      const int sl = lane % SLABS;
+      tma_load_3d(sQ + t * C::kQTile + sl * (kUmmaRows * 128), &tm_q, bar_q, sl * 64,
+                  hk * p.group, (rt * NT + t) * ug.seqs_per_tile);
+    }
+    int issued = 0;  // tiles (K and V) issued so far
+    for (int it = 0; it < nsteps; ++it) {
+      const int st = it % NSTAGE;
+      const uint32_t par = stage_parity(it - NSTAGE);
+      if (it >= NSTAGE &&
+          !__all_sync(0xffffffffu, mbar_wait_or_abort(bar_kfree + 8 * st, par, abort)))
+        break;
+      load_tile(&tm_k, sK + st * C::kTileBytes, bar_kfull + 8 * st, it);
+      if (it >= NSTAGE &&
+          !__all_sync(0xffffffffu, mbar_wait_or_abort(bar_vfree + 8 * st, par, abort))) {
+        issued = 2 * it + 1;
+        break;
+      }
+      load_tile(&tm_v, sV + st * C::kTileBytes, bar_vfull + 8 * st, it);
+      issued = 2 * it + 2;
+    }
+    // every issued copy has landed before the CTA can exit (normally the
+    // MMA warp has waited for all of them already)
+    if (lane == 0) {
       for (int i = issued - 2 * NSTAGE > 0 ? issued - 2 * NSTAGE : 0; i < issued; ++i) {
         const int it = i >> 1;
         const uint32_t bar = ((i & 1) ? bar_vfull : bar_kfull) + 8 * (it % NSTAGE);
