@@ -520,9 +520,11 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const int64_t new_row = (static_cast<int64_t>(b) * p.num_kv_heads + hk) * D;  // elements
   const TQ* knew = has_new ? reinterpret_cast<const TQ*>(p.k_new) + new_row : nullptr;
   const TQ* vnew = has_new ? reinterpret_cast<const TQ*>(p.v_new) + new_row : nullptr;
-  if (has_new && part == nparts - 1 && hgrp == 0) {
-    // store it in the cache, as pa_append_kv would; the slot must be the one
-    // the table gives position L - 1
+  // Store the new token in the cache, as pa_append_kv would; the slot must
+  // be the one the table gives position L - 1. Done by the CTA of the last
+  // partition (first head group); nothing in this launch reads the slot.
+  auto store_new_token = [&]() {
+    if (!(has_new && part == nparts - 1 && hgrp == 0)) return;
     const int64_t slot = p.slot_mapping[b];
     const int64_t expect =
         (static_cast<int64_t>(p.block_tables[static_cast<int64_t>(b) * p.max_blocks_per_seq +
@@ -545,7 +547,10 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src + 8 * ch);
       }
     }
-  }
+  };
+  // a 16-bit row is a plain copy: done up front; the E4M3 quantisation is
+  // done at the end of the CTA, where it adds no register pressure to the loop
+  if constexpr (FUSED && CK != kE4M3) store_new_token();
 
   // One 16-byte chunk of row r: from the cache at `off`, or from the fused
   // new token (16-bit: the same bytes by cp.async; E4M3: no copy here, the
@@ -728,6 +733,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
             make_float2(r_stat[2 * row], r_stat[2 * row + 1]);
     }
   }
+  if constexpr (FUSED && CK == kE4M3) store_new_token();
 }
 
 // grid: (partitions, num_kv_heads * head_groups, batch)
