@@ -297,19 +297,30 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// A 3-D map of 16-bit elements, 128-byte swizzle, zeros out of range.
-bool make_map_3d(CUtensorMap* m, bool bf16, const void* base, const uint64_t (&dims)[3],
-                 const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
+// A tiled map with 128-byte swizzle, zeros out of range (loads) and
+// clipping (stores). Strides in bytes for dimensions 1 .. rank-1.
+template <int R>
+bool make_map(CUtensorMap* m, CUtensorMapDataType type, const void* base,
+              const uint64_t (&dims)[R], const uint64_t (&strides)[R - 1],
+              const uint32_t (&box)[R]) {
   const EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
-  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  cuuint64_t st[2] = {strides[0], strides[1]};
-  cuuint32_t b[3] = {box[0], box[1], box[2]};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-            const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t d[R], st[R - 1];
+  cuuint32_t b[R], es[R];
+  for (int i = 0; i < R; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i < R - 1) st[i] = strides[i];
+  }
+  return fn(m, type, R, const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map_3d(CUtensorMap* m, bool bf16, const void* base, const uint64_t (&dims)[3],
+                 const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
+  return make_map<3>(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     base, dims, strides, box);
 }
 
 constexpr int kUmmaMaxChunks = 64;
@@ -456,6 +467,18 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
                     static_cast<uint64_t>(ug.num_slots)},
                    {row, row * p.num_kv_heads}, {64u, 1u, static_cast<uint32_t>(ug.unit_tokens)}))
     return PA_ERR_CUDA;
+  // partial outputs ws_o [batch][Hq][partition][D] f32: box of 32 channels x
+  // 1 partition x the group's heads x the tile's sequences
+  CUtensorMap to;
+  const uint64_t prow = static_cast<uint64_t>(D) * 4;
+  const uint64_t np = static_cast<uint64_t>(p.num_partitions);
+  if (!make_map<4>(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_o,
+                   {static_cast<uint64_t>(D), np, static_cast<uint64_t>(p.num_q_heads),
+                    static_cast<uint64_t>(p.batch)},
+                   {prow, prow * np, prow * np * p.num_q_heads},
+                   {32u, 1u, static_cast<uint32_t>(p.group),
+                    static_cast<uint32_t>(ug.seqs_per_tile)}))
+    return PA_ERR_CUDA;
   const int64_t ctas = static_cast<int64_t>(ug.n_chunks) * ug.n_rowtiles * p.num_kv_heads;
   if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_side_mu);
@@ -464,7 +487,8 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
   if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
       cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
     return PA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kRequest, ss->stream>>>(p, ug, tq, tk, tv);
+  kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kRequest, ss->stream>>>(p, ug, tq, tk, tv,
+                                                                             to);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return PA_ERR_CUDA;
   const pa_status rs = launch_decode_d<TQ, CK>(p, D, std::max(pl.suffix_partitions, 1), st,

@@ -149,6 +149,36 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 4-D tiled TMA store of one box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], "
+      "[%1];\n" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+// Barrier `id` over `count` threads that also returns whether `pred` held in
+// all of them.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      "  .reg .pred p, q;\n"
+      "  setp.ne.u32 p, %1, 0;\n"
+      "  bar.red.and.pred q, %2, %3, p;\n"
+      "  selp.u32 %0, 1, 0, q;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot),
                "r"(ncols)
@@ -271,7 +301,8 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     pa_prefix_umma_kernel(const DecodeParams p, const UmmaGrid ug,
                           const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v) {
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o) {
   constexpr bool BF16 = std::is_same<TQ, __nv_bfloat16>::value;
   using C = UmmaCfg<D, NT, NSTAGE>;
   constexpr int SLABS = C::kSlabs;
@@ -579,27 +610,42 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     }
 
     // ---- one partial per query row -------------------------------------------
+    // Rows are staged in shared memory (free now: every MMA has completed)
+    // as D/32 quarters of 128-byte rows with the 128-byte swizzle (conflict
+    // free), then one thread per tile stores the tile with D/32 TMA stores
+    // into ws_o viewed as [batch][Hq][partition][D] (rows past the batch or
+    // the tile's sequences are clipped by the map / the box).
     const int si = my_row / p.group;
     const int bq = (rt * NT + tile) * ug.seqs_per_tile + si;
     const bool write = ok && si < ug.seqs_per_tile && bq < p.batch;
     const int64_t bh =
         static_cast<int64_t>(bq) * p.num_q_heads + hk * p.group + (my_row - si * p.group);
     const float inv = 1.f / l_run;
+    constexpr int kQuarter = kUmmaRows * 128;  // 32 channels of 128 rows
+    const uint32_t stage = base + tile * (D / 32) * kQuarter;
     if (ok) {
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         float o[32];
         tmem_ld32(tO + c, o);
         tmem_ld_wait();
-        if (write) {
-          float4* dst =
-              reinterpret_cast<float4*>(p.ws_o + (bh * p.num_partitions + chunk) * D + c);
+        const uint32_t row = stage + (c / 32) * kQuarter + my_row * 128;
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(o[4 * e] * inv, o[4 * e + 1] * inv, o[4 * e + 2] * inv,
-                                 o[4 * e + 3] * inv);
-        }
+        for (int e = 0; e < 8; ++e)
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                           row + ((e ^ (my_row & 7)) << 4)),
+                       "f"(o[4 * e] * inv), "f"(o[4 * e + 1] * inv), "f"(o[4 * e + 2] * inv),
+                       "f"(o[4 * e + 3] * inv)
+                       : "memory");
       }
+    }
+    fence_async_smem();
+    if (bar_and(1 + tile, kUmmaRows, ok) && my_row == 0) {
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q)
+        tma_store_4d(&tm_o, stage + q * kQuarter, 32 * q, chunk, hk * p.group,
+                     (rt * NT + tile) * ug.seqs_per_tile);
+      bulk_commit_and_wait();
     }
     if (write) p.ws_ml[bh * p.num_partitions + chunk] = make_float2(m_run, l_run);
   }
