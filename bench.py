@@ -319,8 +319,8 @@ def run_ours(args):
         decode_name = f"pa_decode_sliding_window (window {args.window}; main + split-K reduce)"
     elif spb:
         prefix_len = spb * w.block_size
-        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
-            w.batch, max(w.max_context - prefix_len, 0), step.cache)
+        plan_pt = args.partition_tokens or B.pa_decode_shared_prefix_partition_tokens(
+            w.batch, w.num_q_heads, w.max_context, spb, step.cache)
         n_parts = max(1, math.ceil((w.max_context - prefix_len) / plan_pt))
         decode_launches = 3  # prefix kernel, suffix kernel, merge
         decode_name = "pa_decode_shared_prefix (prefix + suffix + merge kernels)"

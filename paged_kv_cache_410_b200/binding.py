@@ -30,7 +30,8 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_version", "pa_decode_static_workspace",
             "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
             "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
-            "pa_append_decode", "pa_copy_blocks_layers"]
+            "pa_append_decode", "pa_copy_blocks_layers",
+            "pa_decode_shared_prefix_partition_tokens"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -97,6 +98,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_copy_blocks_layers.argtypes = [P, i32, ctypes.POINTER(P), ctypes.POINTER(P), i32, D,
                                           P]
     lib.pa_copy_blocks_layers.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_partition_tokens.argtypes = [i32, i32, i32, i32, D]
+    lib.pa_decode_shared_prefix_partition_tokens.restype = i32
     _lib = lib
     return lib
 
@@ -219,6 +222,14 @@ def pa_decode_shared_prefix_workspace_size(batch, num_q_heads, max_context, pref
     return int(lib.pa_decode_shared_prefix_workspace_size(batch, num_q_heads, max_context,
                                                           prefix_blocks, partition_tokens,
                                                           ctypes.byref(d)))
+
+
+def pa_decode_shared_prefix_partition_tokens(batch, num_q_heads, max_context, prefix_blocks,
+                                             cache: PagedCache) -> int:
+    lib = load_library()
+    d = cache.desc()
+    return int(lib.pa_decode_shared_prefix_partition_tokens(batch, num_q_heads, max_context,
+                                                            prefix_blocks, ctypes.byref(d)))
 
 
 def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, scale, out,

@@ -361,6 +361,13 @@ CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_co
   const int64_t suffix_max = std::max<int64_t>(max_context - pl.prefix_len, 0);
   pl.suffix_partition_tokens =
       partition_tokens > 0 ? partition_tokens : auto_partition(batch, suffix_max, cd);
+  if (partition_tokens == 0 && cascade_uses_umma(cd, group)) {
+    // every row already merges the prefix partials: take twice the plain
+    // decode's partition while that still leaves two CTAs per SM
+    const int64_t pt2 = 2 * static_cast<int64_t>(pl.suffix_partition_tokens);
+    if (batch * cd->num_kv_heads * ((suffix_max + pt2 - 1) / pt2) >= 2 * kNumSMs)
+      pl.suffix_partition_tokens = static_cast<int>(pt2);
+  }
   pl.suffix_partitions =
       static_cast<int>((suffix_max + pl.suffix_partition_tokens - 1) / pl.suffix_partition_tokens);
   pl.num_partitions = pl.num_chunks + pl.suffix_partitions;
@@ -702,6 +709,18 @@ pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch
   p.num_partitions = pl.num_partitions;
   p.window = window;
   return launch_decode(p, q_dtype, cache, as_stream(stream));
+}
+
+int32_t pa_decode_shared_prefix_partition_tokens(int32_t batch, int32_t num_q_heads,
+                                                 int32_t max_context, int32_t prefix_blocks,
+                                                 const pa_cache_desc* cache) {
+  int bs_log2 = 0;
+  if (check_cache(cache, &bs_log2) != PA_OK || batch <= 0 || num_q_heads <= 0 ||
+      max_context < 0 || prefix_blocks < 0 || num_q_heads % cache->num_kv_heads != 0)
+    return 0;
+  if (prefix_blocks == 0) return auto_partition(batch, max_context, cache);
+  return make_cascade_plan(batch, num_q_heads, max_context, prefix_blocks, 0, cache)
+      .suffix_partition_tokens;
 }
 
 size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads,

@@ -205,3 +205,21 @@ def test_copy_blocks_layers_argument_checks(lib):
     assert call(None, None, 2) == 1
     bad = np.asarray([[1, 2], [2, 5]], np.int32)                   # destination is a source
     assert call(ptrs(FAKE, FAKE), ptrs(FAKE, FAKE), 2, bad) == 1
+
+
+def test_shared_prefix_partition_rule(lib):
+    # 70B-shaped cascade (batch 128, 64 / 8 heads, 2000-token prefix, suffixes
+    # up to 2049): twice the plain rule's 512 tokens; E4M3 keeps the plain rule
+    d = _desc(num_blocks=20000, num_kv_heads=8, head_dim=128, cache_dtype=B.PA_BF16)
+    assert lib.pa_decode_partition_tokens(128, 2049, ctypes.byref(d)) == 512
+    assert lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d)) == 1024
+    assert (lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 0, ctypes.byref(d)) ==
+            lib.pa_decode_partition_tokens(128, 4049, ctypes.byref(d)))
+    # a small batch keeps the plain rule (doubling would leave < 2 CTAs per SM)
+    small = lib.pa_decode_partition_tokens(2, 2049, ctypes.byref(d))
+    assert lib.pa_decode_shared_prefix_partition_tokens(2, 64, 4049, 125, ctypes.byref(d)) == small
+    d8 = _desc(num_blocks=20000, num_kv_heads=8, head_dim=128, cache_dtype=B.PA_E4M3,
+               k_scale=FAKE, v_scale=FAKE)
+    assert (lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d8)) ==
+            lib.pa_decode_partition_tokens(128, 2049, ctypes.byref(d8)))
+    assert lib.pa_decode_shared_prefix_partition_tokens(0, 64, 4049, 125, ctypes.byref(d)) == 0
