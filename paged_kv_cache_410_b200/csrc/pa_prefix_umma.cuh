@@ -550,9 +550,15 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
       mbar_arrive(bar_sfree + 8 * (it & 1));
 
       const int nvalid = c1 - (c0 + it * kUmmaTokens);
+      const bool full = nvalid >= kUmmaTokens;  // every step but a chunk's ragged last one
       float mx = -INFINITY;
+      if (full) {
 #pragma unroll
-      for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, j < nvalid ? s[j] : -INFINITY);
+        for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, s[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, j < nvalid ? s[j] : -INFINITY);
+      }
       mx *= p.scale_log2;
       const bool up = mx > m_run + kRescaleLog2;  // the first step always moves it
       const float m_ref = up ? mx : m_run;
@@ -562,14 +568,23 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
       // still be running
       uint32_t pw[kUmmaTokens / 2];
       float sum = 0.f;
+      auto expo = [&](int j) { return ex2(fmaf(s[j], p.scale_log2, -m_ref)); };
+      if (full) {
 #pragma unroll
-      for (int j = 0; j < kUmmaTokens; j += 2) {
-        float p0 = ex2(fmaf(s[j], p.scale_log2, -m_ref));
-        float p1 = ex2(fmaf(s[j + 1], p.scale_log2, -m_ref));
-        p0 = j < nvalid ? p0 : 0.f;
-        p1 = j + 1 < nvalid ? p1 : 0.f;
-        sum += p0 + p1;
-        pw[j / 2] = pack2<BF16>(p0, p1);
+        for (int j = 0; j < kUmmaTokens; j += 2) {
+          const float p0 = expo(j);
+          const float p1 = expo(j + 1);
+          sum += p0 + p1;
+          pw[j / 2] = pack2<BF16>(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kUmmaTokens; j += 2) {
+          const float p0 = j < nvalid ? expo(j) : 0.f;
+          const float p1 = j + 1 < nvalid ? expo(j + 1) : 0.f;
+          sum += p0 + p1;
+          pw[j / 2] = pack2<BF16>(p0, p1);
+        }
       }
       l_run = l_run * alpha + sum;
       m_run = m_ref;
