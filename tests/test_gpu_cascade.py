@@ -107,3 +107,37 @@ def test_dirty_workspace_and_repeat():
         torch.cuda.synchronize()
         assert step.device_errors() == 0
         assert torch.equal(step.out, first)
+
+
+def test_cuda_graph_capture_and_replay():
+    # the 16-bit cascade forks onto the library's side stream and joins back:
+    # captured from the caller's stream it must replay to the eager result
+    w = W.llama2_70b_prefix(batch=16, prefix_len=512, max_suffix=600)
+    step, _ = run_cascade(w, w.meta["shared_prefix_blocks"], check_caches=False)
+    eager = step.out.clone()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step.decode()  # warm up on the capture stream (plans, smem attributes)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    step.out.zero_()
+    with torch.cuda.graph(graph):
+        step.decode()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert step.device_errors() == 0
+    assert torch.equal(step.out, eager)
+    # plain split-K decode of the same batch, captured too
+    plain = DecodeStep(w, "cuda", partition_tokens=64)
+    plain.run()
+    torch.cuda.synchronize()
+    want = plain.out.clone()
+    g2 = torch.cuda.CUDAGraph()
+    plain.out.zero_()
+    with torch.cuda.graph(g2):
+        plain.decode()
+    g2.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(plain.out, want)
