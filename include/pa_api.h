@@ -202,10 +202,10 @@ pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch
                                    size_t workspace_bytes, void* stream);
 
 /* Tokens per suffix partition that pa_decode_shared_prefix uses for these
- * sizes when called with partition_tokens == 0 (for 16-bit caches twice
- * pa_decode's choice while that still gives two CTAs per SM: every row
- * already merges the prefix partials). 0 for invalid sizes. Pure host
- * function. */
+ * sizes when called with partition_tokens == 0 (for 16-bit caches up to
+ * four times pa_decode's choice while that still gives two CTAs per SM:
+ * every row already merges the prefix partials). 0 for invalid sizes. Pure
+ * host function. */
 int32_t pa_decode_shared_prefix_partition_tokens(int32_t batch, int32_t num_q_heads,
                                                  int32_t max_context, int32_t prefix_blocks,
                                                  const pa_cache_desc* cache);

@@ -362,11 +362,13 @@ CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_co
   pl.suffix_partition_tokens =
       partition_tokens > 0 ? partition_tokens : auto_partition(batch, suffix_max, cd);
   if (partition_tokens == 0 && cascade_uses_umma(cd, group)) {
-    // every row already merges the prefix partials: take twice the plain
-    // decode's partition while that still leaves two CTAs per SM
-    const int64_t pt2 = 2 * static_cast<int64_t>(pl.suffix_partition_tokens);
-    if (batch * cd->num_kv_heads * ((suffix_max + pt2 - 1) / pt2) >= 2 * kNumSMs)
+    // every row already merges the prefix partials: take up to four times
+    // the plain decode's partition while that still leaves two CTAs per SM
+    for (int i = 0; i < 2; ++i) {
+      const int64_t pt2 = 2 * static_cast<int64_t>(pl.suffix_partition_tokens);
+      if (batch * cd->num_kv_heads * ((suffix_max + pt2 - 1) / pt2) < 2 * kNumSMs) break;
       pl.suffix_partition_tokens = static_cast<int>(pt2);
+    }
   }
   pl.suffix_partitions =
       static_cast<int>((suffix_max + pl.suffix_partition_tokens - 1) / pl.suffix_partition_tokens);

@@ -209,10 +209,13 @@ def test_copy_blocks_layers_argument_checks(lib):
 
 def test_shared_prefix_partition_rule(lib):
     # 70B-shaped cascade (batch 128, 64 / 8 heads, 2000-token prefix, suffixes
-    # up to 2049): twice the plain rule's 512 tokens; E4M3 keeps the plain rule
+    # up to 2049): four times the plain rule's 512 tokens; E4M3 keeps the plain rule
     d = _desc(num_blocks=20000, num_kv_heads=8, head_dim=128, cache_dtype=B.PA_BF16)
     assert lib.pa_decode_partition_tokens(128, 2049, ctypes.byref(d)) == 512
-    assert lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d)) == 1024
+    assert lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d)) == 2048
+    # 16 sequences: doubling once keeps >= 2 CTAs per SM (16 x 8 x 3 = 384), twice does not
+    assert lib.pa_decode_partition_tokens(16, 2049, ctypes.byref(d)) == 512
+    assert lib.pa_decode_shared_prefix_partition_tokens(16, 64, 4049, 125, ctypes.byref(d)) == 1024
     assert (lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 0, ctypes.byref(d)) ==
             lib.pa_decode_partition_tokens(128, 4049, ctypes.byref(d)))
     # a small batch keeps the plain rule (doubling would leave < 2 CTAs per SM)
