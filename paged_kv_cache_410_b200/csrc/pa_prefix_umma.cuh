@@ -5,8 +5,9 @@
 // first token_start tokens (KV cache article, section
 // "PagedAttention：把操作系统的老智慧搬进推理引擎": a common prompt is stored
 // once and shared). For one KV head the batch's query rows against those
-// tokens are one dense problem, so a CTA takes 128 query rows (of any
-// sequences) and one chunk of prefix tokens, 64 tokens per step:
+// tokens are one dense problem, so a CTA takes NT tiles of 128 query rows
+// (of any sequences) and one chunk of prefix tokens, 64 tokens per step;
+// per tile:
 //   S (128 x 64, f32, TMEM)  = Q (128 x D, smem) . K_tile^T (64 x D, smem)
 //   P (128 x 64, 16-bit, smem) = 2^(S * scale * log2(e) - m)     [one row per thread]
 //   O (128 x D, f32, TMEM)  += P . V_tile (64 x D, smem)
@@ -17,10 +18,12 @@
 // chunk c of row r stored at chunk c ^ (r % 8), 8-row atoms of 1024 bytes);
 // a D-channel row is split into D/64 slabs of 64 channels. Q, K and P are
 // K-major operands (channels or tokens contiguous); V is read MN-major
-// straight from its token-major tile. One thread moves the tiles with TMA
-// (3-D tensor maps over q [batch][Hq][D] and the caches [slot][Hkv][D], one
-// box per cache block of >= 8 tokens, no multicast) and issues the MMAs;
-// every wait on a copy or an MMA is bounded in time.
+// straight from its token-major tile. A producer warp moves the tiles with
+// TMA (3-D tensor maps over q [batch][Hq][D] and the caches [slot][Hkv][D],
+// one box per cache block of >= 8 tokens and 64-channel slab, no
+// multicast), one thread of an MMA warp issues the MMAs, and the partial
+// outputs leave through TMA stores; every wait on a copy or an MMA is
+// bounded in time.
 #pragma once
 
 #include <cuda.h>
