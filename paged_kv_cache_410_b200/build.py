@@ -53,6 +53,25 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+BENCH_BM = os.path.join(HERE, "pa_block_manager_bench")
+BENCH_BM_SOURCES = [os.path.join(HERE, "csrc", "pa_block_manager_bench.cpp"),
+                    os.path.join(HERE, "csrc", "pa_block_manager.cpp")]
+
+
+def build_block_manager_bench(force: bool = False) -> str:
+    """The host benchmark of the block manager (a plain C++ program)."""
+    deps = BENCH_BM_SOURCES + [os.path.join(ROOT, "include", "pa_block_manager.h")]
+    if (not force and os.path.exists(BENCH_BM) and
+            all(os.path.getmtime(d) <= os.path.getmtime(BENCH_BM) for d in deps)):
+        return BENCH_BM
+    cxx = os.environ.get("CXX", "g++")
+    cmd = [cxx, "-O2", "-std=c++17", "-I", os.path.join(ROOT, "include"), "-o", BENCH_BM + ".tmp",
+           *BENCH_BM_SOURCES]
+    subprocess.run(cmd, check=True)
+    os.replace(BENCH_BM + ".tmp", BENCH_BM)
+    return BENCH_BM
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)

@@ -192,3 +192,20 @@ def test_invalid_calls():
     with pytest.raises(BM.BlockManagerError) as e:
         bm.block_tables([2], 2)
     assert e.value.code == BM.ERR_CAPACITY
+
+
+def test_host_benchmark_runs():
+    # the block manager's host benchmark (serving-step loop) builds and
+    # reports sensible numbers on a small case
+    import json
+    import subprocess
+    from paged_kv_cache_410_b200 import build
+    exe = build.build_block_manager_bench()
+    out = subprocess.run([exe, "16", "100", "256", "16", "16", "10"], check=True,
+                         capture_output=True, text=True).stdout
+    r = json.loads(out.strip().splitlines()[-1])
+    assert r["batch"] == 16 and r["steps"] == 100
+    # every request after the first reuses the 256-token system prompt (16 blocks)
+    assert r["prompt_tokens_cached"] == 15 * 256
+    assert r["forks"] == 40 and r["cow_pairs"] > 0
+    assert r["append_ns_per_token"] > 0 and r["step_us"] > 0
