@@ -9,6 +9,7 @@
 #include <memory>
 #include <new>
 #include <set>
+#include <algorithm>
 #include <unordered_map>
 #include <utility>
 #include <vector>
@@ -339,17 +340,22 @@ int32_t pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, i
   if (!bm || n_seqs < 0 || max_blocks_per_seq <= 0 ||
       (n_seqs > 0 && (!seq_ids || !block_tables || !context_lens)))
     return PA_BM_ERR_INVALID;
+  // check every sequence before writing anything
+  std::vector<const Seq*> rows(static_cast<size_t>(n_seqs));
   for (int32_t i = 0; i < n_seqs; ++i) {
     auto it = bm->seqs.find(seq_ids[i]);
     if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
     if (static_cast<int64_t>(it->second.blocks.size()) > max_blocks_per_seq)
       return PA_BM_ERR_CAPACITY;
+    rows[static_cast<size_t>(i)] = &it->second;
   }
   for (int32_t i = 0; i < n_seqs; ++i) {
-    const Seq& s = bm->seqs.find(seq_ids[i])->second;
+    const Seq& s = *rows[static_cast<size_t>(i)];
     int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks_per_seq;
-    for (int32_t k = 0; k < max_blocks_per_seq; ++k)
-      row[k] = k < static_cast<int32_t>(s.blocks.size()) ? static_cast<int32_t>(s.blocks[k]) : 0;
+    const int32_t n = static_cast<int32_t>(s.blocks.size());
+    const int64_t* src = s.blocks.data();
+    for (int32_t k = 0; k < n; ++k) row[k] = static_cast<int32_t>(src[k]);
+    std::fill(row + n, row + max_blocks_per_seq, 0);
     context_lens[i] = s.length;
   }
   return PA_BM_OK;
