@@ -277,6 +277,14 @@ pa_status pa_copy_blocks_layers(const int32_t* pairs_host, int32_t num_pairs,
                                 void* const* k_caches, void* const* v_caches, int32_t num_layers,
                                 const pa_cache_desc* cache, void* stream);
 
+/* Test hook for the failure path of pa_decode_shared_prefix's tensor-core
+ * prefix kernel (16-bit caches). While on (process-wide), that kernel's MMA
+ * warp issues nothing: its softmax warps' waits run out after their 1 s
+ * limit, every role of the CTA drains, no partial is written and the device
+ * error word gets PA_DEVERR_TIMEOUT; the context stays usable. Off by
+ * default; not for production calls. */
+void pa_testing_withhold_prefix_scores(int32_t on);
+
 /* Synchronise `stream`, then read and clear the current device's error
  * word into *flags (PA_DEVERR_* bits). Returns PA_ERR_DEVICE_BOUNDS when
  * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure. */

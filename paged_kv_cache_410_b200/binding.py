@@ -23,6 +23,7 @@ PA_OK = 0
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_CUDA",
           4: "PA_ERR_WORKSPACE", 5: "PA_ERR_DEVICE_BOUNDS"}
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_PREFIX = 0x1, 0x2, 0x4, 0x8
+DEVERR_TIMEOUT = 0x10
 
 # names of every symbol include/pa_api.h declares
 EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tokens",
@@ -31,7 +32,7 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
             "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
             "pa_append_decode", "pa_copy_blocks_layers",
-            "pa_decode_shared_prefix_partition_tokens"]
+            "pa_decode_shared_prefix_partition_tokens", "pa_testing_withhold_prefix_scores"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -100,6 +101,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_copy_blocks_layers.restype = ctypes.c_int
     lib.pa_decode_shared_prefix_partition_tokens.argtypes = [i32, i32, i32, i32, D]
     lib.pa_decode_shared_prefix_partition_tokens.restype = i32
+    lib.pa_testing_withhold_prefix_scores.argtypes = [i32]
+    lib.pa_testing_withhold_prefix_scores.restype = None
     _lib = lib
     return lib
 
@@ -319,6 +322,12 @@ def pa_copy_blocks_layers(pairs, k_caches, v_caches, cache: PagedCache, stream=N
     rc = lib.pa_copy_blocks_layers(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], kp, vp, n,
                                    ctypes.byref(d), _stream(stream))
     _check(rc, "pa_copy_blocks_layers")
+
+
+def pa_testing_withhold_prefix_scores(on: bool):
+    """Test hook (process-wide): the shared-prefix tensor-core kernel's MMA
+    warp issues nothing, so its bounded waits run out (PA_DEVERR_TIMEOUT)."""
+    load_library().pa_testing_withhold_prefix_scores(1 if on else 0)
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -423,6 +423,7 @@ struct SideStream {
 };
 std::mutex g_side_mu;
 SideStream g_side[64];
+int g_withhold_prefix_scores = 0;  // pa_testing_withhold_prefix_scores
 
 cudaError_t side_stream(SideStream** out) {
   int dev = 0;
@@ -452,6 +453,7 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
     return PA_ERR_CUDA;
   pa::UmmaGrid ug{};
   ug.n_chunks = pl.num_chunks;
+  ug.withhold_scores = g_withhold_prefix_scores;
   ug.seqs_per_tile = pa::kUmmaRows / p.group;
   const int seqs_per_cta = kUmmaTiles * ug.seqs_per_tile;
   ug.n_rowtiles = (p.batch + seqs_per_cta - 1) / seqs_per_cta;
@@ -543,6 +545,11 @@ const char* pa_status_string(int32_t s) {
 }
 
 int32_t pa_version(void) { return 100; }
+
+void pa_testing_withhold_prefix_scores(int32_t on) {
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  g_withhold_prefix_scores = on != 0;
+}
 
 pa_status pa_append_kv(const void* k, const void* v, int32_t in_dtype, int64_t num_tokens,
                        const int64_t* slot_mapping, void* k_cache, void* v_cache,

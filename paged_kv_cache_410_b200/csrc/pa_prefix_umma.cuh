@@ -76,6 +76,8 @@ struct UmmaGrid {
   int n_chunks;
   int n_rowtiles;     // CTAs per (KV head, chunk): NT row tiles each
   int seqs_per_tile;  // a row tile holds seqs_per_tile x group query rows (<= 128)
+  int withhold_scores;  // test hook: the MMA warp issues nothing, so the softmax
+                        // warps' bounded waits run out (PA_DEVERR_TIMEOUT)
   int unit_tokens;    // tokens per TMA box: min(block_size, 64)
   int num_slots;      // num_blocks * block_size (an out-of-range slot loads zeros)
 };
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
         umma_commit(bar_kfree + 8 * (i % NSTAGE));
         return true;
       };
-      ok = mbar_wait_or_abort(bar_q, 0, abort) && issue_s(0);
+      ok = mbar_wait_or_abort(bar_q, 0, abort) && !ug.withhold_scores && issue_s(0);
       for (int it = 0; ok && it < nsteps; ++it) {
         if (it + 1 < nsteps && !issue_s(it + 1)) {
           ok = false;

@@ -141,3 +141,27 @@ def test_cuda_graph_capture_and_replay():
     g2.replay()
     torch.cuda.synchronize()
     assert torch.equal(plain.out, want)
+
+
+def test_prefix_wait_timeout_is_reported_and_recoverable():
+    # the test hook withholds the tensor-core prefix kernel's scores: its
+    # softmax warps' bounded waits run out (1 s), the CTA drains and the
+    # device error word reports PA_DEVERR_TIMEOUT; afterwards the context
+    # is still usable and a normal call matches the oracle
+    w = W.custom_shared_prefix(128, [3, 20], num_q_heads=8, num_kv_heads=1, head_dim=128,
+                               block_size=16, dtype="bf16", seed=3)
+    step = DecodeStep(w, "cuda", shared_prefix_blocks=w.meta["shared_prefix_blocks"])
+    step.copy()
+    step.append()
+    B.pa_testing_withhold_prefix_scores(1)
+    try:
+        step.decode()
+        torch.cuda.synchronize()
+        assert step.device_errors() & B.DEVERR_TIMEOUT
+    finally:
+        B.pa_testing_withhold_prefix_scores(0)
+    step.decode()
+    torch.cuda.synchronize()
+    assert step.device_errors() == 0
+    _, _, want = oracle_step(w)
+    assert max_abs_err(step.out_f64(), want) <= TOL["bf16"]
