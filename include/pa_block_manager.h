@@ -99,6 +99,22 @@ int32_t pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, i
                            int32_t max_blocks_per_seq, int32_t* block_tables,
                            int32_t* context_lens);
 
+/* Incremental form of pa_bm_block_tables for a caller that keeps the same
+ * arrays from step to step: only the rows whose block list changed since
+ * this call last wrote them are rewritten (a new block, a copy-on-write
+ * replacement, or another sequence in the row); every length is written.
+ * row_versions [n_seqs] (caller-owned, read and written) holds the stamp of
+ * the table each row holds; stamps are never 0 and unique across the
+ * manager's sequences, so zero-filled row_versions make the first call write
+ * every row, and moving sequences between rows needs no reset. Reset
+ * row_versions to 0 after writing the arrays by other means or changing
+ * max_blocks_per_seq. *rows_written (may be NULL) receives the number of
+ * rows rewritten. Errors as pa_bm_block_tables, with nothing written. */
+int32_t pa_bm_block_tables_update(const pa_block_manager* bm, const int64_t* seq_ids,
+                                  int32_t n_seqs, int32_t max_blocks_per_seq,
+                                  int32_t* block_tables, int32_t* context_lens,
+                                  uint64_t* row_versions, int32_t* rows_written);
+
 #ifdef __cplusplus
 }
 #endif

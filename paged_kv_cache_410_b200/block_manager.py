@@ -13,7 +13,7 @@ OK, ERR_INVALID, ERR_NO_BLOCKS, ERR_CAPACITY = 0, -1, -2, -3
 EXPORTED = ["pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_num_cached_blocks",
             "pa_bm_block_refcount", "pa_bm_add_sequence", "pa_bm_append_token", "pa_bm_fork",
             "pa_bm_free_sequence", "pa_bm_release_before", "pa_bm_sequence_length",
-            "pa_bm_slots", "pa_bm_block_tables"]
+            "pa_bm_slots", "pa_bm_block_tables", "pa_bm_block_tables_update"]
 
 _declared = False
 
@@ -50,6 +50,8 @@ def _lib():
         lib.pa_bm_slots.restype = i32
         lib.pa_bm_block_tables.argtypes = [P, P, i32, i32, P, P]
         lib.pa_bm_block_tables.restype = i32
+        lib.pa_bm_block_tables_update.argtypes = [P, P, i32, i32, P, P, P, ctypes.POINTER(i32)]
+        lib.pa_bm_block_tables_update.restype = i32
         _declared = True
     return lib
 
@@ -145,3 +147,25 @@ class BlockManager:
                                           lens.ctypes.data_as(ctypes.c_void_p))
         _ok(rc, "pa_bm_block_tables")
         return tables, lens
+
+    def block_tables_update(self, seq_ids, tables: np.ndarray, lens: np.ndarray,
+                            row_versions: np.ndarray) -> int:
+        """Rewrites, in place, the rows of `tables` (int32 [n, max_blocks]) whose block list
+        changed since they were last written; writes every entry of `lens` (int32 [n]);
+        `row_versions` (uint64 [n], zeros at first) tracks what each row holds. Returns the
+        number of rows rewritten."""
+        ids = np.ascontiguousarray(np.asarray(seq_ids, dtype=np.int64))
+        n = len(ids)
+        for a, dt, shape in ((tables, np.int32, None), (lens, np.int32, (n,)),
+                             (row_versions, np.uint64, (n,))):
+            if a.dtype != dt or not a.flags.c_contiguous or (shape and a.shape != shape):
+                raise BlockManagerError(ERR_INVALID, "pa_bm_block_tables_update")
+        if tables.ndim != 2 or tables.shape[0] != n:
+            raise BlockManagerError(ERR_INVALID, "pa_bm_block_tables_update")
+        written = ctypes.c_int32(0)
+        rc = self._lib.pa_bm_block_tables_update(
+            self._h, ids.ctypes.data_as(ctypes.c_void_p), n, tables.shape[1],
+            tables.ctypes.data_as(ctypes.c_void_p), lens.ctypes.data_as(ctypes.c_void_p),
+            row_versions.ctypes.data_as(ctypes.c_void_p), ctypes.byref(written))
+        _ok(rc, "pa_bm_block_tables_update")
+        return int(written.value)

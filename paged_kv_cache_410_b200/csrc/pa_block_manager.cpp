@@ -33,6 +33,7 @@ struct Seq {
   int32_t released = 0;          // leading blocks already released (sliding window)
   Node* tail = nullptr;          // tree node of the last leading block known to the cache
   int32_t tail_blocks = 0;       // leading blocks covered by the path ending at `tail`
+  uint64_t version = 0;          // stamp of the last change to `blocks` (never 0)
 };
 
 uint64_t hash_tokens(const int32_t* t, int32_t n) {
@@ -60,6 +61,9 @@ struct pa_block_manager {
   std::unordered_map<int64_t, std::unique_ptr<Node>> nodes;  // cached block -> node
   std::set<std::pair<uint64_t, int64_t>> evictable;           // (last_use, block)
   uint64_t tick = 0;
+  uint64_t versions = 0;  // last stamp handed out; stamps are unique across sequences
+
+  void changed(Seq& s) { s.version = ++versions; }
 
   bool is_evictable(const Node* n) const {
     return n->block >= 0 && refcount[n->block] == 1 && n->children.empty();
@@ -240,6 +244,7 @@ int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* 
     s.blocks.push_back(b);
   }
   s.length = n_tokens;
+  bm->changed(s);
   if (cached_tokens) *cached_tokens = static_cast<int32_t>(matched.size()) * bs;
   auto& ins = bm->seqs.emplace(seq_id, std::move(s)).first->second;
   // 3. the prompt's full blocks join the cache as soon as they exist
@@ -260,6 +265,7 @@ int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, 
     const int64_t b = bm->alloc();
     if (b < 0) return PA_BM_ERR_NO_BLOCKS;
     s.blocks.push_back(b);
+    bm->changed(s);
   } else {
     const int64_t last = s.blocks.back();
     if (bm->refcount[last] > 1) {  // shared partial block: copy on write
@@ -269,6 +275,7 @@ int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, 
       dst = static_cast<int32_t>(b);
       bm->unref(last);
       s.blocks.back() = b;
+      bm->changed(s);
     }
   }
   *slot = s.blocks[pos / bs] * bs + pos % bs;
@@ -285,6 +292,7 @@ int32_t pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id) {
   auto it = bm->seqs.find(parent_id);
   if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
   Seq child = it->second;
+  bm->changed(child);  // same blocks, but a row that held another table must be rewritten
   for (size_t k = static_cast<size_t>(child.released); k < child.blocks.size(); ++k)
     bm->ref(child.blocks[k]);
   bm->seqs.emplace(child_id, std::move(child));
@@ -334,14 +342,15 @@ int32_t pa_bm_slots(const pa_block_manager* bm, int64_t seq_id, int32_t first, i
   return PA_BM_OK;
 }
 
-int32_t pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, int32_t n_seqs,
-                           int32_t max_blocks_per_seq, int32_t* block_tables,
-                           int32_t* context_lens) {
-  if (!bm || n_seqs < 0 || max_blocks_per_seq <= 0 ||
-      (n_seqs > 0 && (!seq_ids || !block_tables || !context_lens)))
-    return PA_BM_ERR_INVALID;
-  // check every sequence before writing anything
-  std::vector<const Seq*> rows(static_cast<size_t>(n_seqs));
+}  // extern "C"
+
+namespace {
+
+// Looks up every sequence of a batch and checks that its table fits, before
+// anything is written.
+int32_t lookup_rows(const pa_block_manager* bm, const int64_t* seq_ids, int32_t n_seqs,
+                    int32_t max_blocks_per_seq, std::vector<const Seq*>& rows) {
+  rows.resize(static_cast<size_t>(n_seqs));
   for (int32_t i = 0; i < n_seqs; ++i) {
     auto it = bm->seqs.find(seq_ids[i]);
     if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
@@ -349,15 +358,58 @@ int32_t pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, i
       return PA_BM_ERR_CAPACITY;
     rows[static_cast<size_t>(i)] = &it->second;
   }
+  return PA_BM_OK;
+}
+
+void write_row(const Seq& s, int32_t max_blocks_per_seq, int32_t* row) {
+  const int32_t n = static_cast<int32_t>(s.blocks.size());
+  const int64_t* src = s.blocks.data();
+  for (int32_t k = 0; k < n; ++k) row[k] = static_cast<int32_t>(src[k]);
+  std::fill(row + n, row + max_blocks_per_seq, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, int32_t n_seqs,
+                           int32_t max_blocks_per_seq, int32_t* block_tables,
+                           int32_t* context_lens) {
+  if (!bm || n_seqs < 0 || max_blocks_per_seq <= 0 ||
+      (n_seqs > 0 && (!seq_ids || !block_tables || !context_lens)))
+    return PA_BM_ERR_INVALID;
+  std::vector<const Seq*> rows;
+  const int32_t rc = lookup_rows(bm, seq_ids, n_seqs, max_blocks_per_seq, rows);
+  if (rc != PA_BM_OK) return rc;
   for (int32_t i = 0; i < n_seqs; ++i) {
     const Seq& s = *rows[static_cast<size_t>(i)];
-    int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks_per_seq;
-    const int32_t n = static_cast<int32_t>(s.blocks.size());
-    const int64_t* src = s.blocks.data();
-    for (int32_t k = 0; k < n; ++k) row[k] = static_cast<int32_t>(src[k]);
-    std::fill(row + n, row + max_blocks_per_seq, 0);
+    write_row(s, max_blocks_per_seq, block_tables + static_cast<int64_t>(i) * max_blocks_per_seq);
     context_lens[i] = s.length;
   }
+  return PA_BM_OK;
+}
+
+int32_t pa_bm_block_tables_update(const pa_block_manager* bm, const int64_t* seq_ids,
+                                  int32_t n_seqs, int32_t max_blocks_per_seq,
+                                  int32_t* block_tables, int32_t* context_lens,
+                                  uint64_t* row_versions, int32_t* rows_written) {
+  if (!bm || n_seqs < 0 || max_blocks_per_seq <= 0 ||
+      (n_seqs > 0 && (!seq_ids || !block_tables || !context_lens || !row_versions)))
+    return PA_BM_ERR_INVALID;
+  std::vector<const Seq*> rows;
+  const int32_t rc = lookup_rows(bm, seq_ids, n_seqs, max_blocks_per_seq, rows);
+  if (rc != PA_BM_OK) return rc;
+  int32_t written = 0;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const Seq& s = *rows[static_cast<size_t>(i)];
+    if (row_versions[i] != s.version) {
+      write_row(s, max_blocks_per_seq, block_tables + static_cast<int64_t>(i) * max_blocks_per_seq);
+      row_versions[i] = s.version;
+      ++written;
+    }
+    context_lens[i] = s.length;
+  }
+  if (rows_written) *rows_written = written;
   return PA_BM_OK;
 }
 

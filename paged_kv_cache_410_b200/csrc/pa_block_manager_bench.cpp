@@ -8,11 +8,15 @@
 //           prompt's full blocks;
 //   step:   one token per sequence (pa_bm_append_token: slot, copy-on-write
 //           pairs after forks), then the batch's block tables and lengths
-//           (pa_bm_block_tables, the layout pa_decode reads);
+//           (pa_bm_block_tables, the layout pa_decode reads), and the same
+//           through pa_bm_block_tables_update into arrays kept across steps
+//           (only rows whose block list changed are rewritten);
 //   churn:  every `churn` steps, 4 sequences fork a beam and 4 beams end.
 //
 // Usage: pa_block_manager_bench [batch steps prompt own block_size churn]
-// Prints one JSON line.
+// Prints one JSON line; `step_us` is the appends plus the incremental export,
+// `step_us_full_tables` the appends plus the full one. Exits non-zero if the
+// two exports ever differ.
 #include <chrono>
 #include <cstdio>
 #include <cstdlib>
@@ -69,8 +73,11 @@ int main(int argc, char** argv) {
   // ---- decode steps -----------------------------------------------------------
   std::vector<int32_t> tables(static_cast<size_t>(batch) * max_blocks);
   std::vector<int32_t> lens(batch);
-  int64_t appends = 0, cow_pairs = 0, forks = 0, next_id = batch;
-  double append_us = 0.0, tables_us = 0.0, churn_us = 0.0;
+  std::vector<int32_t> kept_tables(static_cast<size_t>(batch) * max_blocks);
+  std::vector<int32_t> kept_lens(batch);
+  std::vector<uint64_t> versions(batch, 0);
+  int64_t appends = 0, cow_pairs = 0, forks = 0, next_id = batch, rewritten = 0;
+  double append_us = 0.0, tables_us = 0.0, update_us = 0.0, churn_us = 0.0;
   for (int s = 0; s < steps; ++s) {
     double t0 = now_us();
     for (int b = 0; b < batch; ++b) {
@@ -85,11 +92,19 @@ int main(int argc, char** argv) {
         PA_BM_OK)
       return 6;
     double t2 = now_us();
+    int32_t written = 0;
+    if (pa_bm_block_tables_update(bm, seqs.data(), batch, max_blocks, kept_tables.data(),
+                                  kept_lens.data(), versions.data(), &written) != PA_BM_OK)
+      return 6;
+    double t3 = now_us();
+    if (kept_tables != tables || kept_lens != lens) return 9;
+    rewritten += written;
     append_us += t1 - t0;
     tables_us += t2 - t1;
+    update_us += t3 - t2;
     if ((s + 1) % churn == 0) {
       // 4 sequences fork a beam that takes the place of 4 others, which end
-      const double t3 = now_us();
+      const double t4 = now_us();
       for (int k = 0; k < 4; ++k) {
         const int parent = (s / churn * 4 + k) % batch;
         const int victim = (parent + batch / 2) % batch;
@@ -98,17 +113,20 @@ int main(int argc, char** argv) {
         seqs[victim] = next_id++;
         ++forks;
       }
-      churn_us += now_us() - t3;
+      churn_us += now_us() - t4;
     }
   }
   std::printf(
       "{\"batch\": %d, \"steps\": %d, \"prompt_tokens\": %d, \"own_tokens\": %d, "
       "\"block_size\": %d, \"admit_us_per_request\": %.3f, \"prompt_tokens_cached\": %lld, "
       "\"append_ns_per_token\": %.1f, \"block_tables_us_per_step\": %.3f, "
-      "\"step_us\": %.3f, \"cow_pairs\": %lld, \"forks\": %lld, \"fork_free_us\": %.3f, "
+      "\"block_tables_update_us_per_step\": %.3f, \"rows_rewritten_per_step\": %.2f, "
+      "\"step_us\": %.3f, \"step_us_full_tables\": %.3f, "
+      "\"cow_pairs\": %lld, \"forks\": %lld, \"fork_free_us\": %.3f, "
       "\"free_blocks_left\": %lld}\n",
       batch, steps, prompt, own, bs, admit_us / batch, static_cast<long long>(cached_total),
-      1000.0 * append_us / static_cast<double>(appends), tables_us / steps,
+      1000.0 * append_us / static_cast<double>(appends), tables_us / steps, update_us / steps,
+      static_cast<double>(rewritten) / steps, (append_us + update_us) / steps,
       (append_us + tables_us) / steps, static_cast<long long>(cow_pairs),
       static_cast<long long>(forks), forks ? churn_us / (forks / 4.0) : 0.0,
       static_cast<long long>(pa_bm_num_free_blocks(bm)));

@@ -194,6 +194,83 @@ def test_invalid_calls():
     assert e.value.code == BM.ERR_CAPACITY
 
 
+def test_incremental_tables_rewrite_only_changed_rows():
+    bm = BM.BlockManager(64, 4)
+    for sid in (1, 2, 3):
+        bm.add_sequence(sid, range(6))              # 2 blocks each, last one half full
+    ids = [1, 2, 3]
+    tables = np.full((3, 5), -7, dtype=np.int32)     # garbage the first call must overwrite
+    lens = np.zeros(3, dtype=np.int32)
+    ver = np.zeros(3, dtype=np.uint64)
+    assert bm.block_tables_update(ids, tables, lens, ver) == 3
+    assert (ver != 0).all() and len(set(ver.tolist())) == 3   # unique, never 0
+    full_t, full_l = bm.block_tables(ids, 5)
+    assert (tables == full_t).all() and (lens == full_l).all()
+    assert bm.block_tables_update(ids, tables, lens, ver) == 0  # nothing changed
+    bm.append_token(1)                               # position 6: same block
+    bm.append_token(1)                               # position 7: same block
+    bm.append_token(2); bm.append_token(2); bm.append_token(2)  # position 8: new block
+    assert bm.block_tables_update(ids, tables, lens, ver) == 1
+    full_t, full_l = bm.block_tables(ids, 5)
+    assert (tables == full_t).all() and (lens == full_l).all()
+    # fork 3 into a row that held 1's table; appending to the shared partial block copies it
+    bm.fork(3, 4)
+    ids = [4, 2, 3]
+    assert bm.block_tables_update(ids, tables, lens, ver) == 1
+    _, cow = bm.append_token(4)
+    assert cow is not None
+    assert bm.block_tables_update(ids, tables, lens, ver) == 1
+    # two sequences trade rows: both rewritten
+    ids = [2, 4, 3]
+    assert bm.block_tables_update(ids, tables, lens, ver) == 2
+    full_t, full_l = bm.block_tables(ids, 5)
+    assert (tables == full_t).all() and (lens == full_l).all()
+    # releasing blocks outside a window keeps the table (the full export keeps it too)
+    bm.release_before(2, 4)
+    assert bm.block_tables_update(ids, tables, lens, ver) == 0
+    assert (tables == bm.block_tables(ids, 5)[0]).all()
+    # a failing call writes nothing
+    bm.add_sequence(9, range(30))                    # 8 blocks > 5
+    before = (tables.copy(), lens.copy(), ver.copy())
+    with pytest.raises(BM.BlockManagerError) as e:
+        bm.block_tables_update([2, 9, 3], tables, lens, ver)
+    assert e.value.code == BM.ERR_CAPACITY
+    for x, y in zip(before, (tables, lens, ver)):
+        assert (x == y).all()
+
+
+def test_incremental_tables_match_the_full_export_under_churn():
+    rng = np.random.default_rng(7)
+    bm = BM.BlockManager(4000, 8, prefix_cache=True)
+    prompt = list(range(40))
+    batch, max_blocks = 24, 64
+    ids = []
+    for b in range(batch):
+        bm.add_sequence(b, prompt + [1000 + b] * int(rng.integers(1, 20)))
+        ids.append(b)
+    tables = np.zeros((batch, max_blocks), dtype=np.int32)
+    lens = np.zeros(batch, dtype=np.int32)
+    ver = np.zeros(batch, dtype=np.uint64)
+    next_id, total_written = batch, 0
+    for step in range(200):
+        for sid in ids:
+            bm.append_token(sid, int(rng.integers(0, 50)))
+        if step % 7 == 3:                            # a beam forks into another's row
+            parent, victim = rng.choice(batch, 2, replace=False)
+            bm.fork(ids[parent], next_id)
+            bm.free_sequence(ids[victim])
+            ids[victim] = next_id
+            next_id += 1
+        if step % 11 == 5:                           # two rows trade places
+            i, j = rng.choice(batch, 2, replace=False)
+            ids[i], ids[j] = ids[j], ids[i]
+        total_written += bm.block_tables_update(ids, tables, lens, ver)
+        full_t, full_l = bm.block_tables(ids, max_blocks)
+        assert (tables == full_t).all() and (lens == full_l).all(), step
+    # a row changes about once per block_size appends, plus the churn
+    assert batch * 200 // 16 <= total_written < batch * 200 // 2
+
+
 def test_host_benchmark_runs():
     # the block manager's host benchmark (serving-step loop) builds and
     # reports sensible numbers on a small case
@@ -209,3 +286,4 @@ def test_host_benchmark_runs():
     assert r["prompt_tokens_cached"] == 15 * 256
     assert r["forks"] == 40 and r["cow_pairs"] > 0
     assert r["append_ns_per_token"] > 0 and r["step_us"] > 0
+    assert 0 < r["block_tables_update_us_per_step"] and 0 < r["rows_rewritten_per_step"] < 16
