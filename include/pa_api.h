@@ -115,7 +115,10 @@ pa_status pa_append_kv(const void* k, const void* v, int32_t in_dtype, int64_t n
                        const pa_cache_desc* cache, void* stream);
 
 /* Bytes of workspace pa_decode needs for these sizes and this partition
- * choice (0 when one partition covers max_context). Pure host function. */
+ * choice (0 when one partition covers max_context). Pure host function.
+ * Sizes whose workspace would pass 2^60 bytes are refused: this returns 0
+ * and every decode entry point returns PA_ERR_UNSUPPORTED for them (the same
+ * rule holds for the sliding-window and shared-prefix sizes below). */
 size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t max_context,
                                 int32_t partition_tokens, const pa_cache_desc* cache);
 

@@ -78,9 +78,18 @@ struct Plan {
   int num_partitions;
   size_t ws_o_bytes;
   size_t ws_bytes;
+  bool fits;  // false: the workspace would not be addressable (sizes refused)
 };
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// The split-K workspace holds head_dim + 2 floats per (row, partition); plans
+// whose workspace would pass 2^60 bytes are refused rather than let the size
+// wrap around.
+bool workspace_fits(int64_t rows, int64_t parts, int64_t head_dim) {
+  const int64_t lim = (int64_t{1} << 60) / ((head_dim + 2) * 4);
+  return rows <= lim && parts <= lim / std::max<int64_t>(rows, 1);
+}
 
 Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int partition_tokens,
                const pa_cache_desc* cd, int window = 0) {
@@ -93,7 +102,8 @@ Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int part
                             : auto_partition(batch, max_context, cd);
   const int64_t np = (max_context + pl.partition_tokens - 1) / pl.partition_tokens;
   pl.num_partitions = static_cast<int>(std::max<int64_t>(np, 1));
-  if (pl.num_partitions > 1) {
+  pl.fits = workspace_fits(batch * num_q_heads, pl.num_partitions, cd->head_dim);
+  if (pl.num_partitions > 1 && pl.fits) {
     pl.ws_o_bytes = round_up(static_cast<size_t>(batch * num_q_heads) * pl.num_partitions *
                                  cd->head_dim * sizeof(float),
                              256);
@@ -266,6 +276,7 @@ struct CascadePlan {
   int num_partitions;  // chunks + suffix partitions
   size_t ws_o_bytes;
   size_t ws_bytes;
+  bool fits;  // as Plan::fits
 };
 
 // 16-bit caches with blocks of >= 8 tokens (whole 1024-byte swizzle atoms
@@ -373,6 +384,8 @@ CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_co
   pl.suffix_partitions =
       static_cast<int>((suffix_max + pl.suffix_partition_tokens - 1) / pl.suffix_partition_tokens);
   pl.num_partitions = pl.num_chunks + pl.suffix_partitions;
+  pl.fits = workspace_fits(batch * num_q_heads, pl.num_partitions, cd->head_dim);
+  if (!pl.fits) return pl;
   pl.ws_o_bytes = round_up(static_cast<size_t>(batch * num_q_heads) * pl.num_partitions *
                                cd->head_dim * sizeof(float),
                            256);
@@ -620,6 +633,7 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
                                    scale, out, partition_tokens, &bs_log2, &nothing);
   if (st != PA_OK || nothing) return st;
   const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
@@ -655,6 +669,7 @@ pa_status pa_append_decode(const void* q, const void* k, const void* v, int32_t 
        !aligned16(cache->v_inv_scale)))
     return PA_ERR_INVALID_ARG;
   const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
@@ -703,6 +718,7 @@ pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch
   if (window <= 0) return PA_ERR_INVALID_ARG;
   if (nothing) return PA_OK;
   const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache, window);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
   if (pl.ws_bytes > 0) {
     if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
@@ -770,6 +786,7 @@ pa_status pa_decode_shared_prefix(const void* q, int32_t q_dtype, int32_t batch,
                      workspace, workspace_bytes, stream);
   const CascadePlan pl = make_cascade_plan(batch, num_q_heads, max_context, prefix_blocks,
                                            partition_tokens, cache);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
 

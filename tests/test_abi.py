@@ -95,6 +95,14 @@ def test_decode_argument_checks(lib):
     assert call(maxc=5000, pt=64) == 4
     assert call(maxc=5000, pt=64, ws=FAKE + 16, wsb=need) == 4  # not 256-byte aligned
     assert call(maxc=5000, pt=64, ws=FAKE, wsb=need - 1) == 4
+    # sizes whose split-K workspace would wrap around size_t are refused, not
+    # sized modulo 2^64 (65535 sequences x 1048544 query heads x 2^27 partitions)
+    big = dict(batch=65535, hq=2 * 524272, maxc=(1 << 31) - 1, pt=16)
+    assert lib.pa_decode_workspace_size(big["batch"], big["hq"], big["maxc"], 16,
+                                        ctypes.byref(d)) == 0
+    assert call(**big, ws=FAKE, wsb=(1 << 64) - 1) == 2
+    assert lib.pa_decode_shared_prefix_workspace_size(big["batch"], big["hq"], big["maxc"], 2,
+                                                      16, ctypes.byref(d)) == 0
     # E4M3 caches need scales
     d8 = _desc(cache_dtype=B.PA_E4M3)
     assert lib.pa_decode(FAKE, 0, 1, 2, FAKE, FAKE, ctypes.byref(d8), FAKE, 4, FAKE, 64, 0.1,
