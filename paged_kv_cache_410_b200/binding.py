@@ -117,8 +117,30 @@ def _dtype_code(t: torch.dtype) -> int:
     raise TypeError(f"unsupported dtype {t}")
 
 
-def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+_IO = (torch.float16, torch.bfloat16)
+_E4M3 = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _on_device(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
+def _dev(t, name: str, dtypes=None, shape=None) -> int | None:
+    """Device address of a contiguous CUDA tensor, after checking its dtype and
+    shape (None, where the C call allows NULL, passes through)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not _on_device(t) or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA tensor")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if shape is not None and t.shape != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def _stream(stream) -> int | None:
@@ -142,9 +164,23 @@ class PagedCache:
     v_inv_scale: torch.Tensor | None = None
 
     def desc(self) -> _CacheDesc:
+        sc = (self.num_kv_heads, self.head_dim)
+        f32 = (torch.float32,)
         return _CacheDesc(self.num_blocks, self.block_size, self.num_kv_heads, self.head_dim,
-                          _dtype_code(self.dtype), _ptr(self.k_scale), _ptr(self.v_scale),
-                          _ptr(self.k_inv_scale), _ptr(self.v_inv_scale))
+                          _dtype_code(self.dtype), _dev(self.k_scale, "k_scale", f32, sc),
+                          _dev(self.v_scale, "v_scale", f32, sc),
+                          _dev(self.k_inv_scale, "k_inv_scale", f32, sc),
+                          _dev(self.v_inv_scale, "v_inv_scale", f32, sc))
+
+    @property
+    def shape(self):
+        return (self.num_blocks, self.block_size, self.num_kv_heads, self.head_dim)
+
+    def cache_ptrs(self, k_cache, v_cache):
+        """Device addresses of this layer's K and V caches (checked against the
+        shape and dtype described here)."""
+        dt = _E4M3 if self.dtype in _E4M3 else (self.dtype,)
+        return _dev(k_cache, "k_cache", dt, self.shape), _dev(v_cache, "v_cache", dt, self.shape)
 
     @staticmethod
     def for_tensor(cache: torch.Tensor, **scales) -> "PagedCache":
@@ -157,12 +193,38 @@ def _check(rc: int, what: str):
         raise PagedAttentionError(rc, what)
 
 
+def _new_tokens(k, v, slot_mapping, cache: PagedCache, rows=None):
+    """Checked addresses of new tokens' k, v ([T, Hkv, D], one 16-bit dtype)
+    and slot_mapping ([T] int64)."""
+    t = k.shape[0] if rows is None else rows
+    shape = (t, cache.num_kv_heads, cache.head_dim)
+    pk = _dev(k, "k", _IO, shape)
+    pv = _dev(v, "v", (k.dtype,), shape)
+    return pk, pv, _dev(slot_mapping, "slot_mapping", (torch.int64,), (t,))
+
+
+def _decode_io(q, block_tables, context_lens, out, cache: PagedCache):
+    """Checked addresses of q [B, Hq, D], block_tables [B, MB] int32,
+    context_lens [B] int32 and out (q's shape and dtype)."""
+    if q.dim() != 3:
+        raise ValueError("q: expected [batch, num_q_heads, head_dim]")
+    batch, hq = q.shape[0], q.shape[1]
+    pq = _dev(q, "q", _IO, (batch, hq, cache.head_dim))
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables: expected [batch, max_blocks_per_seq]")
+    pt = _dev(block_tables, "block_tables", (torch.int32,), (batch, block_tables.shape[1]))
+    pl = _dev(context_lens, "context_lens", (torch.int32,), (batch,))
+    po = _dev(out, "out", (q.dtype,), tuple(q.shape))
+    return pq, pt, pl, po
+
+
 def pa_append_kv(k, v, slot_mapping, k_cache, v_cache, cache: PagedCache, stream=None):
     """Store k, v ([T, Hkv, D], fp16/bf16) at slot_mapping ([T] int64)."""
     lib = load_library()
     d = cache.desc()
-    rc = lib.pa_append_kv(_ptr(k), _ptr(v), _dtype_code(k.dtype), k.shape[0],
-                          _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
+    pk, pv, ps = _new_tokens(k, v, slot_mapping, cache)
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_append_kv(pk, pv, _dtype_code(k.dtype), k.shape[0], ps, kc, vc, ctypes.byref(d),
                           _stream(stream))
     _check(rc, "pa_append_kv")
 
@@ -188,12 +250,12 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache
     pa_decode_workspace_size(...) bytes (or None when that is 0)."""
     lib = load_library()
     d = cache.desc()
-    batch, hq = q.shape[0], q.shape[1]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.pa_decode(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache), _ptr(v_cache),
-                       ctypes.byref(d), _ptr(block_tables), block_tables.shape[1],
-                       _ptr(context_lens), int(max_context), float(scale), _ptr(out),
-                       int(partition_tokens), _ptr(workspace), ws_bytes, _stream(stream))
+    pq, pt, pl, po = _decode_io(q, block_tables, context_lens, out, cache)
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_decode(pq, _dtype_code(q.dtype), q.shape[0], q.shape[1], kc, vc,
+                       ctypes.byref(d), pt, block_tables.shape[1], pl, int(max_context),
+                       float(scale), po, int(partition_tokens), _dev(workspace, "workspace"),
+                       _nbytes(workspace), _stream(stream))
     _check(rc, "pa_decode")
 
 
@@ -208,13 +270,13 @@ def pa_append_decode(q, k, v, slot_mapping, k_cache, v_cache, block_tables, cont
         raise TypeError("pa_append_decode: q, k and v share one dtype")
     lib = load_library()
     d = cache.desc()
-    batch, hq = q.shape[0], q.shape[1]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.pa_append_decode(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), batch, hq,
-                              _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
-                              _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-                              int(max_context), float(scale), _ptr(out), int(partition_tokens),
-                              _ptr(workspace), ws_bytes, _stream(stream))
+    pq, pt, pl, po = _decode_io(q, block_tables, context_lens, out, cache)
+    pk, pv, ps = _new_tokens(k, v, slot_mapping, cache, rows=q.shape[0])
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_append_decode(pq, pk, pv, _dtype_code(q.dtype), q.shape[0], q.shape[1], ps, kc,
+                              vc, ctypes.byref(d), pt, block_tables.shape[1], pl,
+                              int(max_context), float(scale), po, int(partition_tokens),
+                              _dev(workspace, "workspace"), _nbytes(workspace), _stream(stream))
     _check(rc, "pa_append_decode")
 
 
@@ -243,14 +305,13 @@ def pa_decode_shared_prefix(q, k_cache, v_cache, block_tables, context_lens, sca
     KV head for all sequences, then merged with each sequence's suffix."""
     lib = load_library()
     d = cache.desc()
-    batch, hq = q.shape[0], q.shape[1]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.pa_decode_shared_prefix(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache),
-                                     _ptr(v_cache), ctypes.byref(d), _ptr(block_tables),
-                                     block_tables.shape[1], _ptr(context_lens), int(max_context),
-                                     int(prefix_blocks), float(scale), _ptr(out),
-                                     int(partition_tokens), _ptr(workspace), ws_bytes,
-                                     _stream(stream))
+    pq, pt, pl, po = _decode_io(q, block_tables, context_lens, out, cache)
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_decode_shared_prefix(pq, _dtype_code(q.dtype), q.shape[0], q.shape[1], kc, vc,
+                                     ctypes.byref(d), pt, block_tables.shape[1], pl,
+                                     int(max_context), int(prefix_blocks), float(scale), po,
+                                     int(partition_tokens), _dev(workspace, "workspace"),
+                                     _nbytes(workspace), _stream(stream))
     _check(rc, "pa_decode_shared_prefix")
 
 
@@ -269,14 +330,13 @@ def pa_decode_sliding_window(q, k_cache, v_cache, block_tables, context_lens, sc
     """pa_decode attending only to each sequence's last `window` tokens."""
     lib = load_library()
     d = cache.desc()
-    batch, hq = q.shape[0], q.shape[1]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.pa_decode_sliding_window(_ptr(q), _dtype_code(q.dtype), batch, hq, _ptr(k_cache),
-                                      _ptr(v_cache), ctypes.byref(d), _ptr(block_tables),
-                                      block_tables.shape[1], _ptr(context_lens),
-                                      int(max_context), int(window), float(scale), _ptr(out),
-                                      int(partition_tokens), _ptr(workspace), ws_bytes,
-                                      _stream(stream))
+    pq, pt, pl, po = _decode_io(q, block_tables, context_lens, out, cache)
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_decode_sliding_window(pq, _dtype_code(q.dtype), q.shape[0], q.shape[1], kc, vc,
+                                      ctypes.byref(d), pt, block_tables.shape[1], pl,
+                                      int(max_context), int(window), float(scale), po,
+                                      int(partition_tokens), _dev(workspace, "workspace"),
+                                      _nbytes(workspace), _stream(stream))
     _check(rc, "pa_decode_sliding_window")
 
 
@@ -289,12 +349,12 @@ def pa_decode_static_workspace(q, k_cache, v_cache, block_tables, context_lens, 
     race on the shared array)."""
     lib = load_library()
     d = cache.desc()
-    batch, hq = q.shape[0], q.shape[1]
-    rc = lib.pa_decode_static_workspace(_ptr(q), _dtype_code(q.dtype), batch, hq,
-                                        _ptr(k_cache), _ptr(v_cache), ctypes.byref(d),
-                                        _ptr(block_tables), block_tables.shape[1],
-                                        _ptr(context_lens), int(max_context), float(scale),
-                                        _ptr(out), int(partition_tokens), _stream(stream))
+    pq, pt, pl, po = _decode_io(q, block_tables, context_lens, out, cache)
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_decode_static_workspace(pq, _dtype_code(q.dtype), q.shape[0], q.shape[1], kc, vc,
+                                        ctypes.byref(d), pt, block_tables.shape[1], pl,
+                                        int(max_context), float(scale), po,
+                                        int(partition_tokens), _stream(stream))
     _check(rc, "pa_decode_static_workspace")
 
 
@@ -303,8 +363,9 @@ def pa_copy_blocks(pairs, k_cache, v_cache, cache: PagedCache, stream=None):
     lib = load_library()
     d = cache.desc()
     arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
-    rc = lib.pa_copy_blocks(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], _ptr(k_cache),
-                            _ptr(v_cache), ctypes.byref(d), _stream(stream))
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_copy_blocks(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], kc, vc,
+                            ctypes.byref(d), _stream(stream))
     _check(rc, "pa_copy_blocks")
 
 
@@ -317,8 +378,9 @@ def pa_copy_blocks_layers(pairs, k_caches, v_caches, cache: PagedCache, stream=N
     d = cache.desc()
     arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
     n = len(k_caches)
-    kp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in k_caches])
-    vp = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in v_caches])
+    ptrs = [cache.cache_ptrs(k, v) for k, v in zip(k_caches, v_caches)]
+    kp = (ctypes.c_void_p * max(n, 1))(*[a for a, _ in ptrs])
+    vp = (ctypes.c_void_p * max(n, 1))(*[b for _, b in ptrs])
     rc = lib.pa_copy_blocks_layers(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], kp, vp, n,
                                    ctypes.byref(d), _stream(stream))
     _check(rc, "pa_copy_blocks_layers")
