@@ -107,6 +107,33 @@ struct pa_block_manager {
     return true;
   }
 
+  // Whether `need` blocks can be had from the free list plus evictions,
+  // without evicting anything: a cached block is reclaimable when it and every
+  // block below it in the tree is held by the cache alone (eviction takes
+  // leaves first, so exactly those subtrees can go).
+  bool can_reclaim(int64_t need) const {
+    int64_t have = static_cast<int64_t>(free_list.size());
+    if (have >= need) return true;
+    std::vector<const Node*> order;  // pre-order: parents before children
+    std::vector<const Node*> stack{&root};
+    while (!stack.empty()) {
+      const Node* n = stack.back();
+      stack.pop_back();
+      order.push_back(n);
+      for (const auto& c : n->children) stack.push_back(c.second);
+    }
+    std::unordered_map<const Node*, bool> clean;
+    for (auto it = order.rbegin(); it != order.rend(); ++it) {
+      const Node* n = *it;
+      if (n == &root) break;
+      bool ok = refcount[n->block] == 1;
+      for (const auto& c : n->children) ok = ok && clean[c.second];
+      clean[n] = ok;
+      if (ok && ++have >= need) return true;
+    }
+    return false;
+  }
+
   int64_t alloc() {
     if (free_list.empty() && !evict_one()) return -1;
     const int64_t b = free_list.back();
@@ -226,18 +253,24 @@ int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* 
       node = next;
     }
   }
+  for (Node* m : matched) bm->ref(m->block);
+  // 2. fail before anything changes if the rest cannot be allocated (a
+  // reference taken and dropped leaves a node exactly as it was)
+  const int32_t need = (n_tokens + bs - 1) / bs;
+  if (!bm->can_reclaim(need - static_cast<int64_t>(matched.size()))) {
+    for (Node* m : matched) bm->unref(m->block);
+    return PA_BM_ERR_NO_BLOCKS;
+  }
   for (Node* m : matched) {
     s.blocks.push_back(m->block);
-    bm->ref(m->block);
     bm->touch(m);
   }
   s.tail = matched.empty() ? nullptr : matched.back();
   s.tail_blocks = static_cast<int32_t>(matched.size());
-  // 2. private blocks for the rest
-  const int32_t need = (n_tokens + bs - 1) / bs;
+  // 3. private blocks for the rest
   for (int32_t i = static_cast<int32_t>(matched.size()); i < need; ++i) {
     const int64_t b = bm->alloc();
-    if (b < 0) {  // roll back
+    if (b < 0) {  // roll back (not reached after the check above)
       for (size_t k = 0; k < s.blocks.size(); ++k) bm->unref(s.blocks[k]);
       return PA_BM_ERR_NO_BLOCKS;
     }
@@ -247,7 +280,7 @@ int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* 
   bm->changed(s);
   if (cached_tokens) *cached_tokens = static_cast<int32_t>(matched.size()) * bs;
   auto& ins = bm->seqs.emplace(seq_id, std::move(s)).first->second;
-  // 3. the prompt's full blocks join the cache as soon as they exist
+  // 4. the prompt's full blocks join the cache as soon as they exist
   for (int32_t i = ins.tail_blocks; (i + 1) * bs <= n_tokens; ++i) bm->cache_full_block(ins, i);
   return PA_BM_OK;
 }

@@ -8,6 +8,7 @@ reference-counted, and branches copy a block only where they diverge (KV cache
 article, section 'PagedAttention：把操作系统的老智慧搬进推理引擎'); a radix tree
 of token ids lets later requests reuse a cached prefix (chapter '第2章 KV
 Cache：模型内部的显存复用')."""
+import functools
 import re
 import os
 
@@ -287,3 +288,129 @@ def test_host_benchmark_runs():
     assert r["forks"] == 40 and r["cow_pairs"] > 0
     assert r["append_ns_per_token"] > 0 and r["step_us"] > 0
     assert 0 < r["block_tables_update_us_per_step"] and 0 < r["rows_rewritten_per_step"] < 16
+
+
+def _check_contents(bm, seqs, released, content, bs):
+    """Every live sequence still reads its own tokens through its slots."""
+    for sid, toks in seqs.items():
+        first = released[sid] // bs * bs
+        if first >= len(toks):
+            continue
+        slots = bm.slots(sid, first, len(toks) - first)
+        got = [content.get(int(s)) for s in slots]
+        assert got == toks[first:], (sid, first)
+
+
+@functools.lru_cache(maxsize=None)
+def _random_serving(seed):
+    """A random mix of admissions (prompts built from a few shared system
+    prompts), appends, forks, ends and window releases on a small pool, with
+    the caller's K/V writes mirrored in a model of the cache contents: each
+    slot holds the token written there last; prompt tokens past the cached
+    prefix are written after admission; copy-on-write pairs are applied
+    before the append. After every operation each live sequence must read
+    exactly its own tokens (so no block it uses was handed to another
+    sequence, evicted, or written by a sibling), failed calls must change
+    nothing, and the block accounting must add up."""
+    rng = np.random.default_rng(seed)
+    bs = int(rng.choice([1, 2, 4, 8]))
+    nb = int(rng.integers(24, 64))
+    bm = BM.BlockManager(nb, bs, prefix_cache=seed % 4 != 3)
+    systems = [list(rng.integers(0, 5, size=int(rng.integers(0, 3 * bs + 2))))
+               for _ in range(3)]
+    content, seqs, released = {}, {}, {}
+    next_id, failures, hits, copies = 0, 0, 0, 0
+
+    def write(slot, tok):
+        content[int(slot)] = int(tok)
+
+    def snapshot():
+        return bm.num_free_blocks, bm.num_cached_blocks
+
+    for step in range(400):
+        op = rng.choice(["add", "append", "append", "append", "fork", "free", "release"])
+        live = list(seqs)
+        if op == "add" or not live:
+            toks = [int(t) for t in systems[int(rng.integers(0, 3))]]
+            toks += [int(t) for t in rng.integers(0, 5, size=int(rng.integers(1, 2 * bs + 2)))]
+            before = snapshot()
+            try:
+                cached = bm.add_sequence(next_id, toks)
+            except BM.BlockManagerError as e:
+                assert e.code == BM.ERR_NO_BLOCKS and snapshot() == before
+                failures += 1
+                continue
+            assert cached % bs == 0 and cached <= len(toks)
+            hits += cached > 0
+            # the reused prefix already holds these very tokens
+            if cached:
+                got = [content.get(int(s)) for s in bm.slots(next_id, 0, cached)]
+                assert got == toks[:cached]
+            for s_, t in zip(bm.slots(next_id, cached, len(toks) - cached), toks[cached:]):
+                write(s_, t)
+            seqs[next_id], released[next_id] = toks, 0
+            next_id += 1
+        elif op == "append":
+            sid = live[int(rng.integers(0, len(live)))]
+            tok = int(rng.integers(0, 5))
+            before = snapshot()
+            try:
+                slot, cow = bm.append_token(sid, tok)
+            except BM.BlockManagerError as e:
+                assert e.code == BM.ERR_NO_BLOCKS and snapshot() == before
+                failures += 1
+                continue
+            if cow:
+                copies += 1
+                src, dst = cow
+                for r in range(bs):
+                    if src * bs + r in content:
+                        content[dst * bs + r] = content[src * bs + r]
+                    else:
+                        content.pop(dst * bs + r, None)
+            write(slot, tok)
+            seqs[sid] = seqs[sid] + [tok]
+        elif op == "fork":
+            parent = live[int(rng.integers(0, len(live)))]
+            bm.fork(parent, next_id)
+            seqs[next_id], released[next_id] = list(seqs[parent]), released[parent]
+            next_id += 1
+        elif op == "free":
+            sid = live[int(rng.integers(0, len(live)))]
+            bm.free_sequence(sid)
+            del seqs[sid], released[sid]
+        else:
+            sid = live[int(rng.integers(0, len(live)))]
+            pos = int(rng.integers(0, len(seqs[sid]) + 1))
+            bm.release_before(sid, pos)
+            released[sid] = max(released[sid], pos)
+        _check_contents(bm, seqs, released, content, bs)
+        # accounting: every block is free or referenced, never both
+        refs = [bm.refcount(b) for b in range(nb)]
+        assert bm.num_free_blocks == sum(r == 0 for r in refs)
+        held = {}
+        for sid, toks in seqs.items():
+            t, _ = bm.block_tables([sid], max(1, (len(toks) + bs - 1) // bs))
+            for k in range(released[sid] // bs, (len(toks) + bs - 1) // bs):
+                held[int(t[0, k])] = held.get(int(t[0, k]), 0) + 1
+        for b, n in held.items():
+            assert refs[b] - n in (0, 1), (b, refs[b], n)   # plus the cache's own reference
+        cache_only = [b for b in range(nb) if refs[b] > 0 and b not in held]
+        assert all(refs[b] == 1 for b in cache_only)
+        assert bm.num_cached_blocks == len(cache_only)
+    return dict(seqs=next_id, hits=hits, copies=copies, failures=failures)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_serving_keeps_every_sequence_cache_intact(seed):
+    _random_serving(seed)
+
+
+def test_random_serving_reaches_every_case():
+    # across the seeds the loop exercises prefix hits, copy-on-write and a
+    # full pool (so the checks above are not vacuous)
+    stats = [_random_serving(seed) for seed in range(8)]
+    assert sum(s["hits"] for s in stats) > 20
+    assert sum(s["copies"] for s in stats) > 20
+    assert sum(s["failures"] for s in stats) > 5
+    assert all(s["seqs"] > 20 for s in stats)
