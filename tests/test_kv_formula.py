@@ -57,3 +57,35 @@ def test_bench_byte_accounting_uses_the_formula(oracle_mod):
     per_tok = oracle_mod.kv_cache_bytes(1, p.num_kv_heads, p.head_dim, 1, 1, 2)
     assert acc["kv_logical"] == per_tok * int(p.context_lens.sum())
     assert acc["kv_unique"] == per_tok * (2000 + int((p.context_lens - 2000).sum()))
+
+
+def test_accounting_of_window_fused_and_fp8(oracle_mod):
+    from paged_kv_cache_410_b200 import accounting, workloads
+    w = workloads.custom([5, 40, 77, 300], num_q_heads=8, num_kv_heads=2, head_dim=128)
+    per_tok = oracle_mod.kv_cache_bytes(1, 2, 128, 1, 1, 2)
+    # a window of 32 reads min(L, 32) tokens per sequence, and the table entries of
+    # the blocks those tokens lie in
+    acc = accounting.decode_bytes(w, window=32)
+    lens = [5, 40, 77, 300]
+    assert acc["kv_unique"] == acc["kv_logical"] == per_tok * sum(min(L, 32) for L in lens)
+    blocks = sum((L - 1) // 16 - max(L - 32, 0) // 16 + 1 for L in lens)
+    qo = 2 * 4 * 8 * 128 * 2
+    assert acc["other"] == qo + 4 * blocks + 4 * 4
+    # append + decode in one pass: the new rows are not read back from the cache
+    a = accounting.append_bytes(w)
+    assert a == 2 * 4 * 2 * 128 * (2 + 2) + 8 * 4
+    new_rows = 4 * per_tok
+    assert accounting.fused_bytes(w) == accounting.decode_bytes(w)["total_unique"] + a - new_rows
+    st = accounting.step_bytes(w, fused=True)
+    assert st["total"] == st["append_decode"] + st["copy"]
+    # E4M3: one byte per element, plus both scale arrays (fp32 [Hkv][D]) read once
+    f = workloads.fp8_beams(batch=24, beam_groups=2, median_len=40, max_len=200)
+    acc8 = accounting.decode_bytes(f)
+    slots = set()
+    for b in range(f.batch):
+        for j in range(int(f.context_lens[b])):
+            slots.add(int(f.block_tables[b, j // 16]) * 16 + j % 16)
+    assert acc8["kv_unique"] == len(slots) * 2 * 8 * 128
+    assert acc8["kv_logical"] == int(f.context_lens.sum()) * 2 * 8 * 128
+    assert acc8["kv_unique"] < acc8["kv_logical"]                 # beams share prompt blocks
+    assert accounting.copy_bytes(f) == len(f.copy_pairs) * 16 * 8 * 128 * 2 * 2
