@@ -234,3 +234,65 @@ def test_shared_prefix_partition_rule(lib):
     assert (lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d8)) ==
             lib.pa_decode_partition_tokens(128, 2049, ctypes.byref(d8)))
     assert lib.pa_decode_shared_prefix_partition_tokens(0, 64, 4049, 125, ctypes.byref(d)) == 0
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "pa_api.h"
+#include "pa_block_manager.h"
+
+int main(void) {
+  pa_cache_desc cd;
+  memset(&cd, 0, sizeof cd);
+  cd.num_blocks = 1024; cd.block_size = 16; cd.num_kv_heads = 8; cd.head_dim = 128;
+  cd.cache_dtype = PA_BF16;
+  size_t ws = pa_decode_workspace_size(4, 64, 131072, 0, &cd);
+  int32_t pt = pa_decode_partition_tokens(4, 131072, &cd);
+  /* a host-side check fails before anything reaches a GPU */
+  pa_status bad = pa_decode(NULL, PA_BF16, 1, 64, NULL, NULL, &cd, NULL, 4, NULL, 64, 0.1f,
+                            NULL, 0, NULL, 0, NULL);
+  pa_block_manager* bm = pa_bm_create(64, 16, 1);
+  int32_t toks[40], cached = -1, src = 0, dst = 0, tables[8], lens[2];
+  int64_t slot = -1, ids[2] = {1, 2};
+  int i, rc = 0;
+  for (i = 0; i < 40; ++i) toks[i] = 1000 + i;
+  rc |= pa_bm_add_sequence(bm, 1, toks, 40, &cached);
+  rc |= pa_bm_add_sequence(bm, 2, toks, 40, &cached);
+  rc |= pa_bm_append_token(bm, 2, 7, &slot, &src, &dst);
+  rc |= pa_bm_block_tables(bm, ids, 2, 4, tables, lens);
+  printf("%d|%s|%zu|%d|%d|%d|%d|%d|%d|%d|%d\n", (int)pa_version(),
+         pa_status_string(PA_ERR_WORKSPACE), ws, (int)pt, (int)bad, rc, (int)cached, (int)src,
+         (int)lens[0], (int)lens[1], tables[0] == tables[4] && tables[1] == tables[5]);
+  pa_bm_destroy(bm);
+  return 0;
+}
+"""
+
+
+def test_headers_are_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    """Both headers compile as strict C99 with warnings as errors, and a C
+    program linked against libpagedattn.so calls its host-side entry points
+    (no GPU involved)."""
+    import subprocess
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lpagedattn", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    f = out.split("|")
+    d = _desc(num_blocks=1024, block_size=16, num_kv_heads=8, head_dim=128,
+              cache_dtype=B.PA_BF16)
+    assert int(f[0]) == lib.pa_version()
+    assert f[1] == "workspace missing or too small"
+    assert int(f[2]) == lib.pa_decode_workspace_size(4, 64, 131072, 0, ctypes.byref(d)) > 0
+    assert int(f[3]) == lib.pa_decode_partition_tokens(4, 131072, ctypes.byref(d)) == 512
+    assert int(f[4]) == 1                         # PA_ERR_INVALID_ARG
+    assert int(f[5]) == 0                         # every block-manager call succeeded
+    assert int(f[6]) == 32                        # two full 16-token blocks reused
+    assert int(f[7]) == -1                        # the partial block was private: no copy
+    assert (int(f[8]), int(f[9])) == (40, 41)
+    assert int(f[10]) == 1                        # both tables start with the same blocks
