@@ -191,21 +191,41 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle ---
 
+_ORACLE_CACHES = {}
+
+
+def oracle_caches(w):
+    """The oracle's copy of the workload's caches, made once per workload (set-up,
+    not timed): the 16-bit pools as drawn, or an E4M3 pool that the oracle's own
+    append fills from the workload's history tokens."""
+    if id(w) not in _ORACLE_CACHES:
+        if w.cache_dtype == "e4m3":
+            import oracle
+            shape = (w.num_blocks, w.block_size, w.num_kv_heads, w.head_dim)
+            kc, vc = np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+            oracle.append_kv(w.fill_k, w.fill_v, w.io_dtype, w.fill_slots, kc, vc, "e4m3",
+                             w.block_size, w.k_inv_scale, w.v_inv_scale)
+        else:
+            kc, vc = w.k_pool, w.v_pool
+        _ORACLE_CACHES[id(w)] = (w, kc, vc)
+    return _ORACLE_CACHES[id(w)][1:]
+
+
 def oracle_step_time(w, seqs, reps=1):
-    """Seconds for `reps` oracle passes (append of the sample's tokens +
-    decode of the sample) over the sampled sequences."""
+    """Seconds for `reps` oracle passes over the sampled sequences: their
+    copy-on-write pairs, the append of their new tokens and their decode."""
     import oracle
     from paged_kv_cache_410_b200 import workloads as W
     s = W.subset(w, seqs)
-    if w.cache_dtype == "e4m3":
-        raise NotImplementedError("the CPU baseline is timed on 16-bit caches")
-    kc, vc = w.k_pool, w.v_pool  # the oracle append rewrites the same slots each pass
+    kc, vc = oracle_caches(w)  # each pass rewrites the same slots and blocks
     t0 = time.perf_counter()
     for _ in range(reps):
+        if len(s.copy_pairs):
+            oracle.copy_blocks(s.copy_pairs, kc, vc, s.cache_dtype)
         oracle.append_kv(s.k_new, s.v_new, s.io_dtype, s.slot_mapping, kc, vc, s.cache_dtype,
-                         s.block_size)
+                         s.block_size, s.k_inv_scale, s.v_inv_scale)
         oracle.decode(s.q, s.io_dtype, kc, vc, s.cache_dtype, s.block_tables, s.context_lens,
-                      s.scale)
+                      s.scale, k_scale=s.k_scale, v_scale=s.v_scale)
     return time.perf_counter() - t0, s
 
 
@@ -225,7 +245,7 @@ def cpu_baseline(w, target_s=12.0):
     nbytes = A.step_bytes(s)["total"] * reps
     return {"value": nbytes / t / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"{n} of {w.batch} sequences x {reps} passes (append + decode), "
+            "sample": f"{n} of {w.batch} sequences x {reps} passes (copies + append + decode), "
                       f"{t:.1f} s, float64 C oracle, OpenMP over (sequence, head)",
             "seconds": t, "tokens_per_s_per_layer": n * reps / t}
 
@@ -277,7 +297,7 @@ def run_reference(args):
                  "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                                   "kind": "oracle",
                                   "sample": f"{n} of {w.batch} sequences per step "
-                                            "(append + decode), float64 C oracle"},
+                                            "(copies + append + decode), float64 C oracle"},
                  "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                          "d2h_bytes_per_step": 0},
                  "gpu_launches": 0})

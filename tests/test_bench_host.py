@@ -68,3 +68,27 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "--workload", "tiny_mha", "--steps", "2", "--warmup", "3"],
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_on_the_fp8_beams_workload():
+    # E4M3 cache: the oracle fills its own cache from the history tokens, then
+    # times copies + append + decode
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "fp8_beams", "--batch", "64", "--steps", "2",
+                        "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["config"]["kv_cache_dtype"] == "e4m3"
+
+
+def test_oracle_step_covers_copies_append_and_decode():
+    from paged_kv_cache_410_b200 import workloads as W
+    w = W.fp8_beams(batch=24, beam_groups=2, median_len=40, max_len=200)
+    t, s = bench.oracle_step_time(w, np.arange(8))
+    assert t > 0 and s.batch == 8 and len(s.copy_pairs) == len(w.copy_pairs)
+    kc, vc = bench.oracle_caches(w)
+    assert kc.dtype == np.uint8 and kc.any()              # filled by the oracle's append
+    assert bench.oracle_caches(w)[0] is kc                # made once per workload
