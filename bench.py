@@ -211,9 +211,11 @@ def oracle_caches(w):
     return _ORACLE_CACHES[id(w)][1:]
 
 
-def oracle_step_time(w, seqs, reps=1):
+def oracle_step_time(w, seqs, reps=1, window=0):
     """Seconds for `reps` oracle passes over the sampled sequences: their
-    copy-on-write pairs, the append of their new tokens and their decode."""
+    copy-on-write pairs, the append of their new tokens and their decode
+    (over the last `window` tokens when window > 0). Also returns the sample
+    and the last pass's float64 output [n, Hq, D]."""
     import oracle
     from paged_kv_cache_410_b200 import workloads as W
     s = W.subset(w, seqs)
@@ -224,30 +226,49 @@ def oracle_step_time(w, seqs, reps=1):
             oracle.copy_blocks(s.copy_pairs, kc, vc, s.cache_dtype)
         oracle.append_kv(s.k_new, s.v_new, s.io_dtype, s.slot_mapping, kc, vc, s.cache_dtype,
                          s.block_size, s.k_inv_scale, s.v_inv_scale)
-        oracle.decode(s.q, s.io_dtype, kc, vc, s.cache_dtype, s.block_tables, s.context_lens,
-                      s.scale, k_scale=s.k_scale, v_scale=s.v_scale)
-    return time.perf_counter() - t0, s
+        out = oracle.decode(s.q, s.io_dtype, kc, vc, s.cache_dtype, s.block_tables,
+                            s.context_lens, s.scale, k_scale=s.k_scale, v_scale=s.v_scale,
+                            window=window)
+    return time.perf_counter() - t0, s, out
 
 
-def cpu_baseline(w, target_s=12.0):
+def cpu_baseline(w, target_s=12.0, window=0):
     """Oracle throughput on a bounded sample: whole passes over the batch (or
-    the first sequences of it) repeated until about `target_s` seconds."""
+    the first sequences of it) repeated until about `target_s` seconds.
+    Returns the JSON object, the sampled sequence indices and the oracle's
+    output for them."""
     import oracle
     from paged_kv_cache_410_b200 import accounting as A
-    t1, s1 = oracle_step_time(w, np.arange(1))
+    t1, _, _ = oracle_step_time(w, np.arange(1), window=window)
     per_seq = max(t1, 1e-4)
     n = int(min(w.batch, max(1, target_s / per_seq)))
     seqs = np.arange(n)
-    t, s = oracle_step_time(w, seqs)
+    t, s, out = oracle_step_time(w, seqs, window=window)
     reps = max(1, int(target_s / max(t, 1e-6)))
     if reps > 1:
-        t, s = oracle_step_time(w, seqs, reps)
-    nbytes = A.step_bytes(s)["total"] * reps
+        t, s, out = oracle_step_time(w, seqs, reps, window=window)
+    nbytes = A.step_bytes(s, window=window)["total"] * reps
     return {"value": nbytes / t / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"{n} of {w.batch} sequences x {reps} passes (copies + append + decode), "
                       f"{t:.1f} s, float64 C oracle, OpenMP over (sequence, head)",
-            "seconds": t, "tokens_per_s_per_layer": n * reps / t}
+            "seconds": t, "tokens_per_s_per_layer": n * reps / t}, seqs, out
+
+
+# decode tolerance on max-abs error against the float64 oracle, by output dtype
+TOLERANCE = {"f16": 2e-3, "bf16": 1e-2}
+
+
+def parity_summary(got: np.ndarray, want: np.ndarray, io_dtype: str) -> dict:
+    """Max-abs error of the GPU output (float64 [n, Hq, D]) against the
+    oracle's for the same sequences."""
+    diff = np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64))
+    err = float(diff.max()) if diff.size else 0.0
+    finite = math.isfinite(err)
+    tol = TOLERANCE[io_dtype]
+    return {"max_abs_err": err if finite else None, "tolerance": tol,
+            "sequences": int(got.shape[0]), "ok": bool(finite and err <= tol),
+            "against": "float64 CPU oracle, same inputs, the cpu_baseline sample"}
 
 
 # ----------------------------------------------------------------- main ----
@@ -277,7 +298,7 @@ def run_reference(args):
     oracle.build()
     # per-step sample sized so warmup + steps fit in about two minutes
     budget = min(10.0, 120.0 / max(1, args.steps + args.warmup))
-    t1, _ = oracle_step_time(w, np.arange(1))
+    t1, _, _ = oracle_step_time(w, np.arange(1))
     n = int(min(w.batch, max(1, budget / max(t1, 1e-4))))
     seqs = np.arange(n)
     for _ in range(args.warmup):
@@ -285,7 +306,7 @@ def run_reference(args):
     times = []
     s = None
     for _ in range(args.steps):
-        t, s = oracle_step_time(w, seqs)
+        t, s, _ = oracle_step_time(w, seqs)
         times.append(t)
     total = sum(times)
     nbytes = A.step_bytes(s)["total"] * args.steps
@@ -462,7 +483,13 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        line["cpu_baseline"] = cpu_baseline(w)
+        cb, seqs, want = cpu_baseline(w, window=args.window)
+        line["cpu_baseline"] = cb
+        try:  # the GPU's output for the sampled sequences (last e2e step, same inputs)
+            got = step.out.double().cpu().numpy()[seqs]
+            line["parity"] = parity_summary(got, want, w.io_dtype)
+        except Exception as e:  # report, never lose the measured line
+            line["parity"] = {"error": repr(e)}
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

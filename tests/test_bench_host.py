@@ -87,8 +87,33 @@ def test_reference_arm_on_the_fp8_beams_workload():
 def test_oracle_step_covers_copies_append_and_decode():
     from paged_kv_cache_410_b200 import workloads as W
     w = W.fp8_beams(batch=24, beam_groups=2, median_len=40, max_len=200)
-    t, s = bench.oracle_step_time(w, np.arange(8))
+    t, s, out = bench.oracle_step_time(w, np.arange(8))
+    assert out.shape == (8, w.num_q_heads, w.head_dim) and np.isfinite(out).all()
     assert t > 0 and s.batch == 8 and len(s.copy_pairs) == len(w.copy_pairs)
     kc, vc = bench.oracle_caches(w)
     assert kc.dtype == np.uint8 and kc.any()              # filled by the oracle's append
     assert bench.oracle_caches(w)[0] is kc                # made once per workload
+
+
+def test_parity_summary_against_the_oracle_sample():
+    """The bench line's parity check: the oracle's output for the cpu_baseline
+    sample, compared with the device output of the same sequences."""
+    import oracle
+    from paged_kv_cache_410_b200 import workloads as W
+    w = W.custom([5, 40, 77, 130], num_q_heads=8, num_kv_heads=2, head_dim=64)
+    cb, seqs, want = bench.cpu_baseline(w, target_s=0.2, window=32)
+    assert cb["kind"] == "oracle" and len(seqs) == 4
+    # the sample's output is the oracle's windowed decode after the append
+    kc, vc = bench.oracle_caches(w)
+    direct = oracle.decode(w.q, "f16", kc, vc, "f16", w.block_tables, w.context_lens, w.scale,
+                           window=32)
+    assert np.array_equal(want, direct[seqs])
+    ok = bench.parity_summary(want + 1e-3, want, "f16")
+    assert ok["ok"] and abs(ok["max_abs_err"] - 1e-3) < 1e-12 and ok["sequences"] == 4
+    bad = bench.parity_summary(want + 3e-3, want, "f16")
+    assert not bad["ok"] and bad["tolerance"] == 2e-3
+    assert bench.parity_summary(want + 3e-3, want, "bf16")["ok"]
+    nan = want.copy()
+    nan[0, 0, 0] = np.nan
+    r = bench.parity_summary(nan, want, "f16")
+    assert r["max_abs_err"] is None and not r["ok"]
