@@ -180,6 +180,12 @@ def _families():
         ("prefix", W.custom_shared_prefix(64, [10, 20, 30]), {"shared_prefix_blocks": 4}),
         ("fp8_beams", fp8, {}),
         ("fp8_subset", W.subset(fp8, [0, 5, 9, 20]), {"fused": True}),
+        # the workloads of __graft_entry__.smoke()
+        ("smoke_fp8", W.fp8_beams(batch=12, beam_groups=1, block_size=16), {}),
+        ("smoke_prefix", W.custom_shared_prefix(128, [0, 5, 40, 300], num_q_heads=8,
+                                                num_kv_heads=2, head_dim=128, block_size=16,
+                                                dtype="bf16", seed=7),
+         {"shared_prefix_blocks": 8}),
     ]
 
 
