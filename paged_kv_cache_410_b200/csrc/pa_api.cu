@@ -466,7 +466,6 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
     return PA_ERR_CUDA;
   pa::UmmaGrid ug{};
   ug.n_chunks = pl.num_chunks;
-  ug.withhold_scores = g_withhold_prefix_scores;
   ug.seqs_per_tile = pa::kUmmaRows / p.group;
   const int seqs_per_cta = kUmmaTiles * ug.seqs_per_tile;
   ug.n_rowtiles = (p.batch + seqs_per_cta - 1) / seqs_per_cta;
@@ -506,6 +505,7 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
   const int64_t ctas = static_cast<int64_t>(ug.n_chunks) * ug.n_rowtiles * p.num_kv_heads;
   if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_side_mu);
+  ug.withhold_scores = g_withhold_prefix_scores;  // written under the same lock
   SideStream* ss = nullptr;
   if (side_stream(&ss) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
