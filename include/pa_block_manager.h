@@ -75,6 +75,19 @@ int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* 
 int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, int64_t* slot,
                            int32_t* cow_src, int32_t* cow_dst);
 
+/* pa_bm_append_token for a batch: one token (tokens[i]) for each of the n
+ * distinct sequences seq_ids[i], in order, in one call. slots[n] receives
+ * each token's slot; the copy-on-write pairs the batch needs, in order, go
+ * to cow_pairs ([n][2] int32 (src, dst), room for n pairs) and their count to
+ * *num_pairs; apply them (pa_copy_blocks) before appending K/V. A sequence
+ * that copies drops its share of the old block, so a later sequence of the
+ * batch that shared it with that one alone writes in place. Returns
+ * PA_BM_ERR_INVALID for an unknown or repeated id and PA_BM_ERR_NO_BLOCKS if
+ * the pool (after evicting cached blocks) cannot supply the batch; either
+ * way nothing has changed. */
+int32_t pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, const int32_t* tokens,
+                            int32_t n, int64_t* slots, int32_t* cow_pairs, int32_t* num_pairs);
+
 /* child_id starts as a copy of parent_id that shares all its blocks. */
 int32_t pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id);
 

@@ -13,7 +13,8 @@ OK, ERR_INVALID, ERR_NO_BLOCKS, ERR_CAPACITY = 0, -1, -2, -3
 EXPORTED = ["pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_num_cached_blocks",
             "pa_bm_block_refcount", "pa_bm_add_sequence", "pa_bm_append_token", "pa_bm_fork",
             "pa_bm_free_sequence", "pa_bm_release_before", "pa_bm_sequence_length",
-            "pa_bm_slots", "pa_bm_block_tables", "pa_bm_block_tables_update"]
+            "pa_bm_slots", "pa_bm_block_tables", "pa_bm_block_tables_update",
+            "pa_bm_append_tokens"]
 
 _declared = False
 
@@ -38,6 +39,8 @@ def _lib():
         lib.pa_bm_append_token.argtypes = [P, i64, i32, ctypes.POINTER(i64), ctypes.POINTER(i32),
                                            ctypes.POINTER(i32)]
         lib.pa_bm_append_token.restype = i32
+        lib.pa_bm_append_tokens.argtypes = [P, P, P, i32, P, P, ctypes.POINTER(i32)]
+        lib.pa_bm_append_tokens.restype = i32
         lib.pa_bm_fork.argtypes = [P, i64, i64]
         lib.pa_bm_fork.restype = i32
         lib.pa_bm_free_sequence.argtypes = [P, i64]
@@ -114,6 +117,22 @@ class BlockManager:
                                           ctypes.byref(src), ctypes.byref(dst))
         _ok(rc, "pa_bm_append_token")
         return int(slot.value), (None if src.value < 0 else (int(src.value), int(dst.value)))
+
+    def append_tokens(self, seq_ids, tokens):
+        """One token for each listed sequence in one call. Returns (slots int64 [n],
+        copy-on-write pairs int32 [k, 2] to apply before the append)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        if toks.shape != ids.shape or ids.ndim != 1:
+            raise BlockManagerError(ERR_INVALID, "pa_bm_append_tokens")
+        n = len(ids)
+        slots = np.empty(n, dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int32)
+        k = ctypes.c_int32(0)
+        rc = self._lib.pa_bm_append_tokens(self._h, ids.ctypes.data, toks.ctypes.data, n,
+                                           slots.ctypes.data, pairs.ctypes.data, ctypes.byref(k))
+        _ok(rc, "pa_bm_append_tokens")
+        return slots, pairs[:k.value].copy()
 
     def fork(self, parent_id: int, child_id: int):
         _ok(self._lib.pa_bm_fork(self._h, parent_id, child_id), "pa_bm_fork")

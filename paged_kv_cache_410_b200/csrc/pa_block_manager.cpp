@@ -34,6 +34,7 @@ struct Seq {
   Node* tail = nullptr;          // tree node of the last leading block known to the cache
   int32_t tail_blocks = 0;       // leading blocks covered by the path ending at `tail`
   uint64_t version = 0;          // stamp of the last change to `blocks` (never 0)
+  uint64_t batch = 0;            // last batched call that listed this sequence
 };
 
 uint64_t hash_tokens(const int32_t* t, int32_t n) {
@@ -62,6 +63,7 @@ struct pa_block_manager {
   std::set<std::pair<uint64_t, int64_t>> evictable;           // (last_use, block)
   uint64_t tick = 0;
   uint64_t versions = 0;  // last stamp handed out; stamps are unique across sequences
+  uint64_t batches = 0;   // batched calls so far (duplicate ids within one are refused)
 
   void changed(Seq& s) { s.version = ++versions; }
 
@@ -155,6 +157,62 @@ struct pa_block_manager {
     ++refcount[b];
     auto it = nodes.find(b);
     if (it != nodes.end()) track(it->second.get());
+  }
+
+  // Appends one token to `s`: a new block at a block boundary, a private
+  // copy of a shared partial last block (copy on write), else the next row of
+  // the last block. Fails (changing nothing) only if a block is needed and
+  // none can be had.
+  int32_t append_one(Seq& s, int32_t token, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
+    const int32_t pos = s.length;
+    int32_t src = -1, dst = -1;
+    if (pos % bs == 0) {
+      const int64_t b = alloc();
+      if (b < 0) return PA_BM_ERR_NO_BLOCKS;
+      s.blocks.push_back(b);
+      changed(s);
+    } else {
+      const int64_t last = s.blocks.back();
+      if (refcount[last] > 1) {  // shared partial block: copy on write
+        const int64_t b = alloc();
+        if (b < 0) return PA_BM_ERR_NO_BLOCKS;
+        src = static_cast<int32_t>(last);
+        dst = static_cast<int32_t>(b);
+        unref(last);
+        s.blocks.back() = b;
+        changed(s);
+      }
+    }
+    *slot = s.blocks[pos / bs] * bs + pos % bs;
+    *cow_src = src;
+    *cow_dst = dst;
+    s.tokens.push_back(token);
+    s.length = pos + 1;
+    if (s.length % bs == 0) cache_full_block(s, s.length / bs - 1);
+    return PA_BM_OK;
+  }
+
+  // Blocks that one append to each of `rows` (distinct sequences, in this
+  // order) takes: one at each block boundary, one for each copy on write.
+  // A sequence that copies drops its share of the old block, so a later row
+  // that shared it with only that sequence writes in place.
+  int64_t blocks_for_appends(const std::vector<Seq*>& rows) const {
+    std::unordered_map<int64_t, int32_t> dropped;
+    int64_t need = 0;
+    for (const Seq* r : rows) {
+      if (r->length % bs == 0) {
+        ++need;
+        continue;
+      }
+      const int64_t last = r->blocks.back();
+      if (refcount[last] == 1) continue;  // private: written in place
+      int32_t& d = dropped[last];
+      if (refcount[last] - d > 1) {
+        ++need;
+        ++d;
+      }
+    }
+    return need;
   }
 
   // Block `index` of `s` is full: extend the cached path with it.
@@ -290,33 +348,42 @@ int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, 
   if (!bm || !slot) return PA_BM_ERR_INVALID;
   auto it = bm->seqs.find(seq_id);
   if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
-  Seq& s = it->second;
-  const int32_t bs = bm->bs;
-  const int32_t pos = s.length;
   int32_t src = -1, dst = -1;
-  if (pos % bs == 0) {
-    const int64_t b = bm->alloc();
-    if (b < 0) return PA_BM_ERR_NO_BLOCKS;
-    s.blocks.push_back(b);
-    bm->changed(s);
-  } else {
-    const int64_t last = s.blocks.back();
-    if (bm->refcount[last] > 1) {  // shared partial block: copy on write
-      const int64_t b = bm->alloc();
-      if (b < 0) return PA_BM_ERR_NO_BLOCKS;
-      src = static_cast<int32_t>(last);
-      dst = static_cast<int32_t>(b);
-      bm->unref(last);
-      s.blocks.back() = b;
-      bm->changed(s);
-    }
-  }
-  *slot = s.blocks[pos / bs] * bs + pos % bs;
+  const int32_t rc = bm->append_one(it->second, token, slot, &src, &dst);
+  if (rc != PA_BM_OK) return rc;
   if (cow_src) *cow_src = src;
   if (cow_dst) *cow_dst = dst;
-  s.tokens.push_back(token);
-  s.length = pos + 1;
-  if (s.length % bs == 0) bm->cache_full_block(s, s.length / bs - 1);
+  return PA_BM_OK;
+}
+
+int32_t pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, const int32_t* tokens,
+                            int32_t n, int64_t* slots, int32_t* cow_pairs, int32_t* num_pairs) {
+  if (!bm || n < 0 || !num_pairs || (n > 0 && (!seq_ids || !tokens || !slots || !cow_pairs)))
+    return PA_BM_ERR_INVALID;
+  // every id known and distinct, and every block the batch needs obtainable,
+  // before anything changes
+  std::vector<Seq*> rows(static_cast<size_t>(n));
+  const uint64_t mark = ++bm->batches;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end() || it->second.batch == mark) return PA_BM_ERR_INVALID;
+    it->second.batch = mark;
+    rows[static_cast<size_t>(i)] = &it->second;
+  }
+  if (!bm->can_reclaim(bm->blocks_for_appends(rows))) return PA_BM_ERR_NO_BLOCKS;
+  int32_t pairs = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    int32_t src = -1, dst = -1;
+    if (bm->append_one(*rows[static_cast<size_t>(i)], tokens[i], &slots[i], &src, &dst) !=
+        PA_BM_OK)
+      return PA_BM_ERR_NO_BLOCKS;  // not reached: the blocks were counted above
+    if (src >= 0) {
+      cow_pairs[2 * pairs] = src;
+      cow_pairs[2 * pairs + 1] = dst;
+      ++pairs;
+    }
+  }
+  *num_pairs = pairs;
   return PA_BM_OK;
 }
 

@@ -288,6 +288,7 @@ def test_host_benchmark_runs():
     assert r["forks"] == 40 and r["cow_pairs"] > 0
     assert r["append_ns_per_token"] > 0 and r["step_us"] > 0
     assert 0 < r["block_tables_update_us_per_step"] and 0 < r["rows_rewritten_per_step"] < 16
+    assert r["append_batched_ns_per_token"] > 0     # the batched pass gave the same slots
 
 
 def _check_contents(bm, seqs, released, content, bs):
@@ -328,7 +329,8 @@ def _random_serving(seed):
         return bm.num_free_blocks, bm.num_cached_blocks
 
     for step in range(400):
-        op = rng.choice(["add", "append", "append", "append", "fork", "free", "release"])
+        op = rng.choice(["add", "append", "append", "append", "batch", "fork", "free",
+                         "release"])
         live = list(seqs)
         if op == "add" or not live:
             toks = [int(t) for t in systems[int(rng.integers(0, 3))]]
@@ -370,6 +372,29 @@ def _random_serving(seed):
                         content.pop(dst * bs + r, None)
             write(slot, tok)
             seqs[sid] = seqs[sid] + [tok]
+        elif op == "batch":
+            # one token for several sequences in one call: every copy pair is
+            # applied first, then every new token is written
+            k = int(rng.integers(1, len(live) + 1))
+            sids = [live[i] for i in rng.choice(len(live), size=k, replace=False)]
+            toks = [int(t) for t in rng.integers(0, 5, size=k)]
+            before = snapshot()
+            try:
+                slots, pairs = bm.append_tokens(sids, toks)
+            except BM.BlockManagerError as e:
+                assert e.code == BM.ERR_NO_BLOCKS and snapshot() == before
+                failures += 1
+                continue
+            for src, dst in pairs.tolist():
+                copies += 1
+                for r in range(bs):
+                    if src * bs + r in content:
+                        content[dst * bs + r] = content[src * bs + r]
+                    else:
+                        content.pop(dst * bs + r, None)
+            for sid, slot, tok in zip(sids, slots.tolist(), toks):
+                write(slot, tok)
+                seqs[sid] = seqs[sid] + [tok]
         elif op == "fork":
             parent = live[int(rng.integers(0, len(live)))]
             bm.fork(parent, next_id)
@@ -414,3 +439,61 @@ def test_random_serving_reaches_every_case():
     assert sum(s["copies"] for s in stats) > 20
     assert sum(s["failures"] for s in stats) > 5
     assert all(s["seqs"] > 20 for s in stats)
+
+
+def test_batched_appends_equal_one_by_one():
+    """pa_bm_append_tokens gives the slots and copy pairs that the same
+    appends made one call at a time give, including beams that shared a
+    partial block (the last beam to append writes in place)."""
+    def setup():
+        bm = BM.BlockManager(200, 4, prefix_cache=True)
+        bm.add_sequence(0, range(10))                # 2 full blocks + 2 tokens
+        for c in (1, 2, 3):
+            bm.fork(0, c)                            # 4 beams share the partial block
+        bm.add_sequence(4, range(100, 108))          # ends on a block boundary
+        bm.add_sequence(5, range(100, 103))
+        return bm
+    one, many = setup(), setup()
+    for step in range(9):
+        ids = [3, 0, 4, 1, 5, 2] if step % 2 else [0, 1, 2, 3, 4, 5]
+        toks = [step * 10 + i for i in ids]
+        want_slots, want_pairs = [], []
+        for sid, t in zip(ids, toks):
+            slot, cow = one.append_token(sid, t)
+            want_slots.append(slot)
+            if cow:
+                want_pairs.append(cow)
+        slots, pairs = many.append_tokens(ids, toks)
+        assert slots.tolist() == want_slots, step
+        assert [tuple(p) for p in pairs.tolist()] == want_pairs, step
+        if step == 0:
+            assert len(pairs) == 3                   # three beams copy, the fourth writes in place
+    t1, l1 = one.block_tables(range(6), 8)
+    t2, l2 = many.block_tables(range(6), 8)
+    assert (t1 == t2).all() and (l1 == l2).all()
+    assert one.num_free_blocks == many.num_free_blocks
+    assert one.num_cached_blocks == many.num_cached_blocks
+
+
+def test_batched_appends_change_nothing_on_error():
+    bm = BM.BlockManager(4, 2)
+    bm.add_sequence(1, [1, 2])                       # 1 block, full
+    bm.add_sequence(2, [3])                          # 1 block, half
+    bm.fork(2, 3)                                    # shares the half block
+    before = (bm.num_free_blocks, bm.block_tables([1, 2, 3], 3))
+    for ids in ([1, 9], [1, 1], [2, 2]):
+        with pytest.raises(BM.BlockManagerError) as e:
+            bm.append_tokens(ids, [0] * len(ids))
+        assert e.value.code == BM.ERR_INVALID
+    # 1 needs a new block, 2 copies the shared block, 3 then writes in place: 2 blocks, 2 free
+    slots, pairs = bm.append_tokens([1, 2, 3], [7, 8, 9])
+    assert len(pairs) == 1 and bm.num_free_blocks == 0
+    # now sequences 2 and 3 each need a new block and none is left
+    state = (bm.num_free_blocks, bm.block_tables([1, 2, 3], 3))
+    with pytest.raises(BM.BlockManagerError) as e:
+        bm.append_tokens([1, 2, 3], [0, 0, 0])
+    assert e.value.code == BM.ERR_NO_BLOCKS
+    after = (bm.num_free_blocks, bm.block_tables([1, 2, 3], 3))
+    assert state[0] == after[0] and all((a == b).all() for a, b in zip(state[1], after[1]))
+    assert before[0] == 2
+    assert bm.append_tokens([], [])[0].shape == (0,)
