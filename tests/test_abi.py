@@ -261,9 +261,16 @@ int main(void) {
   rc |= pa_bm_add_sequence(bm, 2, toks, 40, &cached);
   rc |= pa_bm_append_token(bm, 2, 7, &slot, &src, &dst);
   rc |= pa_bm_block_tables(bm, ids, 2, 4, tables, lens);
-  printf("%d|%s|%zu|%d|%d|%d|%d|%d|%d|%d|%d\n", (int)pa_version(),
+  /* one token for both sequences in one call, then the incremental export */
+  int64_t bslots[2];
+  int32_t btoks[2] = {8, 9}, bpairs[4], npairs = -1, kept[8], klens[2], written = -1;
+  uint64_t versions[2] = {0, 0};
+  rc |= pa_bm_append_tokens(bm, ids, btoks, 2, bslots, bpairs, &npairs);
+  rc |= pa_bm_block_tables_update(bm, ids, 2, 4, kept, klens, versions, &written);
+  printf("%d|%s|%zu|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d\n", (int)pa_version(),
          pa_status_string(PA_ERR_WORKSPACE), ws, (int)pt, (int)bad, rc, (int)cached, (int)src,
-         (int)lens[0], (int)lens[1], tables[0] == tables[4] && tables[1] == tables[5]);
+         (int)lens[0], (int)lens[1], tables[0] == tables[4] && tables[1] == tables[5],
+         (int)npairs, (int)written, (int)klens[0], (int)klens[1]);
   pa_bm_destroy(bm);
   return 0;
 }
@@ -296,3 +303,6 @@ def test_headers_are_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert int(f[7]) == -1                        # the partial block was private: no copy
     assert (int(f[8]), int(f[9])) == (40, 41)
     assert int(f[10]) == 1                        # both tables start with the same blocks
+    assert int(f[11]) == 0                        # no shared partial block: no copies
+    assert int(f[12]) == 2                        # first incremental export writes both rows
+    assert (int(f[13]), int(f[14])) == (41, 42)
