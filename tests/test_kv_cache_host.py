@@ -1,0 +1,127 @@
+"""PagedKVCache (paged_kv_cache_410_b200/kv_cache.py) on the CPU: the step
+plans it uploads follow the host block manager exactly (slots, copy-on-write
+pairs, tables, lengths), copies reach every layer, and each layer's decode is
+one pa_append_decode call on the plan's tensors. The CUDA library is replaced
+by a recording stand-in (the block manager is the real C++ one), so no GPU
+and no kernel is involved."""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_410_b200 import binding as B
+from paged_kv_cache_410_b200.block_manager import BlockManager
+from paged_kv_cache_410_b200.kv_cache import PagedKVCache
+
+
+class Recorder:
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append((name, args))
+            return 0
+        return fn
+
+
+@pytest.fixture
+def rec(monkeypatch):
+    r = Recorder()
+    monkeypatch.setattr(B, "load_library", lambda *a, **k: r)
+    monkeypatch.setattr(B, "_on_device", lambda t: True)
+    return r
+
+
+NB, BS, HKV, D, HQ, LAYERS, MB = 64, 4, 2, 64, 8, 3, 16
+
+
+def kv(n):
+    return torch.zeros((n, HKV, D), dtype=torch.float16)
+
+
+def test_steps_follow_the_block_manager(rec):
+    cache = PagedKVCache(NB, BS, HKV, D, num_layers=LAYERS, device="cpu", max_batch=8, stream=0,
+                         max_blocks_per_seq=MB)
+    twin = BlockManager(NB, BS, prefix_cache=True)
+    prompt = list(range(10))                          # 2 full blocks + 2 tokens
+    cached, slots = cache.add_sequence(0, prompt)
+    twin.add_sequence(0, prompt)
+    assert cached == 0 and slots.tolist() == twin.slots(0, 0, 10).tolist()
+    for layer in range(LAYERS):
+        cache.store_prompt(layer, slots, kv(10), kv(10))
+    stores = [a for n, a in rec.calls if n == "pa_append_kv"]
+    assert [a[5] for a in stores] == [t.data_ptr() for t in cache.k]  # one store per layer
+    for c in (1, 2):                                  # two beams share every block
+        cache.fork(0, c)
+        twin.fork(0, c)
+    order = [[0, 1, 2], [2, 0, 1], [1, 2, 0], [0, 1, 2], [2, 1, 0]]
+    for step, ids in enumerate(order):
+        toks = [100 * step + i for i in ids]
+        rec.calls.clear()
+        plan = cache.begin_step(ids, toks)
+        want_slots, want_pairs = [], []
+        for sid, t in zip(ids, toks):
+            s, cow = twin.append_token(sid, t)
+            want_slots.append(s)
+            if cow:
+                want_pairs.append(list(cow))
+        assert plan.slot_mapping.tolist() == want_slots, step
+        assert plan.copy_pairs.tolist() == want_pairs, step
+        tables, lens = twin.block_tables(ids, MB)
+        assert np.array_equal(plan.block_tables.numpy(), tables), step
+        assert plan.context_lens.tolist() == lens.tolist() and plan.max_context == lens.max()
+        copies = [a for n, a in rec.calls if n == "pa_copy_blocks_layers"]
+        if want_pairs:                                # one call for all layers
+            assert len(copies) == 1 and copies[0][1] == len(want_pairs) and copies[0][4] == LAYERS
+            assert [copies[0][2][i] for i in range(LAYERS)] == [t.data_ptr() for t in cache.k]
+        else:
+            assert copies == []
+        if step == 0:
+            assert len(want_pairs) == 2               # two beams copy, the last writes in place
+        rec.calls.clear()
+        for layer in range(LAYERS):
+            q = torch.zeros((len(ids), HQ, D), dtype=torch.float16)
+            k, v = kv(len(ids)), kv(len(ids))
+            out = cache.attend(plan, layer, q, k, v)
+            name, a = [c for c in rec.calls if c[0] == "pa_append_decode"][-1]
+            assert a[0] == q.data_ptr() and a[1] == k.data_ptr() and a[2] == v.data_ptr()
+            assert a[6] == plan.slot_mapping.data_ptr() and a[7] == cache.k[layer].data_ptr()
+            assert a[10] == plan.block_tables.data_ptr() and a[11] == MB
+            assert a[12] == plan.context_lens.data_ptr() and a[13] == plan.max_context
+            assert abs(a[14] - 1 / 8) < 1e-12 and a[15] == out.data_ptr()
+
+
+def test_prefix_cache_serves_a_second_prompt(rec):
+    cache = PagedKVCache(NB, BS, HKV, D, device="cpu", max_batch=4, max_blocks_per_seq=MB,
+                         stream=0)
+    system = list(range(50, 58))                      # two full blocks
+    c1, s1 = cache.add_sequence(1, system + [1, 2])
+    c2, s2 = cache.add_sequence(2, system + [3])
+    assert (c1, c2) == (0, 8) and len(s2) == 1        # only the new token's K/V is stored
+    plan = cache.begin_step([1, 2], [7, 7])
+    assert (plan.block_tables[0, :2] == plan.block_tables[1, :2]).all()
+
+
+def test_e4m3_layers_carry_their_scales(rec):
+    ks = [torch.full((HKV, D), 0.5 + l) for l in range(2)]
+    vs = [torch.full((HKV, D), 2.0 + l) for l in range(2)]
+    cache = PagedKVCache(NB, BS, HKV, D, num_layers=2, dtype=torch.uint8,
+                         io_dtype=torch.bfloat16, device="cpu", k_scales=ks, v_scales=vs,
+                         stream=0)
+    assert torch.equal(cache.layers[1].k_inv_scale, 1.0 / ks[1])
+    cached, slots = cache.add_sequence(0, [1, 2, 3])
+    cache.store_prompt(1, slots, torch.zeros((3, HKV, D), dtype=torch.bfloat16),
+                       torch.zeros((3, HKV, D), dtype=torch.bfloat16))
+    d = rec.calls[-1][1][7]._obj
+    assert d.cache_dtype == B.PA_E4M3 and d.k_scale == cache.layers[1].k_scale.data_ptr()
+    with pytest.raises(ValueError):
+        PagedKVCache(NB, BS, HKV, D, dtype=torch.uint8, device="cpu")   # no io dtype / scales
+
+
+def test_batch_limit(rec):
+    cache = PagedKVCache(NB, BS, HKV, D, device="cpu", max_batch=2, max_blocks_per_seq=MB,
+                         stream=0)
+    for s in range(3):
+        cache.add_sequence(s, [s])
+    with pytest.raises(ValueError):
+        cache.begin_step([0, 1, 2], [0, 0, 0])
