@@ -306,3 +306,47 @@ def test_headers_are_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert int(f[11]) == 0                        # no shared partial block: no copies
     assert int(f[12]) == 2                        # first incremental export writes both rows
     assert (int(f[13]), int(f[14])) == (41, 42)
+
+
+def test_workspace_sizes_cover_every_partition_plan(lib):
+    """The partition-length queries and the workspace-size queries come from
+    one planner: over random shapes, the workspace each size query asks for
+    holds exactly (plain, window) or at least (shared prefix: one or more
+    prefix chunks besides) the partials the partition queries imply."""
+    rng = np.random.default_rng(11)
+
+    def need(batch, hq, parts, d):
+        o, ml = batch * hq * parts * d * 4, batch * hq * parts * 8
+        return -(-o // 256) * 256 + -(-ml // 256) * 256
+
+    for _ in range(400):
+        hkv = int(rng.choice([1, 2, 8, 32]))
+        hq = hkv * int(rng.choice([1, 2, 4, 8, 16]))
+        d = int(rng.choice([64, 128]))
+        bs = int(rng.choice([1, 8, 16, 64, 256]))
+        dt = int(rng.choice([B.PA_F16, B.PA_BF16, B.PA_E4M3]))
+        batch = int(rng.integers(1, 300))
+        maxc = int(rng.integers(0, 200000))
+        desc = ctypes.byref(_desc(num_kv_heads=hkv, head_dim=d, block_size=bs, cache_dtype=dt,
+                                  num_blocks=1 << 20))
+        pt = lib.pa_decode_partition_tokens(batch, maxc, desc)
+        assert pt >= 64 and pt % 16 == 0
+        parts = max(1, -(-maxc // pt))
+        ws = lib.pa_decode_workspace_size(batch, hq, maxc, 0, desc)
+        assert ws == (need(batch, hq, parts, d) if parts > 1 else 0)
+        # sliding window: the plan spans at most window + 15 tokens
+        window = int(rng.integers(1, 10000))
+        span = min(maxc, window + 15)
+        ptw = lib.pa_decode_partition_tokens(batch, span, desc)
+        partsw = max(1, -(-span // ptw))
+        wsw = lib.pa_decode_sliding_window_workspace_size(batch, hq, maxc, window, 0, desc)
+        assert wsw == (need(batch, hq, partsw, d) if partsw > 1 else 0)
+        # shared prefix: prefix chunks plus the suffix partitions
+        pb = int(rng.integers(1, maxc // bs + 2))
+        if pb * bs > maxc:
+            continue
+        pts = lib.pa_decode_shared_prefix_partition_tokens(batch, hq, maxc, pb, desc)
+        assert pts >= 16 and pts % 16 == 0
+        sparts = -(-(maxc - pb * bs) // pts)
+        wss = lib.pa_decode_shared_prefix_workspace_size(batch, hq, maxc, pb, 0, desc)
+        assert wss >= need(batch, hq, 1 + sparts, d)
