@@ -233,16 +233,18 @@ size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads
  * handled as in pa_decode, and the two are merged as split-K partials.
  * A sequence whose table or length breaks the precondition sets
  * PA_DEVERR_PREFIX (its output is then not meaningful).
- * 16-bit caches: the prefix part runs on tcgen05 tensor cores, on a stream
- * the library owns (one per device, created at the first call): the call
+ * 16-bit caches with blocks of at least 8 tokens, at most 128 query heads
+ * per KV head and fewer than 2^31 slots: the prefix part runs on tcgen05
+ * tensor cores, on a stream the library owns (one per device, created at the
+ * first call): the call
  * records an event on `stream`, makes its stream wait for it, launches the
  * prefix kernel there, and makes `stream` wait for that kernel before the
  * merge. Work enqueued on `stream` after the call therefore sees the
  * complete result, and the call can be captured into a CUDA graph from
  * `stream`. Calls from several host threads are serialised around the
  * fork and join. A tensor-core wait that gives up (1 s) sets
- * PA_DEVERR_TIMEOUT. E4M3 caches run the prefix on mma.sync in the same
- * launch as the suffixes.
+ * PA_DEVERR_TIMEOUT. Other caches (E4M3, smaller blocks, larger groups) run
+ * the prefix on mma.sync in the same launch as the suffixes.
  *   prefix_blocks  number of shared leading blocks (0: plain pa_decode);
  *                  prefix_blocks * block_size must not exceed max_context.
  *   workspace      at least pa_decode_shared_prefix_workspace_size(...) bytes,
