@@ -16,7 +16,11 @@ block manager, one multi-layer block copy for the beams that diverge, the
 block-table rows that changed since the last step, and one upload of slots,
 tables and lengths from pinned memory. ``attend`` is one
 ``pa_append_decode`` launch per layer (the new token's K/V is stored and
-attended in the same kernel). Prompts: ``add_sequence`` places a prompt,
+attended in the same kernel), or, when every sequence of the step starts
+with the same run of at least ``shared_prefix_min_blocks`` physical blocks
+(a system prompt served from the prefix cache), an append and
+``pa_decode_shared_prefix``, which attends that prefix once for the whole
+batch. Prompts: ``add_sequence`` places a prompt,
 reusing cached prefix blocks, and returns the slots of the tokens whose K/V
 the caller still has to store (``store_prompt``).
 """
@@ -45,6 +49,7 @@ class StepPlan:
     context_lens: torch.Tensor   # int32 [n], the new token included
     max_context: int
     copy_pairs: np.ndarray       # int32 [k, 2] copied (every layer) before the step
+    shared_prefix_blocks: int    # leading blocks every sequence's table shares
 
 
 class PagedKVCache:
@@ -59,9 +64,10 @@ class PagedKVCache:
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
                  num_layers: int = 1, dtype=torch.float16, io_dtype=None, device="cuda",
                  prefix_cache: bool = True, max_batch: int = 256, max_blocks_per_seq: int = 512,
-                 k_scales=None, v_scales=None, stream=None):
+                 k_scales=None, v_scales=None, stream=None, shared_prefix_min_blocks: int = 32):
         self.device = torch.device(device)
         self.stream = stream
+        self.shared_prefix_min_blocks = shared_prefix_min_blocks
         self.block_size = block_size
         self.num_kv_heads = num_kv_heads
         self.head_dim = head_dim
@@ -152,30 +158,63 @@ class PagedKVCache:
             if self.device.type == "cuda":
                 self._uploaded = torch.cuda.Event()
                 self._uploaded.record()
+        shared = 0
+        if self.shared_prefix_min_blocks > 0:
+            shared = common_prefix_blocks(self._h_tables.numpy()[:n], h_lens[:n],
+                                          self.block_size)
         return StepPlan(n=n, slot_mapping=self._d_slots[:n], block_tables=self._d_tables[:n],
                         context_lens=self._d_lens[:n],
-                        max_context=int(h_lens[:n].max()) if n else 0, copy_pairs=pairs)
+                        max_context=int(h_lens[:n].max()) if n else 0, copy_pairs=pairs,
+                        shared_prefix_blocks=shared)
 
     def attend(self, plan: StepPlan, layer: int, q, k, v, scale: float | None = None, out=None):
         """Store this layer's new K/V (k, v [n, Hkv, D]) at the plan's slots and
-        return the decode output [n, Hq, D] for queries q [n, Hq, D]; both in
-        one kernel launch (pa_append_decode)."""
+        return the decode output [n, Hq, D] for queries q [n, Hq, D]: one
+        pa_append_decode launch, or pa_append_kv + pa_decode_shared_prefix
+        when the plan's shared prefix is long enough."""
         if out is None:
             out = torch.empty_like(q)
         if scale is None:
             scale = 1.0 / math.sqrt(self.head_dim)
         cache = self.layers[layer]
-        need = B.pa_decode_workspace_size(plan.n, q.shape[1], plan.max_context, cache)
+        spb = plan.shared_prefix_blocks
+        cascade = self.shared_prefix_min_blocks > 0 and spb >= self.shared_prefix_min_blocks
+        if cascade:
+            need = B.pa_decode_shared_prefix_workspace_size(plan.n, q.shape[1], plan.max_context,
+                                                            spb, cache)
+        else:
+            need = B.pa_decode_workspace_size(plan.n, q.shape[1], plan.max_context, cache)
         if need and (self._workspace is None or self._workspace.numel() < need):
             with self._on_stream():
                 self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
-        B.pa_append_decode(q, k, v, plan.slot_mapping, self.k[layer], self.v[layer],
-                           plan.block_tables, plan.context_lens, scale, out, cache,
-                           plan.max_context, workspace=self._workspace if need else None,
-                           stream=self.stream)
+        ws = self._workspace if need else None
+        if cascade:
+            B.pa_append_kv(k, v, plan.slot_mapping, self.k[layer], self.v[layer], cache,
+                           self.stream)
+            B.pa_decode_shared_prefix(q, self.k[layer], self.v[layer], plan.block_tables,
+                                      plan.context_lens, scale, out, cache, plan.max_context,
+                                      spb, workspace=ws, stream=self.stream)
+        else:
+            B.pa_append_decode(q, k, v, plan.slot_mapping, self.k[layer], self.v[layer],
+                               plan.block_tables, plan.context_lens, scale, out, cache,
+                               plan.max_context, workspace=ws, stream=self.stream)
         return out
 
     def _on_stream(self):
         if self.device.type == "cuda" and isinstance(self.stream, torch.cuda.Stream):
             return torch.cuda.stream(self.stream)
         return contextlib.nullcontext()
+
+
+def common_prefix_blocks(tables: np.ndarray, lens: np.ndarray, block_size: int) -> int:
+    """Leading block-table entries that every row shares, counting only
+    blocks every sequence has filled (so none of them is written this step:
+    a sequence that writes into a shared block has been given its own copy)."""
+    n = len(lens)
+    if n < 2:
+        return 0
+    kmax = int(lens.min()) // block_size
+    if kmax == 0:
+        return 0
+    same = (tables[1:, :kmax] == tables[0, :kmax]).all(axis=0)
+    return int(kmax if same.all() else np.argmin(same))

@@ -125,3 +125,40 @@ def test_batch_limit(rec):
         cache.add_sequence(s, [s])
     with pytest.raises(ValueError):
         cache.begin_step([0, 1, 2], [0, 0, 0])
+
+
+def test_common_prefix_blocks():
+    from paged_kv_cache_410_b200.kv_cache import common_prefix_blocks
+    t = np.array([[5, 6, 7, 8, 9], [5, 6, 7, 1, 2], [5, 6, 7, 8, 3]], np.int32)
+    assert common_prefix_blocks(t, np.array([80, 80, 80]), 16) == 3
+    assert common_prefix_blocks(t, np.array([80, 40, 80]), 16) == 2   # only filled blocks count
+    assert common_prefix_blocks(t, np.array([80, 15, 80]), 16) == 0
+    assert common_prefix_blocks(t[:1], np.array([80]), 16) == 0          # one sequence: no sharing
+    assert common_prefix_blocks(t[[0, 2]], np.array([80, 80]), 16) == 4
+
+
+def test_shared_system_prompt_takes_the_shared_prefix_decode(rec):
+    cache = PagedKVCache(NB, BS, HKV, D, device="cpu", max_batch=8, max_blocks_per_seq=MB,
+                         stream=0, shared_prefix_min_blocks=3)
+    system = list(range(200, 214))                    # 3 full blocks + 2 tokens
+    for sid in range(4):
+        cache.add_sequence(sid, system + [sid, sid])
+    plan = cache.begin_step([0, 1, 2, 3], [1, 2, 3, 4])
+    assert plan.shared_prefix_blocks == 3
+    rec.calls.clear()
+    q = torch.zeros((4, HQ, D), dtype=torch.float16)
+    out = cache.attend(plan, 0, q, kv(4), kv(4))
+    names = [n for n, _ in rec.calls if n.startswith("pa_") and "size" not in n]
+    assert names == ["pa_append_kv", "pa_decode_shared_prefix"]
+    a = [c for c in rec.calls if c[0] == "pa_decode_shared_prefix"][0][1]
+    assert a[11] == 3 and a[0] == q.data_ptr() and a[13] == out.data_ptr()
+    # below the threshold, or with the path off: the fused launch
+    short = PagedKVCache(NB, BS, HKV, D, device="cpu", max_batch=8, max_blocks_per_seq=MB,
+                         stream=0, shared_prefix_min_blocks=0)
+    for sid in range(2):
+        short.add_sequence(sid, system)
+    plan = short.begin_step([0, 1], [1, 2])
+    rec.calls.clear()
+    short.attend(plan, 0, torch.zeros((2, HQ, D), dtype=torch.float16), kv(2), kv(2))
+    assert [n for n, _ in rec.calls if n in ("pa_append_decode", "pa_decode_shared_prefix")] == \
+        ["pa_append_decode"]
