@@ -100,6 +100,13 @@ int32_t pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id);
  * pa_decode_sliding_window never reads). */
 int32_t pa_bm_release_before(pa_block_manager* bm, int64_t seq_id, int32_t position);
 
+/* pa_bm_release_before(seq, length - window) for each of n sequences in one
+ * call: after a step of sliding-window decoding (window >= 1 tokens, the
+ * newest included), release the blocks that hold only tokens the window has
+ * left behind. PA_BM_ERR_INVALID (nothing released) for an unknown id. */
+int32_t pa_bm_release_window(pa_block_manager* bm, const int64_t* seq_ids, int32_t n,
+                             int32_t window);
+
 int32_t pa_bm_sequence_length(const pa_block_manager* bm, int64_t seq_id);
 
 /* Slots of positions [first, first + count) of a sequence. */

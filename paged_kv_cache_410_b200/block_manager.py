@@ -14,7 +14,7 @@ EXPORTED = ["pa_bm_create", "pa_bm_destroy", "pa_bm_num_free_blocks", "pa_bm_num
             "pa_bm_block_refcount", "pa_bm_add_sequence", "pa_bm_append_token", "pa_bm_fork",
             "pa_bm_free_sequence", "pa_bm_release_before", "pa_bm_sequence_length",
             "pa_bm_slots", "pa_bm_block_tables", "pa_bm_block_tables_update",
-            "pa_bm_append_tokens"]
+            "pa_bm_append_tokens", "pa_bm_release_window"]
 
 _declared = False
 
@@ -41,6 +41,8 @@ def _lib():
         lib.pa_bm_append_token.restype = i32
         lib.pa_bm_append_tokens.argtypes = [P, P, P, i32, P, P, ctypes.POINTER(i32)]
         lib.pa_bm_append_tokens.restype = i32
+        lib.pa_bm_release_window.argtypes = [P, P, i32, i32]
+        lib.pa_bm_release_window.restype = i32
         lib.pa_bm_fork.argtypes = [P, i64, i64]
         lib.pa_bm_fork.restype = i32
         lib.pa_bm_free_sequence.argtypes = [P, i64]
@@ -142,6 +144,12 @@ class BlockManager:
 
     def release_before(self, seq_id: int, position: int):
         _ok(self._lib.pa_bm_release_before(self._h, seq_id, position), "pa_bm_release_before")
+
+    def release_window(self, seq_ids, window: int):
+        """release_before(seq, length - window) for every listed sequence."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        _ok(self._lib.pa_bm_release_window(self._h, ids.ctypes.data, len(ids), window),
+            "pa_bm_release_window")
 
     def length(self, seq_id: int) -> int:
         n = self._lib.pa_bm_sequence_length(self._h, seq_id)

@@ -421,6 +421,24 @@ int32_t pa_bm_release_before(pa_block_manager* bm, int64_t seq_id, int32_t posit
   return PA_BM_OK;
 }
 
+int32_t pa_bm_release_window(pa_block_manager* bm, const int64_t* seq_ids, int32_t n,
+                             int32_t window) {
+  if (!bm || n < 0 || window < 1 || (n > 0 && !seq_ids)) return PA_BM_ERR_INVALID;
+  std::vector<Seq*> rows(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
+    rows[static_cast<size_t>(i)] = &it->second;
+  }
+  for (Seq* s : rows) {
+    // blocks holding only tokens before length - window
+    const int32_t upto = std::max(s->length - window, 0) / bm->bs;
+    for (int32_t k = s->released; k < upto; ++k) bm->unref(s->blocks[k]);
+    if (upto > s->released) s->released = upto;
+  }
+  return PA_BM_OK;
+}
+
 int32_t pa_bm_sequence_length(const pa_block_manager* bm, int64_t seq_id) {
   if (!bm) return PA_BM_ERR_INVALID;
   auto it = bm->seqs.find(seq_id);

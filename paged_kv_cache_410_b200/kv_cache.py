@@ -20,7 +20,9 @@ attended in the same kernel), or, when every sequence of the step starts
 with the same run of at least ``shared_prefix_min_blocks`` physical blocks
 (a system prompt served from the prefix cache), an append and
 ``pa_decode_shared_prefix``, which attends that prefix once for the whole
-batch. Prompts: ``add_sequence`` places a prompt,
+batch. With ``window`` > 0 every layer attends only each sequence's last
+``window`` tokens (``pa_decode_sliding_window``), and ``begin_step`` hands the
+blocks the window has left behind back to the pool. Prompts: ``add_sequence`` places a prompt,
 reusing cached prefix blocks, and returns the slots of the tokens whose K/V
 the caller still has to store (``store_prompt``).
 """
@@ -64,7 +66,11 @@ class PagedKVCache:
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
                  num_layers: int = 1, dtype=torch.float16, io_dtype=None, device="cuda",
                  prefix_cache: bool = True, max_batch: int = 256, max_blocks_per_seq: int = 512,
-                 k_scales=None, v_scales=None, stream=None, shared_prefix_min_blocks: int = 32):
+                 k_scales=None, v_scales=None, stream=None, shared_prefix_min_blocks: int = 32,
+                 window: int = 0):
+        if window < 0:
+            raise ValueError("window must be >= 0 (0: whole history)")
+        self.window = window
         self.device = torch.device(device)
         self.stream = stream
         self.shared_prefix_min_blocks = shared_prefix_min_blocks
@@ -158,8 +164,13 @@ class PagedKVCache:
             if self.device.type == "cuda":
                 self._uploaded = torch.cuda.Event()
                 self._uploaded.record()
+        if self.window:
+            # blocks holding only tokens before this step's window; their table
+            # entries stay (the window decode never reads them), and they are
+            # reused only by later steps, behind this step's kernels on the stream
+            self.bm.release_window(ids, self.window)
         shared = 0
-        if self.shared_prefix_min_blocks > 0:
+        if self.shared_prefix_min_blocks > 0 and not self.window:
             shared = common_prefix_blocks(self._h_tables.numpy()[:n], h_lens[:n],
                                           self.block_size)
         return StepPlan(n=n, slot_mapping=self._d_slots[:n], block_tables=self._d_tables[:n],
@@ -171,7 +182,8 @@ class PagedKVCache:
         """Store this layer's new K/V (k, v [n, Hkv, D]) at the plan's slots and
         return the decode output [n, Hq, D] for queries q [n, Hq, D]: one
         pa_append_decode launch, or pa_append_kv + pa_decode_shared_prefix
-        when the plan's shared prefix is long enough."""
+        when the plan's shared prefix is long enough, or pa_append_kv +
+        pa_decode_sliding_window with a window."""
         if out is None:
             out = torch.empty_like(q)
         if scale is None:
@@ -179,7 +191,10 @@ class PagedKVCache:
         cache = self.layers[layer]
         spb = plan.shared_prefix_blocks
         cascade = self.shared_prefix_min_blocks > 0 and spb >= self.shared_prefix_min_blocks
-        if cascade:
+        if self.window:
+            need = B.pa_decode_sliding_window_workspace_size(plan.n, q.shape[1],
+                                                             plan.max_context, self.window, cache)
+        elif cascade:
             need = B.pa_decode_shared_prefix_workspace_size(plan.n, q.shape[1], plan.max_context,
                                                             spb, cache)
         else:
@@ -188,7 +203,13 @@ class PagedKVCache:
             with self._on_stream():
                 self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
         ws = self._workspace if need else None
-        if cascade:
+        if self.window:
+            B.pa_append_kv(k, v, plan.slot_mapping, self.k[layer], self.v[layer], cache,
+                           self.stream)
+            B.pa_decode_sliding_window(q, self.k[layer], self.v[layer], plan.block_tables,
+                                       plan.context_lens, scale, out, cache, plan.max_context,
+                                       self.window, workspace=ws, stream=self.stream)
+        elif cascade:
             B.pa_append_kv(k, v, plan.slot_mapping, self.k[layer], self.v[layer], cache,
                            self.stream)
             B.pa_decode_shared_prefix(q, self.k[layer], self.v[layer], plan.block_tables,

@@ -497,3 +497,27 @@ def test_batched_appends_change_nothing_on_error():
     assert state[0] == after[0] and all((a == b).all() for a, b in zip(state[1], after[1]))
     assert before[0] == 2
     assert bm.append_tokens([], [])[0].shape == (0,)
+
+
+def test_release_window_equals_release_before_per_sequence():
+    a, b = BM.BlockManager(40, 4), BM.BlockManager(40, 4)
+    for bm in (a, b):
+        bm.add_sequence(1, range(18))                # 5 blocks
+        bm.add_sequence(2, range(7))                 # 2 blocks
+        bm.fork(1, 3)
+    a.release_window([1, 2, 3], 6)
+    for sid in (1, 2, 3):
+        b.release_before(sid, max(b.length(sid) - 6, 0))
+    assert a.num_free_blocks == b.num_free_blocks
+    assert [a.refcount(x) for x in range(40)] == [b.refcount(x) for x in range(40)]
+    free = a.num_free_blocks
+    a.release_window([2], 100)                       # nothing before the window: no change
+    assert a.num_free_blocks == free
+    with pytest.raises(BM.BlockManagerError):
+        a.release_window([1, 9], 6)                  # unknown id: nothing released
+    with pytest.raises(BM.BlockManagerError):
+        a.release_window([1], 0)
+    a.free_sequence(1)
+    a.free_sequence(3)                               # released blocks are not dropped twice
+    a.free_sequence(2)
+    assert a.num_free_blocks == 40

@@ -162,3 +162,28 @@ def test_shared_system_prompt_takes_the_shared_prefix_decode(rec):
     short.attend(plan, 0, torch.zeros((2, HQ, D), dtype=torch.float16), kv(2), kv(2))
     assert [n for n, _ in rec.calls if n in ("pa_append_decode", "pa_decode_shared_prefix")] == \
         ["pa_append_decode"]
+
+
+def test_sliding_window_releases_blocks_and_decodes_the_window(rec):
+    cache = PagedKVCache(NB, BS, HKV, D, device="cpu", max_batch=4, max_blocks_per_seq=MB,
+                         stream=0, window=6, prefix_cache=False)
+    for sid in range(2):
+        cache.add_sequence(sid, [sid] * 5)           # 2 blocks each
+    free0 = cache.bm.num_free_blocks
+    for step in range(12):
+        plan = cache.begin_step([0, 1], [step, step])
+        rec.calls.clear()
+        cache.attend(plan, 0, torch.zeros((2, HQ, D), dtype=torch.float16), kv(2), kv(2))
+        names = [n for n, _ in rec.calls if n in ("pa_append_kv", "pa_decode_sliding_window",
+                                                  "pa_append_decode", "pa_decode_shared_prefix")]
+        assert names == ["pa_append_kv", "pa_decode_sliding_window"]
+        a = [c for c in rec.calls if c[0] == "pa_decode_sliding_window"][0][1]
+        assert a[11] == 6                            # the window
+    # 17 tokens each: a window of 6 needs at most 3 blocks per sequence
+    L = cache.bm.length(0)
+    assert L == 17
+    held = 2 * (-(-L // BS) - (L - 6) // BS)
+    assert cache.bm.num_free_blocks == NB - held and held <= 6
+    assert free0 == NB - 4
+    with pytest.raises(ValueError):
+        PagedKVCache(NB, BS, HKV, D, device="cpu", window=-1, stream=0)
