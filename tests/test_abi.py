@@ -267,10 +267,13 @@ int main(void) {
   uint64_t versions[2] = {0, 0};
   rc |= pa_bm_append_tokens(bm, ids, btoks, 2, bslots, bpairs, &npairs);
   rc |= pa_bm_block_tables_update(bm, ids, 2, 4, kept, klens, versions, &written);
-  printf("%d|%s|%zu|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d\n", (int)pa_version(),
+  int64_t free_before = pa_bm_num_free_blocks(bm);
+  rc |= pa_bm_release_window(bm, ids, 2, 8); /* 41 and 42 tokens: blocks 0 and 1 go */
+  printf("%d|%s|%zu|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d|%d\n", (int)pa_version(),
          pa_status_string(PA_ERR_WORKSPACE), ws, (int)pt, (int)bad, rc, (int)cached, (int)src,
          (int)lens[0], (int)lens[1], tables[0] == tables[4] && tables[1] == tables[5],
-         (int)npairs, (int)written, (int)klens[0], (int)klens[1]);
+         (int)npairs, (int)written, (int)klens[0], (int)klens[1],
+         (int)(pa_bm_num_free_blocks(bm) - free_before));
   pa_bm_destroy(bm);
   return 0;
 }
@@ -306,6 +309,8 @@ def test_headers_are_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert int(f[11]) == 0                        # no shared partial block: no copies
     assert int(f[12]) == 2                        # first incremental export writes both rows
     assert (int(f[13]), int(f[14])) == (41, 42)
+    # the two shared prompt blocks stay held by the prefix cache: nothing freed
+    assert int(f[15]) == 0
 
 
 def test_workspace_sizes_cover_every_partition_plan(lib):
