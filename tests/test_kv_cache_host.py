@@ -1,9 +1,18 @@
-"""PagedKVCache (paged_kv_cache_410_b200/kv_cache.py) on the CPU: the step
-plans it uploads follow the host block manager exactly (slots, copy-on-write
-pairs, tables, lengths), copies reach every layer, and each layer's decode is
-one pa_append_decode call on the plan's tensors. The CUDA library is replaced
-by a recording stand-in (the block manager is the real C++ one), so no GPU
-and no kernel is involved."""
+"""PagedKVCache (paged_kv_cache_410_b200/kv_cache.py) on the CPU.
+
+With a recording stand-in for the CUDA library (the block manager is the
+real C++ one): the step plans it uploads follow the block manager exactly
+(slots, copy-on-write pairs, tables, lengths), copies reach every layer, and
+each layer's decode is the expected entry point on the plan's tensors.
+
+With the float64 oracle standing in for each entry point: a serving loop
+(two layers, prompts through the prefix cache, a beam fork, nine steps) in
+the fused, shared-prefix and sliding-window modes gives, for every sequence,
+layer and head, the attention computed straight from that sequence's logical
+history. No GPU and no kernel is involved: the kernels' own parity is the
+GPU tests' subject."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -187,3 +196,155 @@ def test_sliding_window_releases_blocks_and_decodes_the_window(rec):
     assert free0 == NB - 4
     with pytest.raises(ValueError):
         PagedKVCache(NB, BS, HKV, D, device="cpu", window=-1, stream=0)
+
+
+# ---- end to end on the CPU: the oracle stands in for the kernels ---------------
+
+class OracleLib:
+    """Test stand-in for libpagedattn.so: every entry point PagedKVCache calls
+    is carried out by the float64 oracle on the tensors behind the pointers,
+    so the cache class's slots, tables, lengths, copies and call order can be
+    checked against attention computed straight from each sequence's history.
+    (Test infrastructure only: the product never calls the oracle.)"""
+
+    def __init__(self, oracle):
+        self.o = oracle
+        self.t = {}
+        self.f64 = {}   # output address -> the oracle's float64 result
+
+    def reg(self, *ts):
+        for t in ts:
+            self.t[t.data_ptr()] = t
+
+    def bits(self, ptr, rows=None):
+        t = self.t[int(ptr)]
+        t = t if rows is None else t[:rows]
+        if t.dtype in (torch.float16, torch.bfloat16):
+            return t.view(torch.int16).numpy().view(np.uint16)
+        return t.numpy()
+
+    @staticmethod
+    def dt(code):
+        return {B.PA_F16: "f16", B.PA_BF16: "bf16", B.PA_E4M3: "e4m3"}[code]
+
+    def __getattr__(self, name):
+        if name.endswith("workspace_size"):
+            return lambda *a: 0
+        raise AttributeError(name)
+
+    def pa_append_kv(self, k, v, dtype, n, slots, kc, vc, desc, stream):
+        d = desc._obj
+        inv = [None if p is None else self.t[p].numpy() for p in (d.k_inv_scale, d.v_inv_scale)]
+        self.o.append_kv(self.bits(k, n), self.bits(v, n), self.dt(dtype), self.bits(slots, n),
+                         self.bits(kc), self.bits(vc), self.dt(d.cache_dtype), d.block_size, *inv)
+        return 0
+
+    def pa_copy_blocks_layers(self, pairs, n, kp, vp, layers, desc, stream):
+        arr = np.ctypeslib.as_array((ctypes.c_int32 * (2 * n)).from_address(pairs.value))
+        for l in range(layers):
+            self.o.copy_blocks(arr.reshape(-1, 2).copy(), self.bits(kp[l]), self.bits(vp[l]),
+                               self.dt(desc._obj.cache_dtype))
+        return 0
+
+    def _decode(self, q, qd, batch, hq, kc, vc, desc, bt, mb, lens, scale, out, window=0):
+        d = desc._obj
+        sc = [None if p is None else self.t[p].numpy() for p in (d.k_scale, d.v_scale)]
+        tables = self.t[int(bt)][:batch].numpy()
+        got = self.o.decode(self.bits(q, batch), self.dt(qd), self.bits(kc), self.bits(vc),
+                            self.dt(d.cache_dtype), tables, self.t[int(lens)][:batch].numpy(),
+                            scale, k_scale=sc[0], v_scale=sc[1], window=window)
+        self.t[int(out)][:batch] = torch.from_numpy(got).to(self.t[int(out)].dtype)
+        self.f64[int(out)] = got
+        return 0
+
+    def pa_append_decode(self, q, k, v, dt, batch, hq, slots, kc, vc, desc, bt, mb, lens, maxc,
+                         scale, out, pt, ws, wsb, stream):
+        self.pa_append_kv(k, v, dt, batch, slots, kc, vc, desc, stream)
+        return self._decode(q, dt, batch, hq, kc, vc, desc, bt, mb, lens, scale, out)
+
+    def pa_decode_shared_prefix(self, q, qd, batch, hq, kc, vc, desc, bt, mb, lens, maxc, pb,
+                                scale, out, pt, ws, wsb, stream):
+        tables = self.t[int(bt)][:batch].numpy()
+        assert (tables[:, :pb] == tables[0, :pb]).all()      # the call's precondition
+        assert (self.t[int(lens)][:batch].numpy() >= pb * desc._obj.block_size).all()
+        self.prefix_calls = getattr(self, "prefix_calls", 0) + 1
+        return self._decode(q, qd, batch, hq, kc, vc, desc, bt, mb, lens, scale, out)
+
+    def pa_decode_sliding_window(self, q, qd, batch, hq, kc, vc, desc, bt, mb, lens, maxc, w,
+                                 scale, out, pt, ws, wsb, stream):
+        return self._decode(q, qd, batch, hq, kc, vc, desc, bt, mb, lens, scale, out, window=w)
+
+
+def direct_attention(q, K, V, scale, window=0):
+    """softmax(scale q.K^T) V for one sequence and query head, from its
+    logical history (float64, no paging)."""
+    if window:
+        K, V = K[-window:], V[-window:]
+    s = scale * (K @ q)
+    w = np.exp(s - s.max())
+    return (w[:, None] * V).sum(0) / w.sum()
+
+
+@pytest.mark.parametrize("mode", ["fused", "shared_prefix", "window"])
+def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypatch, oracle_mod,
+                                                                       mode):
+    lib = OracleLib(oracle_mod)
+    monkeypatch.setattr(B, "load_library", lambda *a, **k: lib)
+    monkeypatch.setattr(B, "_on_device", lambda t: True)
+    rng = np.random.default_rng(5)
+    layers, hq, window = 2, 4, 7
+    cache = PagedKVCache(NB, BS, HKV, D, num_layers=layers, device="cpu", max_batch=8,
+                         max_blocks_per_seq=MB, stream=0,
+                         shared_prefix_min_blocks=2 if mode == "shared_prefix" else 0,
+                         window=window if mode == "window" else 0)
+    for l in range(layers):
+        lib.reg(cache.k[l], cache.v[l])
+    lib.reg(cache._d_slots, cache._d_tables, cache._d_lens)
+    half = lambda *shape: torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
+    hist = {}  # (seq, layer) -> (K [T, Hkv, D], V) float64, the logical history
+    system = list(range(300, 309))                     # 2 full blocks + 1 token
+    for sid in range(3):
+        cached, slots = cache.add_sequence(sid, system + [sid])
+        lib.reg(slots)
+        for l in range(layers):
+            if cached:                                 # the cached blocks hold sequence 0's K/V
+                K0, V0 = hist[(0, l)]
+                K, V = K0[:cached], V0[:cached]
+            else:
+                K = V = np.zeros((0, HKV, D))
+            n = 10 - cached
+            k, v = half(n, HKV, D), half(n, HKV, D)
+            lib.reg(k, v)
+            cache.store_prompt(l, slots, k, v)
+            hist[(sid, l)] = (np.concatenate([K, k.double().numpy()]),
+                              np.concatenate([V, v.double().numpy()]))
+        assert cached == (0 if sid == 0 else 8)
+    cache.fork(1, 3)                                   # beam: shares the partial block
+    for l in range(layers):
+        hist[(3, l)] = tuple(x.copy() for x in hist[(1, l)])
+    ids = [0, 1, 2, 3]
+    scale = 1 / np.sqrt(D)
+    for step in range(9):
+        plan = cache.begin_step(ids, [step] * 4)
+        for l in range(layers):
+            q, k, v = half(4, hq, D), half(4, HKV, D), half(4, HKV, D)
+            out = torch.empty((4, hq, D), dtype=torch.float16)
+            lib.reg(q, k, v, out)
+            cache.attend(plan, l, q, k, v, out=out)
+            got = lib.f64[out.data_ptr()]
+            for i, sid in enumerate(ids):
+                K, V = hist[(sid, l)]
+                K = np.concatenate([K, k[i:i + 1].double().numpy()])
+                V = np.concatenate([V, v[i:i + 1].double().numpy()])
+                hist[(sid, l)] = (K, V)
+                for h in range(hq):
+                    want = direct_attention(q[i, h].double().numpy(), K[:, h // (hq // HKV)],
+                                            V[:, h // (hq // HKV)], np.float32(scale),
+                                            window if mode == "window" else 0)
+                    np.testing.assert_allclose(got[i, h], want, rtol=0, atol=1e-9)
+    if mode == "shared_prefix":
+        assert lib.prefix_calls == 9 * layers
+    if mode == "window":
+        # sequences hold at most the 2 blocks their window spans; every other
+        # block is free or only in the prefix cache (reclaimable)
+        assert cache.bm.num_free_blocks + cache.bm.num_cached_blocks >= NB - 4 * 2
