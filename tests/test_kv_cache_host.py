@@ -285,7 +285,7 @@ def direct_attention(q, K, V, scale, window=0):
     return (w[:, None] * V).sum(0) / w.sum()
 
 
-@pytest.mark.parametrize("mode", ["fused", "shared_prefix", "window"])
+@pytest.mark.parametrize("mode", ["fused", "shared_prefix", "window", "e4m3"])
 def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypatch, oracle_mod,
                                                                        mode):
     lib = OracleLib(oracle_mod)
@@ -293,12 +293,34 @@ def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypa
     monkeypatch.setattr(B, "_on_device", lambda t: True)
     rng = np.random.default_rng(5)
     layers, hq, window = 2, 4, 7
+    e4m3 = mode == "e4m3"
+    ks = [torch.from_numpy(rng.uniform(0.005, 0.02, (HKV, D)).astype(np.float32))
+          for _ in range(layers)]
+    vs = [torch.from_numpy(rng.uniform(0.005, 0.02, (HKV, D)).astype(np.float32))
+          for _ in range(layers)]
     cache = PagedKVCache(NB, BS, HKV, D, num_layers=layers, device="cpu", max_batch=8,
                          max_blocks_per_seq=MB, stream=0,
                          shared_prefix_min_blocks=2 if mode == "shared_prefix" else 0,
-                         window=window if mode == "window" else 0)
+                         window=window if mode == "window" else 0,
+                         dtype=torch.uint8 if e4m3 else torch.float16,
+                         io_dtype=torch.float16, k_scales=ks if e4m3 else None,
+                         v_scales=vs if e4m3 else None)
     for l in range(layers):
         lib.reg(cache.k[l], cache.v[l])
+        if e4m3:
+            c = cache.layers[l]
+            lib.reg(c.k_scale, c.v_scale, c.k_inv_scale, c.v_inv_scale)
+
+    def stored(x, l, which):
+        """The values the cache holds for new K or V rows x of layer l."""
+        x = x.double().numpy()
+        if not e4m3:
+            return x
+        c = cache.layers[l]
+        scale = (c.k_scale if which == "k" else c.v_scale).numpy()
+        inv = (c.k_inv_scale if which == "k" else c.v_inv_scale).numpy()
+        codes = oracle_mod.e4m3_from_float((x.astype(np.float32) * inv).astype(np.float32))
+        return oracle_mod.e4m3_to_double(codes) * scale
     lib.reg(cache._d_slots, cache._d_tables, cache._d_lens)
     half = lambda *shape: torch.from_numpy(rng.standard_normal(shape).astype(np.float16))
     hist = {}  # (seq, layer) -> (K [T, Hkv, D], V) float64, the logical history
@@ -316,8 +338,8 @@ def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypa
             k, v = half(n, HKV, D), half(n, HKV, D)
             lib.reg(k, v)
             cache.store_prompt(l, slots, k, v)
-            hist[(sid, l)] = (np.concatenate([K, k.double().numpy()]),
-                              np.concatenate([V, v.double().numpy()]))
+            hist[(sid, l)] = (np.concatenate([K, stored(k, l, "k")]),
+                              np.concatenate([V, stored(v, l, "v")]))
         assert cached == (0 if sid == 0 else 8)
     cache.fork(1, 3)                                   # beam: shares the partial block
     for l in range(layers):
@@ -334,8 +356,8 @@ def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypa
             got = lib.f64[out.data_ptr()]
             for i, sid in enumerate(ids):
                 K, V = hist[(sid, l)]
-                K = np.concatenate([K, k[i:i + 1].double().numpy()])
-                V = np.concatenate([V, v[i:i + 1].double().numpy()])
+                K = np.concatenate([K, stored(k[i:i + 1], l, "k")])
+                V = np.concatenate([V, stored(v[i:i + 1], l, "v")])
                 hist[(sid, l)] = (K, V)
                 for h in range(hq):
                     want = direct_attention(q[i, h].double().numpy(), K[:, h // (hq // HKV)],
