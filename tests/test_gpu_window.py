@@ -1,6 +1,5 @@
 """GPU parity of pa_decode_sliding_window against the float64 oracle (which
 attends to tokens [max(0, L - window), L) by its own gather)."""
-import numpy as np
 import pytest
 import torch
 

@@ -6,7 +6,6 @@ and the bench's byte accounting against the same formula."""
 import json
 import os
 
-import numpy as np
 import pytest
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
