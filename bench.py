@@ -274,6 +274,8 @@ def parity_summary(got: np.ndarray, want: np.ndarray, io_dtype: str) -> dict:
 # ----------------------------------------------------------------- main ----
 
 def base_line(args, w, n_gpus):
+    elt = 1 if w.cache_dtype == "e4m3" else 2
+    pool_gb = 2 * w.num_blocks * w.block_size * w.num_kv_heads * w.head_dim * elt / 1e9
     return {"metric": METRIC, "unit": UNIT, "n_gpus": n_gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.cache_dtype, "data": "synthetic",
@@ -285,7 +287,7 @@ def base_line(args, w, n_gpus):
                        "kv_cache_dtype": w.cache_dtype, "io_dtype": w.io_dtype,
                        "parallelism": f"independent batch per GPU x{n_gpus}",
                        "l2": "not flushed: the step reads more than the 126 MB L2 "
-                             f"(pool {2 * w.num_blocks * w.block_size * w.num_kv_heads * w.head_dim * (1 if w.cache_dtype == 'e4m3' else 2) / 1e9:.2f} GB)"}}
+                             f"(pool {pool_gb:.2f} GB)"}}
 
 
 def run_reference(args):
@@ -504,7 +506,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama2_7b")
-    ap.add_argument("--batch", type=int, default=None, help="sequences per GPU (default: the family's)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the family's)")
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -21,14 +21,24 @@ with the same run of at least ``shared_prefix_min_blocks`` physical blocks
 (a system prompt served from the prefix cache), an append and
 ``pa_decode_shared_prefix``, which attends that prefix once for the whole
 batch. With ``window`` > 0 every layer attends only each sequence's last
-``window`` tokens (``pa_decode_sliding_window``), and ``begin_step`` hands the
-blocks the window has left behind back to the pool. Prompts: ``add_sequence`` places a prompt,
-reusing cached prefix blocks, and returns the slots of the tokens whose K/V
-the caller still has to store (``store_prompt``).
+``window`` tokens (``pa_decode_sliding_window``), and ``begin_step`` hands
+the blocks the window has left behind back to the pool.
+
+Prompts: ``add_sequence`` places a prompt, reusing cached prefix blocks, and
+returns the slots of the tokens whose K/V the caller still has to store
+(``store_prompt``).
+
+Several GPUs (tensor parallelism over KV heads): every rank builds a cache
+for its own heads and drives its own block manager with the same calls, so
+all ranks place every token in the same slots and no exchange is needed.
+Given a process group (``lockstep_group``), ``begin_step`` checks that: it
+all-gathers a 64-bit digest of the step's slots, copy pairs and lengths and
+raises on every rank if any rank's differs.
 """
 from __future__ import annotations
 
 import contextlib
+import hashlib
 import math
 from dataclasses import dataclass
 
@@ -67,10 +77,11 @@ class PagedKVCache:
                  num_layers: int = 1, dtype=torch.float16, io_dtype=None, device="cuda",
                  prefix_cache: bool = True, max_batch: int = 256, max_blocks_per_seq: int = 512,
                  k_scales=None, v_scales=None, stream=None, shared_prefix_min_blocks: int = 32,
-                 window: int = 0):
+                 window: int = 0, lockstep_group=None):
         if window < 0:
             raise ValueError("window must be >= 0 (0: whole history)")
         self.window = window
+        self.lockstep_group = lockstep_group
         self.device = torch.device(device)
         self.stream = stream
         self.shared_prefix_min_blocks = shared_prefix_min_blocks
@@ -169,6 +180,8 @@ class PagedKVCache:
             # entries stay (the window decode never reads them), and they are
             # reused only by later steps, behind this step's kernels on the stream
             self.bm.release_window(ids, self.window)
+        if self.lockstep_group is not None:
+            self._check_lockstep(slots, pairs, h_lens[:n])
         shared = 0
         if self.shared_prefix_min_blocks > 0 and not self.window:
             shared = common_prefix_blocks(self._h_tables.numpy()[:n], h_lens[:n],
@@ -220,6 +233,20 @@ class PagedKVCache:
                                plan.block_tables, plan.context_lens, scale, out, cache,
                                plan.max_context, workspace=ws, stream=self.stream)
         return out
+
+    def _check_lockstep(self, slots, pairs, lens):
+        import torch.distributed as dist
+        h = hashlib.blake2b(digest_size=8)
+        for a in (slots, pairs, lens):
+            h.update(np.ascontiguousarray(a).tobytes())
+        mine = int.from_bytes(h.digest(), "little", signed=True)
+        dev = self.device if dist.get_backend(self.lockstep_group) == "nccl" else "cpu"
+        t = torch.tensor([mine], dtype=torch.int64, device=dev)
+        every = [torch.empty_like(t) for _ in range(dist.get_world_size(self.lockstep_group))]
+        dist.all_gather(every, t, group=self.lockstep_group)
+        if any(int(x.item()) != mine for x in every):
+            raise RuntimeError("block managers out of lockstep: the ranks placed this step's "
+                               "tokens differently")
 
     def _on_stream(self):
         if self.device.type == "cuda" and isinstance(self.stream, torch.cuda.Stream):

@@ -27,7 +27,8 @@ def _built():
 
 
 def test_header_symbols_are_exported():
-    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "pa_block_manager.h")).read(),
+    header = open(os.path.join(ROOT, "include", "pa_block_manager.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", header,
                   flags=re.S)
     names = sorted(set(re.findall(r"\b(pa_bm_[a-z_]+)\s*\(", text)))
     assert names == sorted(BM.EXPORTED)

@@ -370,3 +370,49 @@ def test_serving_loop_on_the_oracle_matches_attention_over_each_history(monkeypa
         # sequences hold at most the 2 blocks their window spans; every other
         # block is free or only in the prefix cache (reclaimable)
         assert cache.bm.num_free_blocks + cache.bm.num_cached_blocks >= NB - 4 * 2
+
+
+def _lockstep_worker(rank, world, port, diverge, q):
+    import os
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = Recorder()
+        B.load_library = lambda *a, **k: r       # this process only
+        B._on_device = lambda t: True
+        cache = PagedKVCache(NB, BS, HKV // world, D, device="cpu", max_batch=4,
+                             max_blocks_per_seq=MB, stream=0, lockstep_group=dist.group.WORLD)
+        for sid in range(3):
+            prompt = [sid] * (5 + (rank if diverge and sid == 2 else 0))
+            cache.add_sequence(sid, prompt)
+        outcome = "ok"
+        try:
+            for step in range(3):
+                cache.begin_step([0, 1, 2], [step] * 3)
+        except RuntimeError as e:
+            outcome = "lockstep" if "lockstep" in str(e) else repr(e)
+        q.put((rank, outcome))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("diverge", [False, True])
+def test_lockstep_check_over_two_ranks(diverge):
+    """Each rank drives its own block manager; the per-step digest exchange
+    passes when they agree and fails on every rank when one placed a prompt
+    differently."""
+    import os
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29700 + os.getpid() % 200 + (100 if diverge else 0)
+    procs = [ctx.Process(target=_lockstep_worker, args=(r, 2, port, diverge, q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o for _, o in res] == (["lockstep", "lockstep"] if diverge else ["ok", "ok"])

@@ -51,7 +51,8 @@ MUTANTS = [
      "int64_t dst = ((blk * block_size + r) * num_kv_heads + h) * head_dim + (head_dim - 1 - c);"),
     ("append_quantises_without_scale", "float yk = xk * k_inv_scale[h * head_dim + c];",
      "float yk = xk;"),
-    ("copy_skips_v", "(const char*)v_cache + s * block_bytes", "(const char*)v_cache + d * block_bytes"),
+    ("copy_skips_v", "(const char*)v_cache + s * block_bytes",
+     "(const char*)v_cache + d * block_bytes"),
     ("kv_formula_one_factor_short", "return 2 * layers * kv_heads", "return layers * kv_heads"),
 ]
 
