@@ -8,6 +8,7 @@ reference-counted, and branches copy a block only where they diverge (KV cache
 article, section 'PagedAttention：把操作系统的老智慧搬进推理引擎'); a radix tree
 of token ids lets later requests reuse a cached prefix (chapter '第2章 KV
 Cache：模型内部的显存复用')."""
+import ctypes
 import functools
 import re
 import os
@@ -522,3 +523,30 @@ def test_release_window_equals_release_before_per_sequence():
     a.free_sequence(3)                               # released blocks are not dropped twice
     a.free_sequence(2)
     assert a.num_free_blocks == 40
+
+
+def test_null_arguments_are_rejected_not_dereferenced():
+    """Every entry point of the C ABI answers a NULL manager or a NULL array
+    (where one is needed) with PA_BM_ERR_INVALID (or -1 / NULL), never a crash."""
+    lib = BM._lib()
+    bm = BM.BlockManager(8, 4)
+    bm.add_sequence(1, [1, 2, 3])
+    h = bm._h
+    I = BM.ERR_INVALID
+    assert lib.pa_bm_create(0, 4, 0) is None and lib.pa_bm_create(8, 0, 0) is None
+    assert lib.pa_bm_num_free_blocks(None) == -1 and lib.pa_bm_num_cached_blocks(None) == -1
+    assert lib.pa_bm_block_refcount(None, 0) == -1 and lib.pa_bm_block_refcount(h, 8) == -1
+    assert lib.pa_bm_add_sequence(None, 2, None, 0, None) == I
+    assert lib.pa_bm_add_sequence(h, 2, None, 3, None) == I          # tokens missing
+    assert lib.pa_bm_append_token(h, 1, 0, None, None, None) == I    # slot output missing
+    n = ctypes.c_int32(0)
+    assert lib.pa_bm_append_tokens(h, None, None, 2, None, None, ctypes.byref(n)) == I
+    assert lib.pa_bm_append_tokens(h, None, None, 0, None, None, None) == I  # count output missing
+    assert lib.pa_bm_release_window(h, None, 1, 4) == I
+    assert lib.pa_bm_fork(None, 1, 2) == I and lib.pa_bm_free_sequence(None, 1) == I
+    assert lib.pa_bm_release_before(None, 1, 0) == I and lib.pa_bm_sequence_length(None, 1) == I
+    assert lib.pa_bm_slots(h, 1, 0, 2, None) == I
+    assert lib.pa_bm_block_tables(h, None, 1, 4, None, None) == I
+    assert lib.pa_bm_block_tables_update(h, None, 1, 4, None, None, None, None) == I
+    lib.pa_bm_destroy(None)                                           # a no-op
+    assert bm.length(1) == 3                                          # the manager is intact
