@@ -500,17 +500,26 @@ def run_ours(args):
 
 
 def main(argv=None):
-    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama2_7b")
+    ap = argparse.ArgumentParser(
+        description="Time one decode step of one attention layer (block copies, KV append, "
+                    "paged decode) and print one JSON line.")
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one process each, torchrun)")
+    ap.add_argument("--steps", type=int, default=2000, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=20, help="untimed steps first (>= 3)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="the CUDA library, or the float64 CPU oracle")
+    ap.add_argument("--workload", default="llama2_7b",
+                    choices=["tiny_mha", "llama2_7b", "llama2_70b_prefix", "long_context",
+                             "fp8_beams"],
+                    help="input family (its shapes and seed)")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the family's)")
-    ap.add_argument("--partition-tokens", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--partition-tokens", type=int, default=0,
+                    help="split-K partition length (0: the library's choice)")
+    ap.add_argument("--e2e-steps", type=int, default=200,
+                    help="steps of the end-to-end measurement (host copies included)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle baseline and its parity check")
     ap.add_argument("--window", type=int, default=0,
                     help="sliding-window decode over the last WINDOW tokens (0: whole history)")
     ap.add_argument("--fused", action="store_true",
