@@ -92,6 +92,9 @@ def make_workload(name: str, rank: int, batch: int | None):
     params = inspect.signature(fam).parameters
     if batch is not None:
         kw["batch"] = batch
+        if "beam_groups" in params:  # as many 4-beam groups as the batch holds, up to 16
+            kw["beam_groups"] = min(params["beam_groups"].default,
+                                    batch // params["beam_width"].default)
     seed = params["seed"].default
     if seed is None:  # fp8 family derives its seed from the block size
         seed = W.SEED_BASE + 5 + params["block_size"].default

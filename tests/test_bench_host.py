@@ -116,3 +116,15 @@ def test_parity_summary_against_the_oracle_sample():
     nan[0, 0, 0] = np.nan
     r = bench.parity_summary(nan, want, "f16")
     assert r["max_abs_err"] is None and not r["ok"]
+
+
+def test_small_fp8_batches_scale_the_beam_groups():
+    from paged_kv_cache_410_b200 import workloads as W
+    orig = W.normal_bits
+    W.normal_bits = lambda rng, shape, dtype, chunk=0: np.zeros(shape, np.uint16)
+    try:
+        w = bench.make_workload("fp8_beams", 0, 24)
+        assert w.batch == 24 and w.meta["beam_groups"] == 6
+        assert bench.make_workload("fp8_beams", 0, 256).meta["beam_groups"] == 16
+    finally:
+        W.normal_bits = orig
