@@ -81,7 +81,10 @@ int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, 
  * to cow_pairs ([n][2] int32 (src, dst), room for n pairs) and their count to
  * *num_pairs; apply them (pa_copy_blocks) before appending K/V. A sequence
  * that copies drops its share of the old block, so a later sequence of the
- * batch that shared it with that one alone writes in place. Returns
+ * batch that shared it with that one alone writes in place. The batch's
+ * blocks are all taken before any of its tokens joins the prefix cache, so
+ * when the pool must evict cached blocks the choice can differ from n
+ * separate pa_bm_append_token calls (both placements are valid). Returns
  * PA_BM_ERR_INVALID for an unknown or repeated id and PA_BM_ERR_NO_BLOCKS if
  * the pool (after evicting cached blocks) cannot supply the batch; either
  * way nothing has changed. */

@@ -159,14 +159,13 @@ struct pa_block_manager {
     if (it != nodes.end()) track(it->second.get());
   }
 
-  // Appends one token to `s`: a new block at a block boundary, a private
-  // copy of a shared partial last block (copy on write), else the next row of
-  // the last block. Fails (changing nothing) only if a block is needed and
-  // none can be had.
-  int32_t append_one(Seq& s, int32_t token, int64_t* slot, int32_t* cow_src, int32_t* cow_dst) {
-    const int32_t pos = s.length;
-    int32_t src = -1, dst = -1;
-    if (pos % bs == 0) {
+  // The block the next token of `s` goes to: a new block at a block
+  // boundary, a private copy of a shared partial last block (copy on write:
+  // *cow_src / *cow_dst receive the pair), else the last block as it is.
+  // Fails (changing nothing) only if a block is needed and none can be had.
+  int32_t take_block(Seq& s, int32_t* cow_src, int32_t* cow_dst) {
+    *cow_src = *cow_dst = -1;
+    if (s.length % bs == 0) {
       const int64_t b = alloc();
       if (b < 0) return PA_BM_ERR_NO_BLOCKS;
       s.blocks.push_back(b);
@@ -176,20 +175,24 @@ struct pa_block_manager {
       if (refcount[last] > 1) {  // shared partial block: copy on write
         const int64_t b = alloc();
         if (b < 0) return PA_BM_ERR_NO_BLOCKS;
-        src = static_cast<int32_t>(last);
-        dst = static_cast<int32_t>(b);
+        *cow_src = static_cast<int32_t>(last);
+        *cow_dst = static_cast<int32_t>(b);
         unref(last);
         s.blocks.back() = b;
         changed(s);
       }
     }
+    return PA_BM_OK;
+  }
+
+  // Records the token taken by take_block: its slot, its id, and the block
+  // it fills joins the prefix cache.
+  void commit_token(Seq& s, int32_t token, int64_t* slot) {
+    const int32_t pos = s.length;
     *slot = s.blocks[pos / bs] * bs + pos % bs;
-    *cow_src = src;
-    *cow_dst = dst;
     s.tokens.push_back(token);
     s.length = pos + 1;
     if (s.length % bs == 0) cache_full_block(s, s.length / bs - 1);
-    return PA_BM_OK;
   }
 
   // Blocks that one append to each of `rows` (distinct sequences, in this
@@ -349,8 +352,9 @@ int32_t pa_bm_append_token(pa_block_manager* bm, int64_t seq_id, int32_t token, 
   auto it = bm->seqs.find(seq_id);
   if (it == bm->seqs.end()) return PA_BM_ERR_INVALID;
   int32_t src = -1, dst = -1;
-  const int32_t rc = bm->append_one(it->second, token, slot, &src, &dst);
+  const int32_t rc = bm->take_block(it->second, &src, &dst);
   if (rc != PA_BM_OK) return rc;
+  bm->commit_token(it->second, token, slot);
   if (cow_src) *cow_src = src;
   if (cow_dst) *cow_dst = dst;
   return PA_BM_OK;
@@ -371,11 +375,14 @@ int32_t pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, const 
     rows[static_cast<size_t>(i)] = &it->second;
   }
   if (!bm->can_reclaim(bm->blocks_for_appends(rows))) return PA_BM_ERR_NO_BLOCKS;
+  // First every row's block, then the tokens: caching a block a row fills
+  // can pin a released block that only the cache held (it becomes a parent),
+  // which the count above took as reclaimable, so no row may fill the cache
+  // before every block of the batch is taken.
   int32_t pairs = 0;
   for (int32_t i = 0; i < n; ++i) {
     int32_t src = -1, dst = -1;
-    if (bm->append_one(*rows[static_cast<size_t>(i)], tokens[i], &slots[i], &src, &dst) !=
-        PA_BM_OK)
+    if (bm->take_block(*rows[static_cast<size_t>(i)], &src, &dst) != PA_BM_OK)
       return PA_BM_ERR_NO_BLOCKS;  // not reached: the blocks were counted above
     if (src >= 0) {
       cow_pairs[2 * pairs] = src;
@@ -383,6 +390,8 @@ int32_t pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, const 
       ++pairs;
     }
   }
+  for (int32_t i = 0; i < n; ++i)
+    bm->commit_token(*rows[static_cast<size_t>(i)], tokens[i], &slots[i]);
   *num_pairs = pairs;
   return PA_BM_OK;
 }

@@ -428,7 +428,9 @@ def _random_serving(seed):
     return dict(seqs=next_id, hits=hits, copies=copies, failures=failures)
 
 
-@pytest.mark.parametrize("seed", range(8))
+# seeds 190.. once made a batched append fail part-way: a row filling a block
+# pinned a released block only the cache held, which the batch had counted
+@pytest.mark.parametrize("seed", list(range(8)) + [190, 236, 246, 272, 328])
 def test_random_serving_keeps_every_sequence_cache_intact(seed):
     _random_serving(seed)
 
