@@ -418,3 +418,94 @@ def test_lockstep_check_over_two_ranks(diverge):
         p.join(timeout=60)
         assert p.exitcode == 0
     assert [o for _, o in res] == (["lockstep", "lockstep"] if diverge else ["ok", "ok"])
+
+
+def _random_loop(oracle_mod, monkeypatch, seed):
+    """One randomized serving loop through PagedKVCache on the oracle stand-in:
+    random shapes, block size and mode; admissions (some served entirely from
+    the prefix cache), forks and frees between steps. The expected history of
+    a sequence's cached prefix is what was last stored in its slots (a model of
+    every slot's contents: prompt stores, copies, appends)."""
+    rng = np.random.default_rng(seed)
+    lib = OracleLib(oracle_mod)
+    monkeypatch.setattr(B, "load_library", lambda *a, **k: lib)
+    monkeypatch.setattr(B, "_on_device", lambda t: True)
+    bs, hkv, d = int(rng.choice([1, 4, 16])), int(rng.choice([1, 2])), 64
+    hq, layers = hkv * int(rng.choice([1, 2, 4])), int(rng.integers(1, 3))
+    mode = ["fused", "prefix", "window"][seed % 3]
+    window = int(rng.integers(1, 30)) if mode == "window" else 0
+    cache = PagedKVCache(400, bs, hkv, d, num_layers=layers, device="cpu", max_batch=8,
+                         max_blocks_per_seq=256, stream=0, window=window,
+                         shared_prefix_min_blocks=int(rng.integers(1, 3)) if mode == "prefix"
+                         else 0)
+    for l in range(layers):
+        lib.reg(cache.k[l], cache.v[l])
+    lib.reg(cache._d_slots, cache._d_tables, cache._d_lens)
+    half = lambda *s: torch.from_numpy(rng.standard_normal(s).astype(np.float16))
+    hist, content, live, nxt = {}, {}, [], 0
+    system = [int(x) for x in rng.integers(0, 4, size=int(rng.integers(0, 3 * bs + 2)))]
+
+    def admit():
+        nonlocal nxt
+        toks = system + [int(x) for x in rng.integers(0, 4, size=int(rng.integers(1, 2 * bs + 3)))]
+        cached, slots = cache.add_sequence(nxt, toks)
+        lib.reg(slots)
+        pre = cache.bm.slots(nxt, 0, cached) if cached else []
+        for l in range(layers):
+            K0 = np.array([content[(l, int(x))][0] for x in pre]).reshape(-1, hkv, d)
+            V0 = np.array([content[(l, int(x))][1] for x in pre]).reshape(-1, hkv, d)
+            k, v = half(len(toks) - cached, hkv, d), half(len(toks) - cached, hkv, d)
+            lib.reg(k, v)
+            cache.store_prompt(l, slots, k, v)
+            for j, x in enumerate(slots.tolist()):
+                content[(l, x)] = (k[j].double().numpy(), v[j].double().numpy())
+            hist[(nxt, l)] = (np.concatenate([K0, k.double().numpy()]),
+                              np.concatenate([V0, v.double().numpy()]))
+        live.append(nxt)
+        nxt += 1
+
+    for _ in range(int(rng.integers(2, 5))):
+        admit()
+    for step in range(10):
+        r = rng.random()
+        if r < 0.15 and len(live) < 7:
+            admit()
+        elif r < 0.3 and len(live) < 7:
+            p = live[int(rng.integers(0, len(live)))]
+            cache.fork(p, nxt)
+            for l in range(layers):
+                hist[(nxt, l)] = tuple(x.copy() for x in hist[(p, l)])
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.4 and len(live) > 2:
+            cache.free_sequence(live.pop(int(rng.integers(0, len(live)))))
+        ids = [int(x) for x in rng.permutation(live)]
+        plan = cache.begin_step(ids, [int(x) for x in rng.integers(0, 4, size=len(ids))])
+        for l in range(layers):
+            for src, dst in plan.copy_pairs.tolist():
+                for row in range(bs):
+                    if (l, src * bs + row) in content:
+                        content[(l, dst * bs + row)] = content[(l, src * bs + row)]
+            n = len(ids)
+            q, k, v = half(n, hq, d), half(n, hkv, d), half(n, hkv, d)
+            out = torch.empty((n, hq, d), dtype=torch.float16)
+            lib.reg(q, k, v, out)
+            cache.attend(plan, l, q, k, v, out=out)
+            got = lib.f64[out.data_ptr()]
+            for i, x in enumerate(plan.slot_mapping.tolist()):
+                content[(l, x)] = (k[i].double().numpy(), v[i].double().numpy())
+            for i, sid in enumerate(ids):
+                K = np.concatenate([hist[(sid, l)][0], k[i:i + 1].double().numpy()])
+                V = np.concatenate([hist[(sid, l)][1], v[i:i + 1].double().numpy()])
+                hist[(sid, l)] = (K, V)
+                for h in range(hq):
+                    want = direct_attention(q[i, h].double().numpy(), K[:, h // (hq // hkv)],
+                                            V[:, h // (hq // hkv)], np.float32(1 / np.sqrt(d)),
+                                            window)
+                    np.testing.assert_allclose(got[i, h], want, rtol=0, atol=1e-9,
+                                               err_msg=f"seed {seed} step {step} layer {l}")
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_serving_loops_match_attention_over_each_history(oracle_mod, monkeypatch, seed):
+    _random_loop(oracle_mod, monkeypatch, seed)
