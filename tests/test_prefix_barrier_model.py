@@ -36,9 +36,11 @@ class Violation(Exception):
     pass
 
 
-def check(nsteps, fault=None):
+def check(nsteps, fault=None, nstage=NSTAGE):
     """Explore every interleaving; returns the number of states, raises
-    Violation (with a reason) on a hazard, a wrapped parity or a deadlock."""
+    Violation (with a reason) on a hazard, a wrapped parity or a deadlock.
+    `nstage`: K/V stages (the kernel's build-time stage count)."""
+    NSTAGE = nstage  # noqa: N806 (shadows the module default inside the model)
 
     def wait(st, name, k, what):
         c = st["bar"][name]
@@ -129,9 +131,9 @@ def check(nsteps, fault=None):
 
     start = {"prod": 0, "prod_v": False, "mma": ("start", 0), "smx": ("wait_s", 0),
              "pending": (), "s_reading": None, "p_unread": None,
-             "bar": {b: 0 for b in ("kfull0", "kfull1", "vfull0", "vfull1", "kfree0", "kfree1",
-                                    "vfree0", "vfree1", "sfull0", "sfull1", "sfree0", "sfree1",
-                                    "pfull", "pv")}}
+             "bar": {b: 0 for b in [f"{x}{i}" for x in ("kfull", "vfull", "kfree", "vfree")
+                                    for i in range(NSTAGE)] +
+                     ["sfull0", "sfull1", "sfree0", "sfree1", "pfull", "pv"]}}
     seen, q = {freeze(start)}, deque([start])
     while q:
         st = q.popleft()
@@ -148,9 +150,10 @@ def check(nsteps, fault=None):
     return len(seen)
 
 
+@pytest.mark.parametrize("nstage", [1, 2, 3, 4])
 @pytest.mark.parametrize("nsteps", [1, 2, 3, 4, 6, 8])
-def test_the_kernels_protocol_has_no_hazard_wrap_or_deadlock(nsteps):
-    assert check(nsteps) > 0
+def test_the_kernels_protocol_has_no_hazard_wrap_or_deadlock(nsteps, nstage):
+    assert check(nsteps, nstage=nstage) > 0
 
 
 @pytest.mark.parametrize("fault,reason", [
