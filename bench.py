@@ -13,6 +13,14 @@ the step's inputs copied from pinned host memory and the output read back
 inside the timed region; `cpu_baseline` times the float64 CPU oracle on the
 host's cores on the same inputs.
 
+L2 is flushed between timed steps (a 256 MiB buffer, twice the L2, is
+written outside the timed events), so every step reads its KV cache from
+HBM; the line also carries the same measurement without the flush
+(`unflushed`). At one GPU the line adds `other_configs`: the 70B-shaped
+shared-prefix layer, the 128K-token long context at batch 1 and 4 and the
+FP8 cache with beam forks, each timed the same way in the same run, with its
+decode roofline, clocks and a check of sampled outputs against the oracle.
+
 Multi-GPU (torchrun): every rank runs its own independent batch of the same
 shape (sequences are independent; no data-path collective), so per-GPU work
 is fixed ("weak" scaling); the step time is the max over ranks.
@@ -43,6 +51,10 @@ if ROOT not in sys.path:
 METRIC = "paged-decode KV GB/s and % of B200 HBM peak; decode attn tokens/s per layer"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20  # written between timed steps: twice the 126 MB L2
+# measured beside the headline at one GPU: (family, batch; None = the family's)
+OTHER_CONFIGS = [("llama2_70b_prefix", None), ("long_context", 1), ("long_context", 4),
+                 ("fp8_beams", None)]
 SPEC_HBM_GBS = 8000.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "pa_decode_llama2_7b.md")
 # the sources of the plain decode's kernels (main + split-K merge): the
@@ -262,7 +274,8 @@ def cpu_baseline(w, target_s=12.0, window=0):
 TOLERANCE = {"f16": 2e-3, "bf16": 1e-2}
 
 
-def parity_summary(got: np.ndarray, want: np.ndarray, io_dtype: str) -> dict:
+def parity_summary(got: np.ndarray, want: np.ndarray, io_dtype: str,
+                   against: str = "float64 CPU oracle, same inputs, the cpu_baseline sample") -> dict:
     """Max-abs error of the GPU output (float64 [n, Hq, D]) against the
     oracle's for the same sequences."""
     diff = np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64))
@@ -271,14 +284,48 @@ def parity_summary(got: np.ndarray, want: np.ndarray, io_dtype: str) -> dict:
     tol = TOLERANCE[io_dtype]
     return {"max_abs_err": err if finite else None, "tolerance": tol,
             "sequences": int(got.shape[0]), "ok": bool(finite and err <= tol),
-            "against": "float64 CPU oracle, same inputs, the cpu_baseline sample"}
+            "against": against}
+
+
+def parity_sample(w, n: int) -> np.ndarray:
+    """Up to n sequences for a bench-side check: the shortest and the longest,
+    the first beam group when the batch has one, then evenly spaced ones."""
+    if n >= w.batch:
+        return np.arange(w.batch)
+    must = {int(np.argmin(w.context_lens)), int(np.argmax(w.context_lens))}
+    if "beam_groups" in w.meta:
+        must |= {0, 1, 2, 3}
+    rest = [int(i) for i in np.linspace(0, w.batch - 1, n) if int(i) not in must]
+    return np.array(sorted(must | set(rest[:max(0, n - len(must))])))
 
 
 # ----------------------------------------------------------------- main ----
 
-def base_line(args, w, n_gpus):
+def cascade_blocks(args, w) -> int:
+    """Shared-prefix blocks the step decodes through the cascade (0: none)."""
+    if args.cascade != "auto" or args.window or args.fused:
+        return 0
+    return int(w.meta.get("shared_prefix_blocks", 0))
+
+
+def decode_label(args, spb: int) -> str:
+    return ("append fused into decode" if args.fused else
+            f"sliding window {args.window}" if args.window else
+            f"shared-prefix cascade ({spb} blocks)" if spb else
+            "whole history")
+
+
+def l2_note(flushed: bool, w) -> str:
     elt = 1 if w.cache_dtype == "e4m3" else 2
     pool_gb = 2 * w.num_blocks * w.block_size * w.num_kv_heads * w.head_dim * elt / 1e9
+    if flushed:
+        return (f"flushed: a {L2_FLUSH_BYTES >> 20} MiB buffer (twice the L2) is written between "
+                "timed steps, outside the timed events; step time = sum of the per-step "
+                f"event intervals (pool {pool_gb:.2f} GB)")
+    return f"not flushed: steps back to back (pool {pool_gb:.2f} GB)"
+
+
+def base_line(args, w, n_gpus, spb=0):
     return {"metric": METRIC, "unit": UNIT, "n_gpus": n_gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.cache_dtype, "data": "synthetic",
@@ -289,8 +336,8 @@ def base_line(args, w, n_gpus):
                                        f" (mean {float(w.context_lens.mean()):.0f})",
                        "kv_cache_dtype": w.cache_dtype, "io_dtype": w.io_dtype,
                        "parallelism": f"independent batch per GPU x{n_gpus}",
-                       "l2": "not flushed: the step reads more than the 126 MB L2 "
-                             f"(pool {pool_gb:.2f} GB)"}}
+                       "l2": l2_note(not args.no_flush, w),
+                       "decode": decode_label(args, spb)}}
 
 
 def run_reference(args):
@@ -303,20 +350,22 @@ def run_reference(args):
     oracle.build()
     # per-step sample sized so warmup + steps fit in about two minutes
     budget = min(10.0, 120.0 / max(1, args.steps + args.warmup))
-    t1, _, _ = oracle_step_time(w, np.arange(1))
+    t1, _, _ = oracle_step_time(w, np.arange(1), window=args.window)
     n = int(min(w.batch, max(1, budget / max(t1, 1e-4))))
     seqs = np.arange(n)
     for _ in range(args.warmup):
-        oracle_step_time(w, seqs)
+        oracle_step_time(w, seqs, window=args.window)
     times = []
     s = None
     for _ in range(args.steps):
-        t, s, _ = oracle_step_time(w, seqs)
+        t, s, _ = oracle_step_time(w, seqs, window=args.window)
         times.append(t)
     total = sum(times)
-    nbytes = A.step_bytes(s)["total"] * args.steps
+    nbytes = A.step_bytes(s, window=args.window)["total"] * args.steps
     value = nbytes / total / 1e9
-    line = base_line(args, w, world)
+    # the same config object as the GPU arm's line for the same flags (the
+    # oracle has no cascade or fused form: it computes the same result)
+    line = base_line(args, w, world, cascade_blocks(args, w))
     line["dtype"] = "f64"
     line.update({"impl": "reference", "value": value, "ms_per_step": 1e3 * total / args.steps,
                  "tokens_per_s_per_layer": n * args.steps / total,
@@ -331,6 +380,136 @@ def run_reference(args):
     return 0
 
 
+def make_step(args, w, dev, spb):
+    from paged_kv_cache_410_b200.session import DecodeStep
+    return DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb,
+                      window=args.window, fused=args.fused)
+
+
+def decode_plan(args, w, step, spb):
+    """(partition tokens, partitions, decode launches, kernel description)."""
+    from paged_kv_cache_410_b200 import binding as B
+    if args.window:
+        span = min(w.max_context, args.window + 15)
+        pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, span, step.cache)
+        n = max(1, math.ceil(span / pt))
+        return pt, n, 1 + (n > 1), (f"pa_decode_sliding_window (window {args.window}; "
+                                    "main + split-K reduce)")
+    if spb:
+        pt = args.partition_tokens or B.pa_decode_shared_prefix_partition_tokens(
+            w.batch, w.num_q_heads, w.max_context, spb, step.cache)
+        n = max(1, math.ceil((w.max_context - spb * w.block_size) / pt))
+        return pt, n, 3, "pa_decode_shared_prefix (prefix + suffix + merge kernels)"
+    pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context, step.cache)
+    n = max(1, math.ceil(w.max_context / pt))
+    name = ("pa_append_decode (append fused into decode; main + split-K reduce)" if args.fused
+            else "pa_decode (main + split-K reduce)")
+    return pt, n, 1 + (n > 1), name
+
+
+def timed_steps(step, steps: int, fused: bool, stream, flush=None):
+    """Record `steps` steps (copy, append, decode) on `stream` with a pair of
+    events around each step and each decode call; with `flush`, the buffer
+    is rewritten before each step, outside its events. Returns the event
+    pairs; read them after a synchronize."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev_step = [(ev(), ev()) for _ in range(steps)]
+    ev_dec = [(ev(), ev()) for _ in range(steps)]
+    call = step.append_decode if fused else step.decode
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(i & 255)
+        ev_step[i][0].record(stream)
+        step.copy()
+        if not fused:
+            step.append()
+        ev_dec[i][0].record(stream)
+        call()
+        ev_dec[i][1].record(stream)
+        ev_step[i][1].record(stream)
+    return ev_step, ev_dec
+
+
+def elapsed(pairs):
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def peak_gbs():
+    peaks = measured_peaks()
+    if peaks and peaks.get("hbm_gbs"):
+        return float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def measure_other(args, name, batch, dev, stream, local_rank, peak):
+    """One more workload in the same run: warm-up, then steps timed with the
+    L2 flushed between them; its decode roofline, clocks, and sampled outputs
+    checked against the oracle."""
+    import torch
+    from paged_kv_cache_410_b200 import accounting as A
+    t_gen = time.perf_counter()
+    w = make_workload(name, 0, batch)
+    t_gen = time.perf_counter() - t_gen
+    spb = int(w.meta.get("shared_prefix_blocks", 0))
+    from paged_kv_cache_410_b200.session import DecodeStep
+    step = DecodeStep(w, dev, shared_prefix_blocks=spb)
+    sb = A.step_bytes(w)
+    db = A.decode_bytes(w)
+    pt, n_parts, dec_launches, kname = decode_plan(
+        argparse.Namespace(window=0, fused=False, partition_tokens=0), w, step, spb)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize(dev)
+    if step.device_errors():
+        raise RuntimeError(f"{name}: device bounds error during warm-up")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps = args.other_steps
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.25)
+    ev_step, ev_dec = timed_steps(step, steps, False, stream, flush)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    step_ms, dec_ms = elapsed(ev_step), elapsed(ev_dec)
+    errs = step.device_errors()
+    del flush
+    dmean = statistics.mean(dec_ms)
+    achieved = sb["decode"] / (dmean * 1e-3) / 1e9
+    res = {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
+           "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+           "kv_cache_dtype": w.cache_dtype, "io_dtype": w.io_dtype,
+           "context_lens": f"{int(w.context_lens.min())}..{int(w.context_lens.max())} "
+                           f"(mean {float(w.context_lens.mean()):.0f})",
+           "decode": f"shared-prefix cascade ({spb} blocks)" if spb else "whole history",
+           "kernel": kname, "partition_tokens": pt, "partitions": n_parts,
+           "steps": steps, "l2": "flushed between steps",
+           "decode_bytes": sb["decode"], "kv_unique_bytes": db["kv_unique"],
+           "kv_logical_bytes": db["kv_logical"],
+           "decode_ms_mean": dmean, "decode_ms_median": statistics.median(dec_ms),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak},
+           "logical_gbs": (db["total_logical"]) / (dmean * 1e-3) / 1e9,
+           "step_ms_mean": statistics.mean(step_ms),
+           "step_gbs": sb["total"] / (statistics.mean(step_ms) * 1e-3) / 1e9,
+           "tokens_per_s_per_layer": w.batch / (dmean * 1e-3),
+           "gpu_launches_per_step": 1 + dec_launches + math.ceil(len(w.copy_pairs) / 256),
+           "clocks": clk, "device_errors": errs, "workload_gen_s": t_gen}
+    if not args.no_cpu_baseline:
+        try:
+            seqs = parity_sample(w, args.other_parity_seqs)
+            _, _, want = oracle_step_time(w, seqs)
+            got = step.out.double().cpu().numpy()[seqs]
+            res["parity"] = parity_summary(got, want, w.io_dtype,
+                                           "float64 CPU oracle, same inputs, sampled sequences")
+        except Exception as e:  # report, never lose the measured line
+            res["parity"] = {"error": repr(e)}
+    _ORACLE_CACHES.pop(id(w), None)
+    del step
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -343,44 +522,18 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     from paged_kv_cache_410_b200 import accounting as A
-    from paged_kv_cache_410_b200 import binding as B
     from paged_kv_cache_410_b200 import build as libbuild
-    from paged_kv_cache_410_b200.session import DecodeStep
     if not os.path.exists(libbuild.LIB):
         raise RuntimeError("libpagedattn.so is not built; run __graft_entry__.build()")
 
     w = make_workload(args.workload, rank, args.batch)
-    spb = w.meta.get("shared_prefix_blocks", 0) if args.cascade == "auto" else 0
-    if args.window or args.fused:
-        spb = 0
-    step = DecodeStep(w, dev, partition_tokens=args.partition_tokens, shared_prefix_blocks=spb,
-                      window=args.window, fused=args.fused)
+    spb = cascade_blocks(args, w)
+    step = make_step(args, w, dev, spb)
     stream = torch.cuda.current_stream(dev)
     sb = A.step_bytes(w, window=args.window, fused=args.fused)
-    if args.window:
-        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(
-            w.batch, min(w.max_context, args.window + 15), step.cache)
-        n_parts = max(1, math.ceil(min(w.max_context, args.window + 15) / plan_pt))
-        decode_launches = 1 + (1 if n_parts > 1 else 0)
-        decode_name = f"pa_decode_sliding_window (window {args.window}; main + split-K reduce)"
-    elif spb:
-        prefix_len = spb * w.block_size
-        plan_pt = args.partition_tokens or B.pa_decode_shared_prefix_partition_tokens(
-            w.batch, w.num_q_heads, w.max_context, spb, step.cache)
-        n_parts = max(1, math.ceil((w.max_context - prefix_len) / plan_pt))
-        decode_launches = 3  # prefix kernel, suffix kernel, merge
-        decode_name = "pa_decode_shared_prefix (prefix + suffix + merge kernels)"
-    else:
-        plan_pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context,
-                                                                         step.cache)
-        n_parts = max(1, math.ceil(w.max_context / plan_pt))
-        decode_launches = 1 + (1 if n_parts > 1 else 0)
-        decode_name = "pa_decode (main + split-K reduce)"
-    if args.fused:
-        decode_name = "pa_append_decode (append fused into decode; main + split-K reduce)"
+    plan_pt, n_parts, decode_launches, decode_name = decode_plan(args, w, step, spb)
     launches_per_step = (0 if args.fused else 1) + decode_launches + math.ceil(
         len(w.copy_pairs) / 256)
-    timed_call = step.append_decode if args.fused else step.decode
     timed_bytes = sb["append_decode"] if args.fused else sb["decode"]
 
     for _ in range(args.warmup):
@@ -389,33 +542,38 @@ def run_ours(args):
     if step.device_errors():
         raise RuntimeError("device bounds error during warm-up")
 
-    # ---- device-timed steps, per-call events for the decode roofline ----
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # ---- device-timed steps: L2 flushed between steps (default), then the
+    # same steps back to back ----
+    flush = None if args.no_flush else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.25)  # let the sampler start before the timed region
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step.copy()
-        if not args.fused:
-            step.append()
-        ev[i][0].record(stream)
-        timed_call()
-        ev[i][1].record(stream)
-    t_end.record(stream)
+    ev_step, ev_dec = timed_steps(step, args.steps, args.fused, stream, flush)
     torch.cuda.synchronize(dev)
-    clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    ms_local = t_start.elapsed_time(t_end)
-    decode_ms = [a.elapsed_time(b) for a, b in ev]
-    ms_total = max_over_ranks(ms_local, dev)
+    step_ms, decode_ms = elapsed(ev_step), elapsed(ev_dec)
+    # back to back, no flush (the step reads more than L2 holds for the
+    # default workload, so the two should agree)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    ev_dec_nf = None
+    if flush is not None:
+        del flush
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        t_start.record(stream)
+        _, ev_dec_nf = timed_steps(step, args.steps, args.fused, stream, None)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(sum(step_ms), dev)
     ms_per_step = ms_total / args.steps
     total_bytes = sum_over_ranks(sb["total"], dev) * args.steps
     value = total_bytes / (ms_total * 1e-3) / 1e9
@@ -451,21 +609,13 @@ def run_ours(args):
     errs = step.device_errors()
 
     # ---- roofline of the decode call ----
-    peaks = measured_peaks()
-    if peaks and peaks.get("hbm_gbs"):
-        peak, peak_src = float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
-    else:
-        peak, peak_src = FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+    peak, peak_src = peak_gbs()
     dec_ms = statistics.mean(decode_ms)
     achieved = timed_bytes / (dec_ms * 1e-3) / 1e9
     # the committed ncu counters cover the plain whole-history decode only
     traffic = None if (args.window or args.fused or spb) else recorded_traffic(w.name)
 
-    line = base_line(args, w, world)
-    line["config"]["decode"] = ("append fused into decode" if args.fused else
-                                f"sliding window {args.window}" if args.window else
-                                f"shared-prefix cascade ({spb} blocks)" if spb else
-                                "whole history")
+    line = base_line(args, w, world, spb)
     line.update({
         "value": value, "ms_per_step": ms_per_step,
         "tokens_per_s_per_layer": tokens_per_s,
@@ -485,6 +635,15 @@ def run_ours(args):
         "clocks": clk,
         "device_errors": errs,
     })
+    if ev_dec_nf is not None:
+        nf_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+        nf_dec = statistics.mean(elapsed(ev_dec_nf))
+        line["unflushed"] = {
+            "value": total_bytes / (nf_ms * 1e-3) / 1e9, "ms_per_step": nf_ms / args.steps,
+            "decode_ms_mean": nf_dec,
+            "roofline_achieved": timed_bytes / (nf_dec * 1e-3) / 1e9,
+            "roofline_frac": timed_bytes / (nf_dec * 1e-3) / 1e9 / peak,
+            "note": "the same steps back to back, without the L2 flush"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
@@ -495,6 +654,20 @@ def run_ours(args):
             line["parity"] = parity_summary(got, want, w.io_dtype)
         except Exception as e:  # report, never lose the measured line
             line["parity"] = {"error": repr(e)}
+    if world == 1 and not args.no_other_configs:
+        del step
+        _ORACLE_CACHES.clear()
+        torch.cuda.empty_cache()
+        line["other_configs"] = {}
+        for name, batch in OTHER_CONFIGS:
+            if name == args.workload and batch == args.batch:
+                continue
+            key = name if batch is None else f"{name}_b{batch}"
+            try:
+                line["other_configs"][key] = measure_other(args, name, batch, dev, stream,
+                                                           local_rank, peak)
+            except Exception as e:  # report, never lose the headline
+                line["other_configs"][key] = {"error": repr(e)}
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -531,6 +704,16 @@ def main(argv=None):
     ap.add_argument("--cascade", choices=["auto", "off"], default="auto",
                     help="decode a workload whose sequences share prefix blocks through "
                          "pa_decode_shared_prefix (auto) or plain pa_decode (off)")
+    ap.add_argument("--no-flush", action="store_true",
+                    help="time the steps back to back without writing the L2 flush buffer "
+                         "between them")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="measure the headline workload only (at one GPU the line otherwise "
+                         "adds the other benchmark families)")
+    ap.add_argument("--other-steps", type=int, default=100,
+                    help="timed steps of each other workload")
+    ap.add_argument("--other-parity-seqs", type=int, default=16,
+                    help="sequences of each other workload checked against the oracle")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -1,5 +1,6 @@
 """Host-side logic of bench.py on the CPU: the multi-rank reductions over a
 2-rank gloo group, per-rank workloads, and the reference (CPU oracle) arm."""
+import argparse
 import json
 import os
 import subprocess
@@ -128,3 +129,46 @@ def test_small_fp8_batches_scale_the_beam_groups():
         assert bench.make_workload("fp8_beams", 0, 256).meta["beam_groups"] == 16
     finally:
         W.normal_bits = orig
+
+
+def test_reference_arm_config_equals_the_gpu_arms():
+    """Both arms describe the same workload with the same config object, the
+    decode path included (the driver compares them)."""
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    for extra in ([], ["--no-flush"]):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                            "--workload", "tiny_mha", "--steps", "2", "--warmup", "3", *extra],
+                           capture_output=True, text=True, env=env, timeout=300)
+        assert r.returncode == 0, r.stderr
+        d = json.loads(r.stdout.strip().splitlines()[-1])
+        args = argparse.Namespace(steps=2, warmup=3, cascade="auto", window=0, fused=False,
+                                  no_flush=bool(extra))
+        w = bench.make_workload("tiny_mha", 0, None)
+        want = bench.base_line(args, w, 1, bench.cascade_blocks(args, w))["config"]
+        assert d["config"] == want
+        assert d["config"]["decode"] == "whole history"
+        assert d["config"]["l2"].startswith("not flushed" if extra else "flushed")
+
+
+def test_cascade_label_for_the_shared_prefix_family():
+    from paged_kv_cache_410_b200 import workloads as W
+    w = W.custom_shared_prefix(64, [0, 5, 40], num_q_heads=8, num_kv_heads=2, head_dim=64,
+                               block_size=16, dtype="bf16", seed=3)
+    auto = argparse.Namespace(cascade="auto", window=0, fused=False)
+    assert bench.cascade_blocks(auto, w) == 4
+    assert bench.decode_label(auto, 4) == "shared-prefix cascade (4 blocks)"
+    for other in (argparse.Namespace(cascade="off", window=0, fused=False),
+                  argparse.Namespace(cascade="auto", window=64, fused=False),
+                  argparse.Namespace(cascade="auto", window=0, fused=True)):
+        assert bench.cascade_blocks(other, w) == 0
+
+
+def test_parity_sample_takes_the_extremes_and_a_beam_group():
+    from paged_kv_cache_410_b200 import workloads as W
+    w = W.fp8_beams(batch=40, beam_groups=3, median_len=40, max_len=200)
+    s = bench.parity_sample(w, 12)
+    assert len(s) == len(set(s.tolist())) and np.all(np.diff(s) > 0)
+    assert {0, 1, 2, 3} <= set(s.tolist())
+    assert int(np.argmin(w.context_lens)) in s and int(np.argmax(w.context_lens)) in s
+    assert len(s) <= 12 + 2
+    assert np.array_equal(bench.parity_sample(w, 100), np.arange(40))
