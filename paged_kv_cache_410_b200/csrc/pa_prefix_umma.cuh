@@ -9,16 +9,20 @@
 // (of any sequences) and one chunk of prefix tokens, 64 tokens per step;
 // per tile:
 //   S (128 x 64, f32, TMEM)  = Q (128 x D, smem) . K_tile^T (64 x D, smem)
-//   P (128 x 64, 16-bit, smem) = 2^(S * scale * log2(e) - m)     [one row per thread]
-//   O (128 x D, f32, TMEM)  += P . V_tile (64 x D, smem)
+//   P (128 x 64, 16-bit, TMEM) = 2^(S * scale * log2(e) - m)     [one row per thread]
+//   O (128 x D, f32, TMEM)  += P (TMEM) . V_tile (64 x D, smem)
 // and writes, per query row, the normalised partial (O / l, m, l) that the
-// split-K merge combines with the row's suffix partials.
+// split-K merge combines with the row's suffix partials. P is written over
+// the S buffer it was computed from (two 16-bit values per 32-bit column)
+// and is the A operand of the P.V MMA straight from tensor memory, so P
+// needs no shared memory: the CTA's tiles take 128 KB at head_dim 128, and a
+// suffix decode CTA fits on the same SM.
 //
 // Shared-memory tiles use the 128-byte swizzle (rows of 128 bytes, 16-byte
 // chunk c of row r stored at chunk c ^ (r % 8), 8-row atoms of 1024 bytes);
-// a D-channel row is split into D/64 slabs of 64 channels. Q, K and P are
-// K-major operands (channels or tokens contiguous); V is read MN-major
-// straight from its token-major tile. A producer warp moves the tiles with
+// a D-channel row is split into D/64 slabs of 64 channels. Q and K are
+// K-major operands (channels contiguous); V is read MN-major straight from
+// its token-major tile. A producer warp moves the tiles with
 // TMA (3-D tensor maps over q [batch][Hq][D] and the caches [slot][Hkv][D],
 // one box per cache block of >= 8 tokens and 64-channel slab, no
 // multicast), one thread of an MMA warp issues the MMAs, and the partial
@@ -49,7 +53,8 @@ struct UmmaCfg {
   static constexpr int kProducerWarp = kSoftmaxWarps;
   static constexpr int kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
-  // TMEM columns: S of tile t, buffer b at t*128 + b*64; O of tile t at
+  // TMEM columns: S of tile t, buffer b at t*128 + b*64 (P(it), 16-bit
+  // pairs, over the first 32 columns of S(it)'s buffer); O of tile t at
   // NT*128 + t*D; allocated as a power of two
   static constexpr int kOCol = NT * 2 * kUmmaTokens;
   static constexpr int kColsUsed = kOCol + NT * D;
@@ -59,12 +64,13 @@ struct UmmaCfg {
   static constexpr int kQTile = kSlabs * kUmmaRows * 128;     // one row tile of Q
   static constexpr int kTileSlab = kUmmaTokens * 128;          // one slab of a K/V stage
   static constexpr int kTileBytes = kSlabs * kTileSlab;        // one K or V stage
-  static constexpr int kPTile = kUmmaRows * 128;               // P of one row tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + NT * kQTile;
   static constexpr int kV = kK + NSTAGE * kTileBytes;
-  static constexpr int kP = kV + NSTAGE * kTileBytes;
-  static constexpr int kBytes = kP + NT * kPTile;
+  static constexpr int kBytes = kV + NSTAGE * kTileBytes;
+  // the epilogue stages each tile's partial outputs (128 rows x D f32) over
+  // the tiles
+  static_assert(NT * kUmmaRows * D * 4 <= kBytes, "epilogue staging fits in the tiles");
   static constexpr int kSmall = 256;  // mbarriers, TMEM address, abort flag
   // requested: the tiles plus slack to align them to 1024 bytes (the small
   // items live in the slack when it has room, else after the tiles)
@@ -220,6 +226,20 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D (TMEM) (+)= A (TMEM) . B (smem), 16-bit inputs, f32 accumulate; A is
+// M x K with row i in TMEM lane i and two 16-bit K elements per 32-bit
+// column (K = 16: 8 columns from a_tmem).
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  setp.ne.b32 p, %4, 0;\n"
+      "  tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
@@ -247,16 +267,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  uint32_t r[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
       "%28, %29, %30, %31, %32};\n" ::"r"(taddr),
       PA_R32(PA_IN)
       : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  uint32_t r[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
+  tmem_st32u(taddr, r);
 }
 #undef PA_R32
 #undef PA_OUT
@@ -283,10 +306,6 @@ __host__ __device__ constexpr uint32_t umma_idesc() {
          ((B_MN ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(kUmmaRows >> 4) << 24);
 }
-// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled slab.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
 
 // ---- the kernel ---------------------------------------------------------------
 
@@ -298,9 +317,11 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 //   producer:  TMA loads of Q and of the K and V stages, each stage refilled
 //              as soon as the MMAs that read it are done;
 //   MMA warp:  S(it+1) of all tiles is issued before P.V(it), so the tensor
-//              core computes the next scores while the softmax warps work.
-// The roles meet only at mbarriers (full / free per stage, S full / S read,
-// P written, P.V done); every wait is bounded and a timeout aborts all roles.
+//              core computes the next scores while the softmax warps work;
+//              S(it+1) goes into the buffer that held P(it-1), so it is issued
+//              once P.V(it-1) has completed.
+// The roles meet only at mbarriers (full / free per stage, S full, P written,
+// P.V done); every wait is bounded and a timeout aborts all roles.
 template <typename TQ, int D, int NT, int NSTAGE>
 __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     pa_prefix_umma_kernel(const DecodeParams p, const UmmaGrid ug,
@@ -327,7 +348,6 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
   const uint32_t bar_kfree = small + 72;     // + 8 * stage
   const uint32_t bar_vfree = small + 104;    // + 8 * stage
   const uint32_t bar_sfull = small + 136;    // + 8 * S buffer
-  const uint32_t bar_sfree = small + 152;    // + 8 * S buffer
   const uint32_t bar_pfull = small + 168;
   const uint32_t bar_pv = small + 176;
   const uint32_t bar_done = small + 184;
@@ -337,7 +357,6 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
   const uint32_t sQ = base + C::kQ;
   const uint32_t sK = base + C::kK;
   const uint32_t sV = base + C::kV;
-  const uint32_t sP = base + C::kP;
   static_assert(NSTAGE >= 2 && NSTAGE <= 4, "stages");
 
   const int tid = threadIdx.x;
@@ -365,10 +384,7 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
       mbar_init(bar_kfree + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_sfull + 8 * i, 1);
-      mbar_init(bar_sfree + 8 * i, C::kSoftmaxThreads);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(bar_sfull + 8 * i, 1);
     mbar_init(bar_pfull, C::kSoftmaxThreads);
     mbar_init(bar_pv, 1);
     mbar_init(bar_done, 1);
@@ -478,8 +494,8 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
       auto issue_s = [&](int i) -> bool {
         if (!mbar_wait_or_abort(bar_kfull + 8 * (i % NSTAGE), stage_parity(i), abort))
           return false;
-        if (i >= 2 && !mbar_wait_or_abort(bar_sfree + 8 * (i & 1),
-                                          static_cast<uint32_t>(((i - 2) >> 1) & 1), abort))
+        // S buffer i & 1 holds P(i - 2) until P.V(i - 2) has read it
+        if (i >= 2 && !mbar_wait_or_abort(bar_pv, static_cast<uint32_t>((i - 2) & 1), abort))
           return false;
         tc_fence_after();
         const uint32_t kst = sK + (i % NSTAGE) * C::kTileBytes;
@@ -514,9 +530,10 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
         for (int t = 0; t < NT; ++t)
 #pragma unroll
           for (int kk = 0; kk < kUmmaTokens / 16; ++kk) {
-            const uint64_t a = sw128_desc(sP + t * C::kPTile + kk * 32, 16, 1024);
+            // P(it): 16 tokens = 8 columns of tile t's S buffer it & 1
+            const uint32_t a = tmem + t * 2 * kUmmaTokens + (it & 1) * kUmmaTokens + kk * 8;
             const uint64_t b = sw128_desc(vst + kk * 16 * 128, C::kTileSlab, 1024);
-            umma_f16(tmem + C::kOCol + t * D, a, b, kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
+            umma_f16_tmem_a(tmem + C::kOCol + t * D, a, b, kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
           }
         umma_commit(bar_pv);
         umma_commit(bar_vfree + 8 * (it % NSTAGE));
@@ -532,7 +549,6 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
     const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + t_lane + tile * 2 * kUmmaTokens;
     const uint32_t tO = tmem + t_lane + C::kOCol + tile * D;
-    const uint32_t sPt = sP + tile * C::kPTile;
     float m_run = -INFINITY;
     float l_run = 0.f;
     for (int it = 0; it < nsteps; ++it) {
@@ -551,35 +567,40 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
         for (int j = 0; j < 32; ++j) s[32 + j] = h[j];
         tmem_ld_wait();
       }
-      tc_fence_before();
-      mbar_arrive(bar_sfree + 8 * (it & 1));
 
       const int nvalid = c1 - (c0 + it * kUmmaTokens);
       const bool full = nvalid >= kUmmaTokens;  // every step but a chunk's ragged last one
-      float mx = -INFINITY;
+      // row max as a tree of 8 independent partial maxima (a thread owns the
+      // whole row, so a single running max would be a 64-long dependency chain)
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < kUmmaTokens; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
       } else {
 #pragma unroll
-        for (int j = 0; j < kUmmaTokens; ++j) mx = fmaxf(mx, j < nvalid ? s[j] : -INFINITY);
+        for (int j = 0; j < kUmmaTokens; ++j)
+          m8[j & 7] = fmaxf(m8[j & 7], j < nvalid ? s[j] : -INFINITY);
       }
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= p.scale_log2;
       const bool up = mx > m_run + kRescaleLog2;  // the first step always moves it
       const float m_ref = up ? mx : m_run;
       const float alpha = up ? ex2(m_run - m_ref) : 1.f;
 
       // P row (64 tokens, packed in pairs), computed while P.V(it-1) may
-      // still be running
+      // still be running, and written over S(it) (this thread's TMEM lane)
       uint32_t pw[kUmmaTokens / 2];
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (as the max: no long chain)
       auto expo = [&](int j) { return ex2(fmaf(s[j], p.scale_log2, -m_ref)); };
       if (full) {
 #pragma unroll
         for (int j = 0; j < kUmmaTokens; j += 2) {
           const float p0 = expo(j);
           const float p1 = expo(j + 1);
-          sum += p0 + p1;
+          sum4[(j >> 1) & 3] += p0 + p1;
           pw[j / 2] = pack2<BF16>(p0, p1);
         }
       } else {
@@ -587,17 +608,23 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
         for (int j = 0; j < kUmmaTokens; j += 2) {
           const float p0 = j < nvalid ? expo(j) : 0.f;
           const float p1 = j + 1 < nvalid ? expo(j + 1) : 0.f;
-          sum += p0 + p1;
+          sum4[(j >> 1) & 3] += p0 + p1;
           pw[j / 2] = pack2<BF16>(p0, p1);
         }
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run = l_run * alpha + sum;
       m_run = m_ref;
+      static_assert(kUmmaTokens / 2 == 32, "one 32-column store of P");
+      tmem_st32u(tS + (it & 1) * kUmmaTokens, pw);
 
-      if (it > 0) {  // P.V(it-1) done: the P tile and O are free
+      if (it > 0) {  // P.V(it-1) done: O is free
         ok = __all_sync(0xffffffffu,
                         mbar_wait_or_abort(bar_pv, static_cast<uint32_t>((it - 1) & 1), abort));
-        if (!ok) break;
+        if (!ok) {
+          tmem_st_wait();  // (P's store) before the CTA drains
+          break;
+        }
         tc_fence_after();
         // rows whose reference max moved rescale their O row
         if (__any_sync(0xffffffffu, up)) {
@@ -610,16 +637,9 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
             tmem_st32(tO + c, o);
           }
-          tmem_st_wait();
         }
       }
-      // P tile (128-byte swizzled, K-major): 8 chunks of 8 values
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sPt + sw128_off(my_row, c)),
-                     "r"(pw[4 * c]), "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3])
-                     : "memory");
-      fence_async_smem();
+      tmem_st_wait();  // P (and a rescaled O) in tensor memory
       tc_fence_before();
       mbar_arrive(bar_pfull);
     }
