@@ -305,13 +305,16 @@ pa_status pa_get_device_error(void* stream, uint32_t* flags);
  * workspace is a fixed 32 MiB array in the library's own device memory
  * (reserved on every GPU that loads the library, until the process exits),
  * so the call allocates nothing; inputs and outputs are still the caller's.
- * Arguments and results are those of pa_decode (same partition choice), minus
- * the workspace. If the plan needs more than 32 MiB of workspace
+ * Arguments and results are those of pa_decode (same partition choice, same
+ * argument checks and status codes, bitwise the same output), minus the
+ * workspace. If a valid call's plan needs more than 32 MiB of workspace
  * (pa_decode_workspace_size(...) > 32 MiB) the call returns
  * PA_ERR_WORKSPACE and enqueues nothing; use pa_decode with a larger buffer
  * or a longer partition.
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) while that device is current; make that first call
+ * The array's device address belongs to a CUDA context: the first call in
+ * each context (a device's primary context, or a context the caller made
+ * current, or one created after a device reset) looks it up with
+ * cudaGetSymbolAddress while that context is current; make that first call
  * before any stream capture. Every call on a device shares the one array,
  * which keeps the previous call's contents (nothing in it needs a starting
  * value); calls whose kernels overlap on the GPU -- concurrent streams, or

@@ -65,11 +65,27 @@ int64_t elem_bytes(int dtype) { return dtype == PA_E4M3 ? 1 : 2; }
 // Partition length used when the caller passes 0: the tokens whose K rows of
 // one KV head take 128 KB (512 at fp16/bf16 and head_dim 128, 1024 for E4M3
 // or head_dim 64), halved (down to 64) while the launch would have fewer
-// than two CTAs per SM.
+// than two CTAs per SM. When the sequences alone are fewer than one wave of
+// CTAs (batch x KV heads below kWaveCtas, so the split is what fills the
+// GPU: long contexts at small batch), the partition is then lengthened to
+// the shortest multiple of 16 tokens whose CTAs make whole waves: of equal
+// CTAs, a last partial wave costs as long as a full one.
+constexpr int kDecodeCtasPerSm = 3;  // decode CTAs resident per SM at head_dim 128
+constexpr int64_t kWaveCtas = int64_t{kDecodeCtasPerSm} * kNumSMs;
+
 int auto_partition(int64_t batch, int64_t max_context, const pa_cache_desc* cd) {
   int pt = kPartitionRowBytes / static_cast<int>(cd->head_dim * elem_bytes(cd->cache_dtype));
-  auto ctas = [&](int p) { return batch * cd->num_kv_heads * ((max_context + p - 1) / p); };
+  auto ctas = [&](int64_t p) { return batch * cd->num_kv_heads * ((max_context + p - 1) / p); };
   while (pt > kMinAutoPartition && ctas(pt) < 2 * kNumSMs) pt >>= 1;
+  const int64_t rows = batch * cd->num_kv_heads;  // (sequence, KV head) pairs
+  if (cd->head_dim == 128 && rows > 0 && rows < kWaveCtas) {
+    const int64_t waves = ctas(pt) / kWaveCtas;
+    if (waves >= 1 && ctas(pt) % kWaveCtas != 0) {
+      const int64_t parts = waves * kWaveCtas / rows;  // partitions per row in whole waves
+      const int64_t pt2 = ((max_context + parts - 1) / parts + 15) / 16 * 16;
+      if (pt2 <= (int64_t{1} << 20) && ctas(pt2) <= waves * kWaveCtas) pt = static_cast<int>(pt2);
+    }
+  }
   return pt;
 }
 
@@ -115,7 +131,10 @@ Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int part
 }
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device),
-// raised to the largest size requested so far.
+// raised to the largest size requested so far. Every kernel that comes here
+// also prefers the largest shared-memory carveout (228 KB per SM), so that
+// CTAs of the shared-prefix and suffix-decode kernels, which run side by
+// side, find the same split of each SM and fit next to each other.
 cudaError_t ensure_smem(const void* kernel, int bytes) {
   static std::mutex mu;
   static std::unordered_map<const void*, std::array<int, 64>> done;
@@ -127,6 +146,11 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
   if (it == done.end()) it = done.emplace(kernel, std::array<int, 64>{}).first;
   int& have = it->second[dev & 63];
   if (have >= bytes) return cudaSuccess;
+  if (have == 0) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+  }
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) have = bytes;
   return e;
@@ -156,9 +180,10 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
                       : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
-  const int bt_entries =
-      std::min((p.partition_tokens >> p.bs_log2) + 2, pa::kBlockIdsInSmem);
-  const int smem = S::kMainBytes + bt_entries * 4;
+  const int bt_entries = pa::staged_block_ids(p.partition_tokens, p.bs_log2);
+  const int smem = (p.k_new && CK == pa::kE4M3)
+                       ? S::new_rows_offset(bt_entries) + S::kNewRowBytes
+                       : S::kMainBytes + bt_entries * 4;
   if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
   if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
   dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
@@ -896,21 +921,56 @@ constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;  // 32 MiB per device
 // Reserved in every device context that loads this library, until exit.
 static __device__ __align__(256) unsigned char g_pa_static_workspace[kStaticWorkspaceBytes];
 
-// Device address of g_pa_static_workspace on the current device. In host code
-// the array's name is only a host-side handle, so the address is looked up
-// once per device with cudaGetSymbolAddress (the first call on each device).
+// Device address of g_pa_static_workspace in the current CUDA context. In
+// host code the array's name is only a host-side handle; the device address
+// belongs to a context (each device's primary context, or one the caller made
+// current), so it is looked up with cudaGetSymbolAddress on the first call in
+// each context and kept under that context's process-unique id (cuCtxGetId),
+// which a context created after a device reset does not share.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(f);
+}
+
+// Id of the context current on this thread (0 when none is current yet).
+bool current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  *id = 0;
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  return ctx == nullptr || get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 pa_status static_workspace_address(void** out) {
   static std::mutex mu;
-  static std::array<void*, 64> addr{};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  static std::unordered_map<unsigned long long, void*> addr;  // context id -> address
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_pa_static_workspace) != cudaSuccess || !p) return PA_ERR_CUDA;
-    addr[dev] = p;
+  if (id != 0) {
+    const auto it = addr.find(id);
+    if (it != addr.end()) {
+      *out = it->second;
+      return PA_OK;
+    }
   }
-  *out = addr[dev];
+  // first call in this context (or no context yet: the lookup makes the
+  // current device's primary context current)
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_pa_static_workspace) != cudaSuccess || !p) return PA_ERR_CUDA;
+  if (id == 0 && (!current_context_id(&id) || id == 0)) return PA_ERR_CUDA;
+  addr[id] = p;
+  *out = p;
   return PA_OK;
 }
 
@@ -921,14 +981,17 @@ extern "C" pa_status pa_decode_static_workspace(
     const void* v_cache, const pa_cache_desc* cache, const int32_t* block_tables,
     int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context, float scale,
     void* out, int32_t partition_tokens, void* stream) {
+  // the argument checks of pa_decode come first, so that an invalid call
+  // gets the same status from both entry points
   int bs_log2 = 0;
-  pa_status st = check_cache(cache, &bs_log2);
-  if (st != PA_OK) return st;
-  if (batch < 0 || num_q_heads <= 0 || max_context < 0 || partition_tokens < 0)
-    return PA_ERR_INVALID_ARG;
-  const size_t need =
-      batch > 0 ? pa_decode_workspace_size(batch, num_q_heads, max_context, partition_tokens, cache)
-                : 0;
+  bool nothing = false;
+  pa_status st = check_decode_args(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, out, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK || nothing) return st;
+  const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
+  const size_t need = pl.ws_bytes;
   if (need > kStaticWorkspaceBytes) return PA_ERR_WORKSPACE;
   void* ws = nullptr;
   if (need > 0) {

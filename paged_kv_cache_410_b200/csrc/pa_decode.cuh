@@ -10,15 +10,15 @@
 // `partition_tokens` tokens): every query head of the KV head's group
 // (grouped-query attention, KV cache article section "显存账本") is served
 // from one read of the partition's K and V, so KV bytes cross HBM once per
-// KV head. Warps of the CTA take 16-token tiles round-robin, each with its
-// own NSTAGE-deep cp.async pipeline into shared memory (no CTA-wide barrier
-// in the main loop), and keep their own running max / sum / output (online
-// softmax). At the end the warps merge through shared memory; a sequence
+// KV head. Warps of the CTA take tiles of 16 tokens (32 for an E4M3 cache)
+// round-robin, each with its own NSTAGE-deep cp.async pipeline into shared
+// memory (no CTA-wide barrier in the main loop), and keep their own running
+// max / sum / output (online softmax). At the end the warps merge through shared memory; a sequence
 // that spans one partition writes its output directly, longer ones write
 // (max, sum, normalised output) partials that the reduce kernel combines.
 //
-// Tensor cores, transposed products. With 16 tokens per tile and up to 8
-// query heads per MMA column block:
+// Tensor cores, transposed products. With 16 tokens per MMA row block and up
+// to 8 query heads per MMA column block:
 //   S^T (16 tokens x 8 heads) = K_tile (16 x D) . Q^T (D x 8)   [m16n8k16]
 //   O^T (D x 8 heads)        += V_tile^T (D x 16) . P^T (16 x 8)
 // K tiles feed the A operand through ldmatrix, V tiles through
@@ -26,10 +26,16 @@
 // partition; P^T is the S^T accumulator after the softmax, converted to
 // 16 bits and transposed in registers with movmatrix. Rows of every MMA are
 // tokens or channels, so no accumulator row is padding; groups of 9..16
-// query heads use two column blocks. For an E4M3 cache the codes are widened
-// to f16 (exactly) in registers; the K scale is folded into the query (as an
-// f16 hi + lo pair, so the fold costs no precision) and the V scale is
-// applied to the merged output.
+// query heads use two column blocks.
+//
+// E4M3 caches. A tile is 32 tokens (8 KB of K and V at head_dim 128, as a
+// 16-token tile of a 16-bit cache), and S^T = K Q^T runs on E4M3 operands
+// (m16n8k32): K tiles enter the MMA as stored, and the query, with the K
+// scale folded in (q' = q * k_scale), is three E4M3 terms after a power-of-
+// two scaling of its row, so that their sum carries about as many bits as
+// f16. The V codes are widened to f16 (exactly) in registers for
+// O^T += V^T P^T with P in f16, and the V scale is applied to the merged
+// output.
 #pragma once
 
 #include "pa_common.cuh"
@@ -150,12 +156,13 @@ constexpr int kBlockIdsInSmem = 1024;
 // cancels in the final normalisation.
 constexpr float kRescaleLog2 = 8.f;
 
-template <int CK, int D>
+template <int CK, int D, int TOK = 16>
 struct TileGeom {
   static constexpr int ES = (CK == kE4M3) ? 1 : 2;  // bytes per cache element
   static constexpr int RB = D * ES;                  // bytes per token row (one head)
   static constexpr int CPR = RB / 16;                // 16-byte chunks per row
-  static constexpr int TB = 16 * RB;                 // one 16-token tile of K (or V)
+  static constexpr int TOKENS = TOK;                 // rows of a tile
+  static constexpr int TB = TOK * RB;                // one tile of K (or V)
   static_assert(CPR == 4 || CPR == 8 || CPR == 16, "unsupported row size");
   // Byte offset of 16-byte chunk `c` of row `r` inside a tile. Rows of 128 B
   // or more XOR the low three chunk bits with the row, so that 8 rows read
@@ -172,15 +179,35 @@ struct TileGeom {
   }
 };
 
+// Tokens of a decode tile: 16 for 16-bit caches, 32 for E4M3 (the same
+// bytes per tile).
+template <int CK>
+__host__ __device__ constexpr int decode_tile_tokens() {
+  return CK == kE4M3 ? 32 : 16;
+}
+
 template <int CK, int D, int NW, int NSTAGE>
 struct DecodeSmem {
-  using G = TileGeom<CK, D>;
+  using G = TileGeom<CK, D, decode_tile_tokens<CK>()>;
   static constexpr int kStageBytes = 2 * G::TB;  // K tile + V tile
   static constexpr int kPipeBytes = NW * NSTAGE * kStageBytes;
   static constexpr int kMergeBytes = NW * 16 * D * 4 + NW * 16 * 3 * 4 + 32 * 4;
   static constexpr int kMainBytes = kPipeBytes > kMergeBytes ? kPipeBytes : kMergeBytes;
   // + block-table slice of the partition (int32), sized at launch
+  // + (fused append into an E4M3 cache) the new token's quantised K and V
+  //   rows, 16-byte aligned after the block ids
+  static constexpr int kNewRowBytes = 2 * G::RB;
+  __host__ __device__ static constexpr int new_rows_offset(int bt_entries) {
+    return kMainBytes + (4 * bt_entries + 15) / 16 * 16;
+  }
 };
+
+// Block ids of a partition staged in shared memory (the launch sizes the
+// slice for this many).
+__host__ __device__ inline int staged_block_ids(int partition_tokens, int bs_log2) {
+  const int n = (partition_tokens >> bs_log2) + 2;
+  return n < kBlockIdsInSmem ? n : kBlockIdsInSmem;
+}
 
 // ---- per-warp attention math shared by the decode and prefix kernels -------
 //
@@ -188,48 +215,98 @@ struct DecodeSmem {
 // holds the B-operand fragments of column 8*nh + g and the O^T accumulator
 // o[mt][nh] = {(channel row g, columns 2t, 2t+1), (channel row g+8, same)}.
 
-// Q^T fragments: qb[kk][nh] = {channels of k-slots 2t,2t+1 ; 2t+8,2t+9} of the
-// query row rows[nh] (nullptr: a padding column of zeros). For E4M3 the row
-// is first multiplied by the K scale (q' = q * k_scale) and split into f16
-// hi + lo; its channel order inside each 32-channel group gq (shared with the
-// K fragments of attend_tile): k-step 2gq + h holds channels 8t + 4h + {0,1}
-// in slots 2t, 2t+1 and 8t + 4h + {2,3} in slots 2t+8, 2t+9.
-template <typename TQ, int CK, int D, int NH>
-__device__ __forceinline__ void load_query_fragments(
-    const TQ* const (&rows)[NH], const float* k_scale_row, uint32_t (&qb)[D / 16][NH][2],
-    uint32_t (&qlo)[CK == kE4M3 ? D / 16 : 1][NH][2]) {
+// Q^T fragments (16-bit caches): qb[kk][nh] = {channels of k-slots 2t,2t+1 ;
+// 2t+8,2t+9} of the query row rows[nh] (nullptr: a padding column of zeros).
+template <typename TQ, int D, int NH>
+__device__ __forceinline__ void load_query_fragments(const TQ* const (&rows)[NH],
+                                                     uint32_t (&qb)[D / 16][NH][2]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(rows[nh]);
+    const bool ok = q32 != nullptr;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qb[kk][nh][0] = ok ? q32[(kk * 16 + 2 * t) / 2] : 0u;
+      qb[kk][nh][1] = ok ? q32[(kk * 16 + 8 + 2 * t) / 2] : 0u;
+    }
+  }
+}
+
+// E4M3 codes of two floats and the floats they decode to.
+__device__ __forceinline__ uint32_t e4m3x2_round(float lo, float hi, float& rlo, float& rhi) {
+  const uint32_t code = f32x2_to_e4m3x2(lo, hi);
+  uint32_t h, unused;
+  e4m3x4_to_f16x2x2(code, h, unused);
+  const __half2 v = *reinterpret_cast<const __half2*>(&h);
+  rlo = __low2float(v);
+  rhi = __high2float(v);
+  return code;
+}
+
+// Q^T fragments for an E4M3 cache (B operand of m16n8k32). Thread (g, t)
+// holds query row rows[nh] (column g of block nh; nullptr: zeros) times the K
+// scale, q' = q * k_scale, scaled by 2^e with e chosen per row so that
+// max |q'| 2^e lies in [128, 256), as three E4M3 terms: term 1 = e4m3(q' 2^e),
+// term 2 = e4m3 of what term 1 leaves, term 3 = e4m3 of what both leave.
+// qf[j][kk][nh] = {channels 32kk + 4t .. 32kk + 4t + 3 ; 32kk + 16 + 4t ..
+// + 3} of term j. sl2[nh][e] = scale_log2 * 2^-e of the row in accumulator
+// column 2t + e, which undoes the scaling in the softmax.
+template <typename TQ, int D, int NH>
+__device__ __forceinline__ void load_query_e4m3(const TQ* const (&rows)[NH], const float* ks,
+                                                float scale_log2, uint32_t (&qf)[3][D / 32][NH][2],
+                                                float (&sl2)[NH][2]) {
   const int t = threadIdx.x & 3;
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) {
     const TQ* qr = rows[nh];
     const bool ok = qr != nullptr;
-    if constexpr (CK != kE4M3) {
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qr);
+    float x[D / 32][2][4];
+    float mx = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        qb[kk][nh][0] = ok ? q32[(kk * 16 + 2 * t) / 2] : 0u;
-        qb[kk][nh][1] = ok ? q32[(kk * 16 + 8 + 2 * t) / 2] : 0u;
-      }
-    } else {
+    for (int kk = 0; kk < D / 32; ++kk)
 #pragma unroll
-      for (int gq = 0; gq < D / 32; ++gq) {
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int kk = 2 * gq + h;
-          const int c = gq * 32 + 8 * t + 4 * h;
-          float x[4], hi[4], lo[4];
+        for (int i = 0; i < 4; ++i) {
+          const int c = 32 * kk + 16 * h + 4 * t + i;
+          x[kk][h][i] = ok ? to_f32<TQ>(qr[c]) * ks[c] : 0.f;
+          mx = fmaxf(mx, fabsf(x[kk][h][i]));
+        }
+    // the four threads of the group hold the row's channels between them
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    // e = 7 - floor(log2 mx) (from the exponent field; kept within a range
+    // where 2^e and 2^-e are normal floats)
+    int e = 0;
+    if (mx > 0.f) {
+      const int ex = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+      e = min(max(7 - ex, -100), 100);
+    }
+    const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);  // 2^e
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            x[e] = ok ? to_f32<TQ>(qr[c + e]) * k_scale_row[c + e] : 0.f;
-            hi[e] = __half2float(__float2half_rn(x[e]));
-            lo[e] = x[e] - hi[e];
-          }
-          qb[kk][nh][0] = pack2<false>(hi[0], hi[1]);
-          qb[kk][nh][1] = pack2<false>(hi[2], hi[3]);
-          qlo[kk][nh][0] = pack2<false>(lo[0], lo[1]);
-          qlo[kk][nh][1] = pack2<false>(lo[2], lo[3]);
+    for (int kk = 0; kk < D / 32; ++kk)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[i] = x[kk][h][i] * up;  // exact
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          float r[4];
+          const uint32_t c01 = e4m3x2_round(y[0], y[1], r[0], r[1]);
+          const uint32_t c23 = e4m3x2_round(y[2], y[3], r[2], r[3]);
+          qf[j][kk][nh][h] = c01 | (c23 << 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) y[i] -= r[i];  // exact: what the terms so far leave
         }
       }
+    // the accumulator's columns 2t, 2t + 1 are the rows of threads (2t, *) and
+    // (2t + 1, *)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int ec = __shfl_sync(0xffffffffu, e, (2 * t + c) * 4);
+      sl2[nh][c] = scale_log2 * __uint_as_float(static_cast<uint32_t>(127 - ec) << 23);
     }
   }
 }
@@ -241,30 +318,29 @@ __device__ __forceinline__ int2 accumulator_channels(int mt, int g) {
   return make_int2((D / 8) * g + 2 * mt, (D / 8) * g + 2 * mt + 1);
 }
 
-// One 16-token tile of K and V in shared memory (rows < nskip or >= nvalid
-// are zero and masked; FULL: all 16 rows count) against the warp's query
-// columns: S^T = K Q^T, online softmax update of the per-column running max /
-// sum (log2 domain), O^T += V^T P^T.
+// One 16-token tile of K and V of a 16-bit cache in shared memory (rows <
+// nskip or >= nvalid are zero and masked; FULL: all 16 rows count) against
+// the warp's query columns: S^T = K Q^T, online softmax update of the
+// per-column running max / sum (log2 domain), O^T += V^T P^T.
 template <int CK, int D, int NH, bool FULL>
 __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nvalid, int nskip,
                                             float scale_log2,
                                             const uint32_t (&qb)[D / 16][NH][2],
-                                            const uint32_t (&qlo)[CK == kE4M3 ? D / 16 : 1][NH][2],
                                             float (&o)[D / 16][NH][4], float (&m_run)[NH][2],
                                             float (&l_run)[NH][2]) {
+  static_assert(CK != kE4M3, "E4M3 tiles: attend_tile_e4m3");
   using G = TileGeom<CK, D>;
-  constexpr bool kMmaBF16 = (CK == kBF16);  // MMA operand type (E4M3 widens to f16)
+  constexpr bool kMmaBF16 = (CK == kBF16);  // MMA operand type
   constexpr int KSTEPS = D / 16;
   constexpr int MT = D / 16;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
-  const int t = lane & 3;
 
   // S^T = K Q^T: s[nh] = {(token g, columns 2t, 2t+1), (token g+8, same)}
   float s[NH][4];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
-  if constexpr (CK != kE4M3) {
+  {
     const int mi = lane >> 3;
     const int tok = (lane & 7) + 8 * (mi & 1);
     const int chk = mi >> 1;
@@ -274,26 +350,6 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
       ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(tok, 2 * kk + chk));
 #pragma unroll
       for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(s[nh], a, qb[kk][nh][0], qb[kk][nh][1]);
-    }
-  } else {
-#pragma unroll
-    for (int gq = 0; gq < D / 32; ++gq) {
-      const int c = 2 * gq + (t >> 1);
-      const int bo = (t & 1) * 8;
-      const uint2 wl = lds64(sk_a + G::off(g, c) + bo);      // token g
-      const uint2 wh = lds64(sk_a + G::off(g + 8, c) + bo);  // token g + 8
-      uint32_t a0[4], a1[4];
-      e4m3x4_to_f16x2x2(wl.x, a0[0], a0[2]);
-      e4m3x4_to_f16x2x2(wh.x, a0[1], a0[3]);
-      e4m3x4_to_f16x2x2(wl.y, a1[0], a1[2]);
-      e4m3x4_to_f16x2x2(wh.y, a1[1], a1[3]);
-#pragma unroll
-      for (int nh = 0; nh < NH; ++nh) {
-        mma_16816<false>(s[nh], a0, qb[2 * gq][nh][0], qb[2 * gq][nh][1]);
-        mma_16816<false>(s[nh], a0, qlo[2 * gq][nh][0], qlo[2 * gq][nh][1]);
-        mma_16816<false>(s[nh], a1, qb[2 * gq + 1][nh][0], qb[2 * gq + 1][nh][1]);
-        mma_16816<false>(s[nh], a1, qlo[2 * gq + 1][nh][0], qlo[2 * gq + 1][nh][1]);
-      }
     }
   }
 
@@ -345,7 +401,7 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
   }
 
   // O^T += V^T P^T
-  if constexpr (CK != kE4M3) {
+  {
     const int mi = lane >> 3;
     const int tok = (lane & 7) + 8 * (mi >> 1);
     const int chk = mi & 1;
@@ -356,16 +412,125 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
 #pragma unroll
       for (int nh = 0; nh < NH; ++nh) mma_16816<kMmaBF16>(o[mt][nh], a, pb[nh][0], pb[nh][1]);
     }
-  } else {
-    // Row m of O^T block mt is channel DPT*g + 2*mt (m = g) or that + 1
-    // (m = g + 8): this thread reads channels [DPT*g, DPT*g + DPT) of token
-    // rows 2t, 2t+1, 2t+8, 2t+9 and pairs tokens with byte permutes.
-    constexpr int DPT = D / 8;
-    constexpr int WORDS = DPT / 4;
+  }
+}
+
+// One 32-token tile of K and V of an E4M3 cache (rows < nskip or >= nvalid
+// are zero and masked; FULL: all 32 rows count). S^T for the two 16-token
+// row blocks mt = 0, 1 on E4M3 MMAs, s[mt][nh] = {(token 16mt + g, columns
+// 2t, 2t+1), (token 16mt + g + 8, same)}, summed over the query's three terms;
+// one online-softmax update over the 32 tokens (sl2: the per-column log2
+// scale that also undoes the query's power-of-two scaling); then
+// O^T += V^T P^T per 16-token block with V widened to f16.
+template <int D, int NH, bool FULL>
+__device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, int nvalid,
+                                                 int nskip, const float (&sl2)[NH][2],
+                                                 const uint32_t (&qf)[3][D / 32][NH][2],
+                                                 float (&o)[D / 16][NH][4], float (&m_run)[NH][2],
+                                                 float (&l_run)[NH][2]) {
+  using G = TileGeom<kE4M3, D, 32>;
+  constexpr int MT = D / 16;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+
+  float s[2][NH][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) s[mt][nh][0] = s[mt][nh][1] = s[mt][nh][2] = s[mt][nh][3] = 0.f;
+  {
+    // A fragments of 16 tokens x 32 channels straight from the tile (bytes
+    // 4t.. of rows g, g + 8, then bytes 16 + 4t..): ldmatrix's b16 layout
+    const int mi = lane >> 3;
+    const int tok = (lane & 7) + 8 * (mi & 1);
+    const int chk = mi >> 1;
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(16 * mt + tok, 2 * kk + chk));
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+          for (int j = 2; j >= 0; --j)  // smallest term first
+            mma_16832_e4m3(s[mt][nh], a, qf[j][kk][nh][0], qf[j][kk][nh][1]);
+      }
+  }
+
+  // rows g, g + 8, g + 16, g + 24 of the tile
+  bool v[2][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = 16 * mt + 8 * hh + g;
+      v[mt][hh] = FULL || (r < nvalid && r >= nskip);
+    }
+  uint32_t pb[2][NH][2];
+  bool grew = false;
+  float alpha[NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    float pr[2][2][2];  // [mt][row half][column e]
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float mx = fmaxf(fmaxf(v[0][0] ? s[0][nh][e] : -INFINITY, v[0][1] ? s[0][nh][2 + e] : -INFINITY),
+                       fmaxf(v[1][0] ? s[1][nh][e] : -INFINITY, v[1][1] ? s[1][nh][2 + e] : -INFINITY));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float sc = sl2[nh][e];
+      mx *= sc;
+      // mx is finite (some row of the tile exists), so the first tile always
+      // sets the reference
+      const bool up = mx > m_run[nh][e] + kRescaleLog2;
+      grew |= up;
+      const float m_ref = up ? mx : m_run[nh][e];
+      alpha[nh][e] = up ? ex2(m_run[nh][e] - m_ref) : 1.f;
+      float sum = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float pv = ex2(fmaf(s[mt][nh][2 * hh + e], sc, -m_ref));
+          pr[mt][hh][e] = v[mt][hh] ? pv : 0.f;
+          sum += pr[mt][hh][e];
+        }
+      l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + sum;
+      m_run[nh][e] = m_ref;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      pb[mt][nh][0] = movmatrix_trans(pack2<false>(pr[mt][0][0], pr[mt][0][1]));
+      pb[mt][nh][1] = movmatrix_trans(pack2<false>(pr[mt][1][0], pr[mt][1][1]));
+    }
+  }
+  if (__any_sync(0xffffffffu, grew)) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        o[mt][nh][0] *= alpha[nh][0];
+        o[mt][nh][1] *= alpha[nh][1];
+        o[mt][nh][2] *= alpha[nh][0];
+        o[mt][nh][3] *= alpha[nh][1];
+      }
+  }
+
+  // O^T += V^T P^T, one 16-token block at a time. Row m of O^T block mt is
+  // channel DPT*g + 2*mt (m = g) or that + 1 (m = g + 8): this thread reads
+  // channels [DPT*g, DPT*g + DPT) of token rows 2t, 2t+1, 2t+8, 2t+9 of the
+  // block and pairs tokens with byte permutes.
+  constexpr int DPT = D / 8;
+  constexpr int WORDS = DPT / 4;
+#pragma unroll
+  for (int kb = 0; kb < 2; ++kb) {
     uint32_t ra[4][WORDS];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
-      const int r = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
+      const int r = 16 * kb + 2 * t + (q4 & 1) + 8 * (q4 >> 1);
       const int byte0 = DPT * g;
       const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
       if constexpr (WORDS == 4) {
@@ -391,8 +556,8 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
       const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
 #pragma unroll
       for (int nh = 0; nh < NH; ++nh) {
-        mma_16816<false>(o[2 * w][nh], a0, pb[nh][0], pb[nh][1]);
-        mma_16816<false>(o[2 * w + 1][nh], a1, pb[nh][0], pb[nh][1]);
+        mma_16816<false>(o[2 * w][nh], a0, pb[kb][nh][0], pb[kb][nh][1]);
+        mma_16816<false>(o[2 * w + 1][nh], a1, pb[kb][nh][0], pb[kb][nh][1]);
       }
     }
   }
@@ -407,12 +572,14 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED = false>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part, const int by,
                                            const int b) {
-  using G = TileGeom<CK, D>;
   using S = DecodeSmem<CK, D, NW, NSTAGE>;
-  constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T
+  using G = typename S::G;
+  constexpr bool kE4 = (CK == kE4M3);
+  constexpr int TOK = G::TOKENS;            // tokens per tile (16, or 32 for E4M3)
+  constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T (16-bit)
   constexpr int MT = D / 16;                // 16-channel row blocks of O^T
   constexpr int RPI = 32 / G::CPR;          // tile rows one load instruction covers
-  constexpr int LITERS = 16 / RPI;          // load instructions per lane per tile and tensor
+  constexpr int LITERS = TOK / RPI;         // load instructions per lane per tile and tensor
 
   extern __shared__ __align__(128) uint8_t smem[];
   int* s_bt = reinterpret_cast<int*>(smem + S::kMainBytes);
@@ -456,7 +623,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const int lo = span.lo;  // first attended token
   const int t0 = span.base + part * PT;
   const int t1 = min(t0 + PT, L);
-  const int ntiles = (t1 - t0 + 15) >> 4;
+  const int ntiles = (t1 - t0 + TOK - 1) / TOK;
 
   // ---- block ids of this partition -> shared memory ----------------------
   // (up to kBlockIdsInSmem of them; a longer slice is read from global
@@ -480,15 +647,19 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   // ---- Q^T fragments (B operand: k = channel, n = query head) -------------
   const TQ* qbase = reinterpret_cast<const TQ*>(p.q) +
                     (static_cast<int64_t>(b) * p.num_q_heads + hq0) * D;
-  uint32_t qb[KSTEPS][NH][2];
-  uint32_t qlo[CK == kE4M3 ? KSTEPS : 1][NH][2];
+  uint32_t qb[kE4 ? 1 : KSTEPS][NH][2];         // 16-bit caches
+  uint32_t qf[kE4 ? 3 : 1][kE4 ? D / 32 : 1][NH][2];  // E4M3: three query terms
+  float sl2[NH][2];                              // E4M3: per-column log2 scale
   {
     const TQ* rows[NH];
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
       rows[nh] = 8 * nh + g < nrows ? qbase + (8 * nh + g) * D : nullptr;
-    load_query_fragments<TQ, CK, D, NH>(
-        rows, CK == kE4M3 ? p.k_scale + static_cast<int64_t>(hk) * D : nullptr, qb, qlo);
+    if constexpr (kE4)
+      load_query_e4m3<TQ, D, NH>(rows, p.k_scale + static_cast<int64_t>(hk) * D, p.scale_log2,
+                                 qf, sl2);
+    else
+      load_query_fragments<TQ, D, NH>(rows, qb);
   }
   __syncthreads();  // s_bt ready
 
@@ -498,7 +669,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const uint8_t* vc = reinterpret_cast<const uint8_t*>(p.v_cache);
   const int64_t slot_stride = static_cast<int64_t>(p.num_kv_heads) * G::RB;
   const int bs_mask = (1 << p.bs_log2) - 1;
-  const bool block_aligned = p.bs_log2 >= 4;  // a 16-token tile lies inside one block
+  // blocks of >= 16 tokens: each 16-row half of a tile lies inside one block
+  // (tiles start 16-aligned)
+  const bool block_aligned = p.bs_log2 >= 4;
   // this lane's load slots: rows lrow + i*RPI, 16-byte chunk lch
   const int lrow = lane / G::CPR;
   const int lch = lane % G::CPR;
@@ -520,6 +693,24 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const int64_t new_row = (static_cast<int64_t>(b) * p.num_kv_heads + hk) * D;  // elements
   const TQ* knew = has_new ? reinterpret_cast<const TQ*>(p.k_new) + new_row : nullptr;
   const TQ* vnew = has_new ? reinterpret_cast<const TQ*>(p.v_new) + new_row : nullptr;
+  // E4M3: the new token's rows, quantised once (e4m3_rn_satfinite(x *
+  // inv_scale), as pa_append_kv does) into shared memory, for the tile that
+  // holds the token and for the store at the end
+  const uint32_t s_new =
+      smem_addr(smem) + S::new_rows_offset(staged_block_ids(p.partition_tokens, p.bs_log2));
+  if constexpr (FUSED && kE4) {
+    if (has_new && jnew >= max(t0, lo) && jnew < t1 && threadIdx.x < 2 * G::CPR) {
+      const bool is_v = threadIdx.x >= G::CPR;
+      const int ch = threadIdx.x - (is_v ? G::CPR : 0);
+      const uint4 qv = quantize16<TQ>((is_v ? vnew : knew) + 16 * ch,
+                                      (is_v ? p.v_inv_scale : p.k_inv_scale) + hk * D + 16 * ch);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                       s_new + (is_v ? G::RB : 0) + 16 * ch),
+                   "r"(qv.x), "r"(qv.y), "r"(qv.z), "r"(qv.w)
+                   : "memory");
+    }
+    __syncthreads();
+  }
   // Store the new token in the cache, as pa_append_kv would; the slot must
   // be the one the table gives position L - 1. Done by the CTA of the last
   // partition (first head group); nothing in this launch reads the slot.
@@ -541,63 +732,62 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
                      (slot * p.num_kv_heads + hk) * G::RB + ch * 16;
       const TQ* src = is_v ? vnew : knew;
       if constexpr (CK == kE4M3) {
-        const float* inv = (is_v ? p.v_inv_scale : p.k_inv_scale) + hk * D + 16 * ch;
-        *reinterpret_cast<uint4*>(dst) = quantize16<TQ>(src + 16 * ch, inv);
+        *reinterpret_cast<uint4*>(dst) = lds128(s_new + (is_v ? G::RB : 0) + 16 * ch);
       } else {
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src + 8 * ch);
       }
     }
   };
-  // a 16-bit row is a plain copy: done up front; the E4M3 quantisation is
-  // done at the end of the CTA, where it adds no register pressure to the loop
+  // a 16-bit row is a plain copy: done up front; the E4M3 row is stored at
+  // the end of the CTA, from the quantised copy in shared memory
   if constexpr (FUSED && CK != kE4M3) store_new_token();
 
   // One 16-byte chunk of row r: from the cache at `off`, or from the fused
-  // new token (16-bit: the same bytes by cp.async; E4M3: no copy here, the
-  // tile's new-token fix-up below stores the quantised row).
+  // new token (16-bit: the same bytes by cp.async; E4M3: the quantised row
+  // from shared memory).
   auto load_chunk = [&](uint32_t sk_a, uint32_t sv_a, int r, int j, bool ok, int64_t off) {
     const uint32_t so = G::off(r, lch);
     if (FUSED && j == jnew) {
       if constexpr (CK != kE4M3) {
         cp_async_16(sk_a + so, knew + 8 * lch, 16u);
         cp_async_16(sv_a + so, vnew + 8 * lch, 16u);
+      } else {
+        const uint4 kq = lds128(s_new + 16 * lch);
+        const uint4 vq = lds128(s_new + G::RB + 16 * lch);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sk_a + so), "r"(kq.x),
+                     "r"(kq.y), "r"(kq.z), "r"(kq.w)
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(sv_a + so), "r"(vq.x),
+                     "r"(vq.y), "r"(vq.z), "r"(vq.w)
+                     : "memory");
       }
       return;
     }
     cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
     cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
   };
-  // E4M3 fused: the new token's row of the tile starting at tb, quantised
-  // once per tile by lanes 0 .. 2*CPR-1 (K chunks, then V chunks).
-  auto store_new_row = [&](uint32_t sk_a, uint32_t sv_a, int tb) {
-    if constexpr (FUSED && CK == kE4M3) {
-      if (jnew >= tb && jnew < tb + 16 && lane < 2 * G::CPR) {
-        const bool is_v = lane >= G::CPR;
-        const int ch = lane - (is_v ? G::CPR : 0);
-        const uint4 qv = quantize16<TQ>((is_v ? vnew : knew) + 16 * ch,
-                                        (is_v ? p.v_inv_scale : p.k_inv_scale) + hk * D + 16 * ch);
-        const uint32_t a = (is_v ? sv_a : sk_a) + G::off(jnew - tb, ch);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(qv.x),
-                     "r"(qv.y), "r"(qv.z), "r"(qv.w));
-      }
-    }
-  };
-
   auto load_tile = [&](int tile, int stage) {
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
-    const int tb = t0 + tile * 16;
+    const int tb = t0 + tile * TOK;
     if (block_aligned) {
-      const int blk = block_id((tb >> p.bs_log2) - bt0);
-      const int64_t base =
-          ((static_cast<int64_t>(blk) << p.bs_log2) + (tb & bs_mask) + lrow) * slot_stride +
-          lane_goff;
+      constexpr int IPH = LITERS / (TOK / 16);  // load instructions per 16-row half
 #pragma unroll
-      for (int i = 0; i < LITERS; ++i) {
-        const int r = lrow + i * RPI;
-        const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
-        const int64_t off = ok ? base + static_cast<int64_t>(i * RPI) * slot_stride : 0;
-        load_chunk(sk_a, sv_a, r, tb + r, ok, off);
+      for (int h = 0; h < TOK / 16; ++h) {
+        // a half that starts past the partition's end is not looked up (its
+        // block id need not be staged)
+        const int th = tb + 16 * h;
+        const int blk = th < t1 ? block_id((th >> p.bs_log2) - bt0) : -1;
+        const int64_t base =
+            ((static_cast<int64_t>(blk) << p.bs_log2) + (th & bs_mask) + lrow) * slot_stride +
+            lane_goff;
+#pragma unroll
+        for (int ii = 0; ii < IPH; ++ii) {
+          const int r = 16 * h + lrow + ii * RPI;
+          const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
+          const int64_t off = ok ? base + static_cast<int64_t>(ii * RPI) * slot_stride : 0;
+          load_chunk(sk_a, sv_a, r, tb + r, ok, off);
+        }
       }
     } else {
 #pragma unroll
@@ -613,7 +803,6 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
         load_chunk(sk_a, sv_a, r, j, ok, off);
       }
     }
-    store_new_row(sk_a, sv_a, tb);
   };
 
   float o[MT][NH][4];
@@ -648,15 +837,21 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
     const int tile = warp + it * NW;
-    const int ts = t0 + tile * 16;
+    const int ts = t0 + tile * TOK;
     const int nvalid = t1 - ts;                // rows of the tile below the end (>= 1)
     const int nskip = max(lo - ts, 0);         // rows before the window (first tile only)
-    if (nvalid >= 16 && nskip == 0)
-      attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, 0, p.scale_log2, qb, qlo, o, m_run,
-                                   l_run);
-    else
-      attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, nskip, p.scale_log2, qb, qlo, o, m_run,
-                                    l_run);
+    if constexpr (kE4) {
+      if (nvalid >= TOK && nskip == 0)
+        attend_tile_e4m3<D, NH, true>(sk_a, sv_a, nvalid, 0, sl2, qf, o, m_run, l_run);
+      else
+        attend_tile_e4m3<D, NH, false>(sk_a, sv_a, nvalid, nskip, sl2, qf, o, m_run, l_run);
+    } else {
+      if (nvalid >= TOK && nskip == 0)
+        attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, 0, p.scale_log2, qb, o, m_run, l_run);
+      else
+        attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, nskip, p.scale_log2, qb, o, m_run,
+                                      l_run);
+    }
     __syncwarp();  // this stage is reloaded by the next iteration
   }
   cp_async_wait<0>();

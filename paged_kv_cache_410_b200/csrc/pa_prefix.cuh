@@ -43,9 +43,10 @@ __host__ __device__ constexpr int prefix_subtiles() {
 }
 
 // A fragments of 16 query rows: qa[kk] = {row g | row g+8} x {k-slots 2t,2t+1 |
-// 2t+8,2t+9}. E4M3: q' = q * k_scale as f16 hi + lo, with the channel order of
-// load_query_fragments (k-step 2gq + h holds channels 8t + 4h + {0,1} in
-// slots 2t, 2t+1 and 8t + 4h + {2,3} in slots 2t+8, 2t+9).
+// 2t+8,2t+9}. E4M3: q' = q * k_scale as f16 hi + lo, with channels permuted
+// within each 32-channel group gq so that a thread's K codes are contiguous:
+// k-step 2gq + h holds channels 8t + 4h + {0,1} in slots 2t, 2t+1 and
+// 8t + 4h + {2,3} in slots 2t+8, 2t+9.
 template <typename TQ, int CK, int D>
 __device__ __forceinline__ void load_query_rows(const TQ* row_g, const TQ* row_g8,
                                                 const float* k_scale_row,

@@ -172,8 +172,52 @@ def test_workspace_plan(lib):
     assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(_desc(num_kv_heads=32))) == 1024
     d8 = _desc(num_kv_heads=8, head_dim=128, cache_dtype=B.PA_E4M3)
     assert lib.pa_decode_partition_tokens(256, 8192, ctypes.byref(d8)) == 1024
-    assert lib.pa_decode_partition_tokens(1, 4096, ctypes.byref(d)) == 64
+    # (8 rows: halved to 64 tokens = 512 CTAs, then one whole wave of 444:
+    # 80-token partitions, 416 CTAs)
+    assert lib.pa_decode_partition_tokens(1, 4096, ctypes.byref(d)) == 80
     assert lib.pa_decode_partition_tokens(1, 100, ctypes.byref(d)) == 64
+
+
+def test_small_batches_split_into_whole_waves(lib):
+    """With fewer (sequence, KV head) pairs than one wave of decode CTAs (3 per
+    SM on 148 SMs), the automatic partition is lengthened to the shortest
+    multiple of 16 tokens whose CTAs fill whole waves."""
+    waves_of = 3 * 148
+    d = _desc(num_kv_heads=8, head_dim=128, cache_dtype=B.PA_BF16)
+    for batch, ctx, want in ((1, 131072, 592), (4, 131072, 528), (2, 20000, 752)):
+        pt = lib.pa_decode_partition_tokens(batch, ctx, ctypes.byref(d))
+        assert pt == want, (batch, ctx, pt)
+        ctas = batch * 8 * -(-ctx // pt)
+        full = batch * 8 * -(-ctx // 512) // waves_of  # whole waves of the 512-token plan
+        assert ctas <= full * waves_of and pt % 16 == 0
+        # 16 tokens shorter would need one more (partial) wave
+        assert batch * 8 * -(-ctx // (pt - 16)) > full * waves_of
+    # a batch that fills the GPU by itself keeps the byte rule
+    d32 = _desc(num_kv_heads=32, head_dim=128)
+    assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(d32)) == 512
+    assert lib.pa_decode_partition_tokens(14, 8192, ctypes.byref(d32)) == 512  # 448 rows
+
+
+def test_static_workspace_checks_arguments_before_its_size_rule(lib):
+    """The no-allocation decode reports an invalid call exactly as pa_decode
+    does, even when the plan of the call would also exceed its fixed array;
+    only a valid call whose plan needs more than the array gets
+    PA_ERR_WORKSPACE."""
+    d = _desc(num_kv_heads=8, head_dim=128)
+    order = [("q", FAKE), ("q_dtype", 0), ("batch", 8), ("hq", 64), ("k", FAKE), ("v", FAKE),
+             ("desc", ctypes.byref(d)), ("bt", FAKE), ("mb", 8192), ("lens", FAKE),
+             ("maxc", 131072), ("scale", 0.1), ("out", FAKE), ("pt", 0)]
+    static = lambda **kw: lib.pa_decode_static_workspace(
+        *[kw.get(k, v) for k, v in order], None)
+    plain = lambda **kw: lib.pa_decode(*[kw.get(k, v) for k, v in order], None, 0, None)
+    # 8 sequences x 64 heads x 249 partitions of 528 tokens: 66 MB of partials
+    assert lib.pa_decode_workspace_size(8, 64, 131072, 0, ctypes.byref(d)) > 32 << 20
+    for bad, status in ((dict(pt=17), 1), (dict(hq=60), 1), (dict(q=None), 1),
+                        (dict(out=FAKE + 8), 1), (dict(scale=float("inf")), 1),
+                        (dict(q_dtype=1), 2), (dict(mb=0), 1), (dict(batch=0), 0)):
+        assert static(**bad) == status, bad
+        assert plain(**bad) == status, bad
+    assert static() == 4                      # valid, but the plan needs more than 32 MiB
 
 
 def test_append_decode_argument_checks(lib):
@@ -221,9 +265,10 @@ def test_shared_prefix_partition_rule(lib):
     d = _desc(num_blocks=20000, num_kv_heads=8, head_dim=128, cache_dtype=B.PA_BF16)
     assert lib.pa_decode_partition_tokens(128, 2049, ctypes.byref(d)) == 512
     assert lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 125, ctypes.byref(d)) == 2048
-    # 16 sequences: doubling once keeps >= 2 CTAs per SM (16 x 8 x 3 = 384), twice does not
-    assert lib.pa_decode_partition_tokens(16, 2049, ctypes.byref(d)) == 512
-    assert lib.pa_decode_shared_prefix_partition_tokens(16, 64, 4049, 125, ctypes.byref(d)) == 1024
+    # 16 sequences (128 rows, under one wave): one whole wave of 688-token
+    # partitions (384 CTAs); doubling that would leave < 2 CTAs per SM
+    assert lib.pa_decode_partition_tokens(16, 2049, ctypes.byref(d)) == 688
+    assert lib.pa_decode_shared_prefix_partition_tokens(16, 64, 4049, 125, ctypes.byref(d)) == 688
     assert (lib.pa_decode_shared_prefix_partition_tokens(128, 64, 4049, 0, ctypes.byref(d)) ==
             lib.pa_decode_partition_tokens(128, 4049, ctypes.byref(d)))
     # a small batch keeps the plain rule (doubling would leave < 2 CTAs per SM)
@@ -299,7 +344,7 @@ def test_headers_are_plain_c_and_the_library_links_from_c(lib, tmp_path):
     assert int(f[0]) == lib.pa_version()
     assert f[1] == "workspace missing or too small"
     assert int(f[2]) == lib.pa_decode_workspace_size(4, 64, 131072, 0, ctypes.byref(d)) > 0
-    assert int(f[3]) == lib.pa_decode_partition_tokens(4, 131072, ctypes.byref(d)) == 512
+    assert int(f[3]) == lib.pa_decode_partition_tokens(4, 131072, ctypes.byref(d)) == 528
     assert int(f[4]) == 1                         # PA_ERR_INVALID_ARG
     assert int(f[5]) == 0                         # every block-manager call succeeded
     assert int(f[6]) == 32                        # two full 16-token blocks reused
