@@ -14,6 +14,7 @@
 #include <mutex>
 #include <unordered_map>
 #include <unordered_set>
+#include <utility>
 
 #include "pa_api.h"
 #include "pa_append_copy.cuh"
@@ -156,27 +157,53 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
   return e;
 }
 
-// Split-K merge: 1, 2, 4 or 8 warps per (sequence, query head) row by the
-// number of partials per row.
+// Launch `kern` as the programmatic dependent of the kernel before it in
+// `st`: it may start once every CTA of that kernel has started (or exited),
+// and waits (griddepcontrol.wait) before reading that kernel's results.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Split-K merge, the decode kernel's programmatic dependent: 1, 2, 4, 8, 16
+// or 32 warps per (sequence, query head) row by the number of partials per
+// row (a row of 16 or 32 warps is a CTA of its own).
 template <typename TQ, int D>
 pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
-  auto go = [&](auto kern, int rows_per_cta) {
+  auto go = [&](auto kern, int warps, int rows_per_cta) {
     const int64_t ctas = (rows + rows_per_cta - 1) / rows_per_cta;
-    kern<<<static_cast<unsigned>(ctas), pa::kReduceWarps * 32, 0, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_dependent(kern, dim3(static_cast<unsigned>(ctas)), dim3(warps * 32), 0, st, p) ==
+                   cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
   };
-  if (p.num_partitions <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1>, 8);
-  if (p.num_partitions <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2>, 4);
-  if (p.num_partitions <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4>, 2);
-  return go(pa::pa_decode_reduce_kernel<TQ, D, 8>, 1);
+  // one warp per row: 32 rows per CTA, so that a large batch's merge is a few
+  // hundred CTAs that all start at once
+  if (p.num_partitions <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32>, 32, 32);
+  if (p.num_partitions <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32>, 32, 32);
+  if (p.num_partitions <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2, 16, 8>, 8, 4);
+  if (p.num_partitions <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 16, 8>, 8, 2);
+  if (p.num_partitions <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16>, 16, 1);
+  return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 16, 32>, 32, 1);
 }
 
 // Decode kernel over `grid_x` partition columns, then the split-K merge when
 // the plan has more than one partial per sequence (or always, in cascade mode).
 template <typename TQ, int CK, int D, int NH>
 pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st,
-                          bool with_reduce = true) {
+                          bool with_reduce = true, bool dependent = false) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
                       : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
@@ -187,8 +214,13 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
   if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
   if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
   dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
-  kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  if (dependent) {
+    if (launch_dependent(kern, grid, dim3(kDecodeWarps * 32), smem, st, p) != cudaSuccess)
+      return PA_ERR_CUDA;
+  } else {
+    kern<<<grid, kDecodeWarps * 32, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
   if (with_reduce && (p.num_partitions > 1 || p.force_partials)) {
     const pa_status rs = launch_reduce<TQ, D>(p, st);
     if (rs != PA_OK) return rs;
@@ -198,14 +230,14 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
 
 template <typename TQ, int CK>
 pa_status launch_decode_d(const pa::DecodeParams& p, int head_dim, int grid_x,
-                          cudaStream_t st, bool with_reduce = true) {
+                          cudaStream_t st, bool with_reduce = true, bool dependent = false) {
   // query heads per CTA: the whole group up to 16; 8-head column blocks
   const bool two = std::min(p.group, 16) > 8;
   if (head_dim == 64)
-    return two ? launch_decode_t<TQ, CK, 64, 2>(p, grid_x, st, with_reduce)
-               : launch_decode_t<TQ, CK, 64, 1>(p, grid_x, st, with_reduce);
-  return two ? launch_decode_t<TQ, CK, 128, 2>(p, grid_x, st, with_reduce)
-             : launch_decode_t<TQ, CK, 128, 1>(p, grid_x, st, with_reduce);
+    return two ? launch_decode_t<TQ, CK, 64, 2>(p, grid_x, st, with_reduce, dependent)
+               : launch_decode_t<TQ, CK, 64, 1>(p, grid_x, st, with_reduce, dependent);
+  return two ? launch_decode_t<TQ, CK, 128, 2>(p, grid_x, st, with_reduce, dependent)
+             : launch_decode_t<TQ, CK, 128, 1>(p, grid_x, st, with_reduce, dependent);
 }
 
 pa_status launch_decode(const pa::DecodeParams& p, int q_dtype, const pa_cache_desc* cache,
@@ -301,7 +333,8 @@ struct CascadePlan {
   int num_partitions;  // chunks + suffix partitions
   size_t ws_o_bytes;
   size_t ws_bytes;
-  bool fits;  // as Plan::fits
+  bool longest_first;  // the suffix decode visits the sequences longest first
+  bool fits;           // as Plan::fits
 };
 
 // 16-bit caches with blocks of >= 8 tokens (whole 1024-byte swizzle atoms
@@ -417,6 +450,9 @@ CascadePlan make_cascade_plan(int64_t batch, int64_t num_q_heads, int64_t max_co
   pl.ws_bytes = pl.ws_o_bytes + round_up(static_cast<size_t>(batch * num_q_heads) *
                                              pl.num_partitions * sizeof(float2),
                                          256);
+  // the tensor-core path's suffix decode takes long partitions (up to four
+  // times the plain rule), so it visits the sequences longest first
+  pl.longest_first = cascade_uses_umma(cd, group) && batch > 1 && batch <= pa::kOrderMaxBatch;
   return pl;
 }
 
@@ -450,37 +486,13 @@ pa_status launch_cascade_t(const pa::DecodeParams& p, const CascadePlan& pl, cud
   return launch_reduce<TQ, D>(p, st);
 }
 
-// A side stream per device on which the prefix kernel runs next to the
-// suffix decode, with the events that fork it from and join it back to the
-// caller's stream. The mutex keeps each fork / join pair together when
-// several host threads call at once.
-struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join = nullptr;
-};
-std::mutex g_side_mu;
-SideStream g_side[64];
+std::mutex g_hook_mu;
 int g_withhold_prefix_scores = 0;  // pa_testing_withhold_prefix_scores
 
-cudaError_t side_stream(SideStream** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  SideStream& ss = g_side[dev & 63];
-  if (!ss.stream) {
-    if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
-      return e;
-  }
-  *out = &ss;
-  return cudaSuccess;
-}
-
-// 16-bit caches: the tcgen05 prefix kernel on the side stream, concurrently
-// with the suffix decode (cascade mode) on the caller's stream; the merge
-// after both.
+// 16-bit caches: the tcgen05 prefix kernel, then the suffix decode (cascade
+// mode) as its programmatic dependent, so that the two run side by side
+// (every prefix CTA lets it start at once; the suffix grid finishes only
+// after the prefix grid), then the merge as the suffix decode's dependent.
 template <typename TQ, int CK, int D>
 pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl,
                                 cudaStream_t st) {
@@ -529,20 +541,16 @@ pa_status launch_cascade_umma_t(const pa::DecodeParams& p, const CascadePlan& pl
     return PA_ERR_CUDA;
   const int64_t ctas = static_cast<int64_t>(ug.n_chunks) * ug.n_rowtiles * p.num_kv_heads;
   if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  ug.withhold_scores = g_withhold_prefix_scores;  // written under the same lock
-  SideStream* ss = nullptr;
-  if (side_stream(&ss) != cudaSuccess) return PA_ERR_CUDA;
-  if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
-      cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
-    return PA_ERR_CUDA;
-  kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kRequest, ss->stream>>>(p, ug, tq, tk, tv,
-                                                                             to);
+  {
+    std::lock_guard<std::mutex> lock(g_hook_mu);
+    ug.withhold_scores = g_withhold_prefix_scores;
+  }
+  kern<<<static_cast<unsigned>(ctas), C::kThreads, C::kRequest, st>>>(p, ug, tq, tk, tv, to);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return PA_ERR_CUDA;
-  const pa_status rs = launch_decode_d<TQ, CK>(p, D, std::max(pl.suffix_partitions, 1), st,
-                                               /*with_reduce=*/false);
-  if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return PA_ERR_CUDA;
+  pa::DecodeParams ps = p;  // the suffix decode, longest sequences first
+  ps.longest_first = pl.longest_first ? 1 : 0;
+  const pa_status rs = launch_decode_d<TQ, CK>(ps, D, std::max(pl.suffix_partitions, 1), st,
+                                               /*with_reduce=*/false, /*dependent=*/true);
   if (rs != PA_OK) return rs;
   return launch_reduce<TQ, D>(p, st);
 }
@@ -585,7 +593,7 @@ const char* pa_status_string(int32_t s) {
 int32_t pa_version(void) { return 100; }
 
 void pa_testing_withhold_prefix_scores(int32_t on) {
-  std::lock_guard<std::mutex> lock(g_side_mu);
+  std::lock_guard<std::mutex> lock(g_hook_mu);
   g_withhold_prefix_scores = on != 0;
 }
 

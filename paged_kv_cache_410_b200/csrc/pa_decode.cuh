@@ -86,7 +86,15 @@ struct DecodeParams {
   const int64_t* slot_mapping;
   const float* k_inv_scale;  // E4M3 caches
   const float* v_inv_scale;
+  // Nonzero: the grid's z index visits the sequences longest first (by
+  // attended length after token_start; ties by index) instead of in order.
+  // Blocks are dispatched in index order, so this keeps the longest CTAs out
+  // of the launch's tail. Each CTA ranks the batch itself (batch <=
+  // kOrderMaxBatch).
+  int longest_first;
 };
+
+constexpr int kOrderMaxBatch = 256;
 
 // 16 consecutive channels of a 16-bit input row -> 16 E4M3 codes, each
 // e4m3_rn_satfinite(fp32(x) * inv_scale) (the append kernel's rounding).
@@ -415,28 +423,29 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
   }
 }
 
-// One 32-token tile of K and V of an E4M3 cache (rows < nskip or >= nvalid
-// are zero and masked; FULL: all 32 rows count). S^T for the two 16-token
-// row blocks mt = 0, 1 on E4M3 MMAs, s[mt][nh] = {(token 16mt + g, columns
-// 2t, 2t+1), (token 16mt + g + 8, same)}, summed over the query's three terms;
-// one online-softmax update over the 32 tokens (sl2: the per-column log2
-// scale that also undoes the query's power-of-two scaling); then
-// O^T += V^T P^T per 16-token block with V widened to f16.
+// One tile of K and V of an E4M3 cache (rows < nskip or >= nvalid are zero
+// and masked; FULL: all rows count). S^T for each 16-token row block mt on
+// E4M3 MMAs, s[mt][nh] = {(token 16mt + g, columns 2t, 2t+1), (token
+// 16mt + g + 8, same)}, summed over the query's three terms; one online-
+// softmax update over the tile (sl2: the per-column log2 scale that also
+// undoes the query's power-of-two scaling); then O^T += V^T P^T per 16-token
+// block with V widened to f16.
 template <int D, int NH, bool FULL>
 __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, int nvalid,
                                                  int nskip, const float (&sl2)[NH][2],
                                                  const uint32_t (&qf)[3][D / 32][NH][2],
                                                  float (&o)[D / 16][NH][4], float (&m_run)[NH][2],
                                                  float (&l_run)[NH][2]) {
-  using G = TileGeom<kE4M3, D, 32>;
+  using G = TileGeom<kE4M3, D, decode_tile_tokens<kE4M3>()>;
+  constexpr int MB = G::TOKENS / 16;  // 16-token row blocks of the tile
   constexpr int MT = D / 16;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
   const int t = lane & 3;
 
-  float s[2][NH][4];
+  float s[MB][NH][4];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int mt = 0; mt < MB; ++mt)
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh) s[mt][nh][0] = s[mt][nh][1] = s[mt][nh][2] = s[mt][nh][3] = 0.f;
   {
@@ -448,7 +457,7 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
 #pragma unroll
     for (int kk = 0; kk < D / 32; ++kk)
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
+      for (int mt = 0; mt < MB; ++mt) {
         uint32_t a[4];
         ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(16 * mt + tok, 2 * kk + chk));
 #pragma unroll
@@ -459,25 +468,28 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
       }
   }
 
-  // rows g, g + 8, g + 16, g + 24 of the tile
-  bool v[2][2];
+  // rows g, g + 8 (, g + 16, g + 24) of the tile
+  bool v[MB][2];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int mt = 0; mt < MB; ++mt)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int r = 16 * mt + 8 * hh + g;
       v[mt][hh] = FULL || (r < nvalid && r >= nskip);
     }
-  uint32_t pb[2][NH][2];
+  uint32_t pb[MB][NH][2];
   bool grew = false;
   float alpha[NH][2];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) {
-    float pr[2][2][2];  // [mt][row half][column e]
+    float pr[MB][2][2];  // [mt][row half][column e]
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      float mx = fmaxf(fmaxf(v[0][0] ? s[0][nh][e] : -INFINITY, v[0][1] ? s[0][nh][2 + e] : -INFINITY),
-                       fmaxf(v[1][0] ? s[1][nh][e] : -INFINITY, v[1][1] ? s[1][nh][2 + e] : -INFINITY));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int mt = 0; mt < MB; ++mt)
+        mx = fmaxf(mx, fmaxf(v[mt][0] ? s[mt][nh][e] : -INFINITY,
+                             v[mt][1] ? s[mt][nh][2 + e] : -INFINITY));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -491,7 +503,7 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
       alpha[nh][e] = up ? ex2(m_run[nh][e] - m_ref) : 1.f;
       float sum = 0.f;
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < MB; ++mt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const float pv = ex2(fmaf(s[mt][nh][2 * hh + e], sc, -m_ref));
@@ -502,7 +514,7 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
       m_run[nh][e] = m_ref;
     }
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < MB; ++mt) {
       pb[mt][nh][0] = movmatrix_trans(pack2<false>(pr[mt][0][0], pr[mt][0][1]));
       pb[mt][nh][1] = movmatrix_trans(pack2<false>(pr[mt][1][0], pr[mt][1][1]));
     }
@@ -526,7 +538,7 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
   constexpr int DPT = D / 8;
   constexpr int WORDS = DPT / 4;
 #pragma unroll
-  for (int kb = 0; kb < 2; ++kb) {
+  for (int kb = 0; kb < MB; ++kb) {
     uint32_t ra[4][WORDS];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
@@ -934,27 +946,56 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 // grid: (partitions, num_kv_heads * head_groups, batch)
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
 __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
-  decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, blockIdx.x, blockIdx.y, blockIdx.z);
+  // a kernel launched after this one as its programmatic dependent (the
+  // split-K merge) may start as soon as every CTA here has started; it waits
+  // for this grid's completion before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int b = static_cast<int>(blockIdx.z);
+  if (p.longest_first) {
+    // the sequence of rank z in decreasing attended length
+    __shared__ int s_key[kOrderMaxBatch];
+    __shared__ int s_pick;
+    for (int i = threadIdx.x; i < p.batch; i += NW * 32)
+      s_key[i] = max(clamp_context(p, p.context_lens[i]) - p.token_start, 0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < p.batch; i += NW * 32) {
+      const int ki = s_key[i];
+      int rank = 0;
+      for (int j = 0; j < p.batch; ++j) rank += (s_key[j] > ki) || (s_key[j] == ki && j < i);
+      if (rank == b) s_pick = i;
+    }
+    __syncthreads();
+    b = s_pick;
+  }
+  decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, blockIdx.x, blockIdx.y, b);
+  // cascade mode: the shared-prefix kernel runs before this one in the stream
+  // with this launch as its programmatic dependent, so this grid started
+  // early; it completes only after the prefix grid has, so that the merge,
+  // which waits for this grid, also sees the prefix partials
+  if (p.prefix_blocks > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
 // and normalised output o_p, out = sum_p w_p o_p / sum_p w_p where
 // w_p = l_p * 2^(m_p - max_p m_p).
 //
-// A CTA has kReduceWarps warps; WPR warps merge one (sequence, query head)
-// row, so a CTA covers kReduceWarps / WPR rows (the host picks WPR from the
-// number of partials: few partials, several rows per CTA; many partials,
-// several warps per row). Within a warp, lanes read 32 partials' (max, sum)
-// at a time for the global max, then the warp walks its share of the
-// partials: lane l owns channels 4l .. 4l+3 (float4 loads of the partial
-// outputs); the WPR warps' sums are added in shared memory.
-constexpr int kReduceWarps = 8;
-
-template <typename TQ, int D, int WPR>
-__global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(const DecodeParams p) {
+// A CTA has NWARPS warps; WPR warps merge one (sequence, query head) row, so
+// a CTA covers NWARPS / WPR rows (the host picks WPR from the number of
+// partials: few partials, several rows per CTA; many partials, up to 32
+// warps per row). Within a warp, lanes read 32 partials' (max, sum) at a
+// time for the global max, then the warp walks its share of the partials:
+// lane l owns channels 4l .. 4l+3 (float4 loads of the partial outputs); the
+// WPR warps' sums are added in shared memory. With one warp per row (at most
+// NL partials) every load is issued before any is used.
+//
+// The kernel is launched as the programmatic dependent of the kernels that
+// write the partials: it waits for them to complete before reading.
+template <typename TQ, int D, int WPR, int NL, int NWARPS>
+__global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const DecodeParams p) {
   static_assert(D % 4 == 0 && D <= 128, "one float4 per lane");
-  static_assert(kReduceWarps % WPR == 0, "whole rows per CTA");
-  constexpr int RPC = kReduceWarps / WPR;  // rows per CTA
+  static_assert(NWARPS % WPR == 0, "whole rows per CTA");
+  constexpr int RPC = NWARPS / WPR;  // rows per CTA
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int rloc = warp / WPR;
@@ -962,8 +1003,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
   const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + rloc;  // b * Hq + head
   const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
 
-  __shared__ float4 s_acc[kReduceWarps][D / 4];
-  __shared__ float s_wsum[kReduceWarps];
+  __shared__ float4 s_acc[NWARPS][D / 4];
+  __shared__ float s_wsum[NWARPS];
 
   int nparts = 0;
   if (row < rows) {
@@ -974,10 +1015,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
   const bool active = lane < D / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  if (WPR == 1) {
-    // at most 16 partials (the launch picks WPR = 1 only then): every load
-    // is issued before any is used, so a row costs one memory round trip
-    // after its length
+  if constexpr (WPR == 1) {
+    // at most NL partials (the launch picks WPR = 1 only then)
     if (work) {
       const float2* ml = p.ws_ml + row * p.num_partitions;
       const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
@@ -986,9 +1025,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
       // the row's D / 4 lanes; the clamped copies get weight 0 or are not
       // stored), so that they are all issued together
       const int lc = active ? lane : D / 4 - 1;
-      float4 x[16];
+      float4 x[NL];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < NL; ++i)
         x[i] = po[static_cast<int64_t>(min(i, nparts - 1)) * (D / 4) + lc];
       float M = mine.x;
 #pragma unroll
@@ -998,7 +1037,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pa_decode_reduce_kernel(con
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < NL; ++i) {
         const float w = __shfl_sync(0xffffffffu, wl, i);
         acc.x += w * x[i].x;
         acc.y += w * x[i].y;

@@ -27,7 +27,8 @@
 // one box per cache block of >= 8 tokens and 64-channel slab, no
 // multicast), one thread of an MMA warp issues the MMAs, and the partial
 // outputs leave through TMA stores; every wait on a copy or an MMA is
-// bounded in time.
+// bounded in time. The kernel shares the GPU with the suffix decode that is
+// launched after it as its programmatic dependent.
 #pragma once
 
 #include <cuda.h>
@@ -329,6 +330,10 @@ __global__ void __launch_bounds__(UmmaCfg<D, NT, NSTAGE>::kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_o) {
+  // the suffix decode, launched after this kernel as its programmatic
+  // dependent, may start on the SMs this grid leaves free as soon as every
+  // CTA here has started
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr bool BF16 = std::is_same<TQ, __nv_bfloat16>::value;
   using C = UmmaCfg<D, NT, NSTAGE>;
   constexpr int SLABS = C::kSlabs;

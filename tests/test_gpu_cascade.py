@@ -110,8 +110,9 @@ def test_dirty_workspace_and_repeat():
 
 
 def test_cuda_graph_capture_and_replay():
-    # the 16-bit cascade forks onto the library's side stream and joins back:
-    # captured from the caller's stream it must replay to the eager result
+    # the 16-bit cascade chains its prefix, suffix and merge kernels on the
+    # caller's stream as programmatic dependents: captured from that stream it
+    # must replay to the eager result
     w = W.llama2_70b_prefix(batch=16, prefix_len=512, max_suffix=600)
     step, _ = run_cascade(w, w.meta["shared_prefix_blocks"], check_caches=False)
     eager = step.out.clone()
