@@ -13,13 +13,15 @@ the step's inputs copied from pinned host memory and the output read back
 inside the timed region; `cpu_baseline` times the float64 CPU oracle on the
 host's cores on the same inputs.
 
-L2 is flushed between timed steps (a 256 MiB buffer, twice the L2, is
-written outside the timed events), so every step reads its KV cache from
-HBM; the line also carries the same measurement without the flush
-(`unflushed`). At one GPU the line adds `other_configs`: the 70B-shaped
-shared-prefix layer, the 128K-token long context at batch 1 and 4 and the
-FP8 cache with beam forks, each timed the same way in the same run, with its
-decode roofline, clocks and a check of sampled outputs against the oracle.
+L2 is flushed between timed steps, outside the timed events: a 256 MiB
+buffer (twice the L2) is written, then another one is read, so every step
+reads its KV cache from HBM and starts with clean lines in L2 (a write alone
+would leave the step to pay the write-back of the flush's dirty lines). The
+line also carries the same measurement without the flush (`unflushed`). At
+one GPU the line adds `other_configs`: the 70B-shaped shared-prefix layer,
+the 128K-token long context at batch 1 and 4 and the FP8 cache with beam
+forks, each timed the same way in the same run, with its decode roofline,
+clocks and a check of sampled outputs against the oracle.
 
 Multi-GPU (torchrun): every rank runs its own independent batch of the same
 shape (sequences are independent; no data-path collective), so per-GPU work
@@ -51,7 +53,7 @@ if ROOT not in sys.path:
 METRIC = "paged-decode KV GB/s and % of B200 HBM peak; decode attn tokens/s per layer"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-L2_FLUSH_BYTES = 256 << 20  # written between timed steps: twice the 126 MB L2
+L2_FLUSH_BYTES = 256 << 20  # written, then another as large read, between timed steps
 # measured beside the headline at one GPU: (family, batch; None = the family's)
 OTHER_CONFIGS = [("llama2_70b_prefix", None), ("long_context", 1), ("long_context", 4),
                  ("fp8_beams", None)]
@@ -319,9 +321,9 @@ def l2_note(flushed: bool, w) -> str:
     elt = 1 if w.cache_dtype == "e4m3" else 2
     pool_gb = 2 * w.num_blocks * w.block_size * w.num_kv_heads * w.head_dim * elt / 1e9
     if flushed:
-        return (f"flushed: a {L2_FLUSH_BYTES >> 20} MiB buffer (twice the L2) is written between "
-                "timed steps, outside the timed events; step time = sum of the per-step "
-                f"event intervals (pool {pool_gb:.2f} GB)")
+        return (f"flushed: between timed steps, outside the timed events, a {L2_FLUSH_BYTES >> 20} "
+                "MiB buffer (twice the L2) is written and another one read; step time = sum of "
+                f"the per-step event intervals (pool {pool_gb:.2f} GB)")
     return f"not flushed: steps back to back (pool {pool_gb:.2f} GB)"
 
 
@@ -407,10 +409,27 @@ def decode_plan(args, w, step, spb):
     return pt, n, 1 + (n > 1), name
 
 
+class L2Flush:
+    """Two buffers of L2_FLUSH_BYTES: `run()` writes the first and reads the
+    second, so that L2 ends up holding clean lines of neither the step's
+    data nor dirty ones whose write-back the next step would pay."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+        self.n = 0
+
+    def run(self):
+        self.n += 1
+        self.w.fill_(self.n & 255)
+        self.sink = self.r.sum()
+
+
 def timed_steps(step, steps: int, fused: bool, stream, flush=None):
     """Record `steps` steps (copy, append, decode) on `stream` with a pair of
-    events around each step and each decode call; with `flush`, the buffer
-    is rewritten before each step, outside its events. Returns the event
+    events around each step and each decode call; with `flush` (an L2Flush),
+    L2 is flushed before each step, outside its events. Returns the event
     pairs; read them after a synchronize."""
     import torch
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -419,7 +438,7 @@ def timed_steps(step, steps: int, fused: bool, stream, flush=None):
     call = step.append_decode if fused else step.decode
     for i in range(steps):
         if flush is not None:
-            flush.fill_(i & 255)
+            flush.run()
         ev_step[i][0].record(stream)
         step.copy()
         if not fused:
@@ -463,7 +482,7 @@ def measure_other(args, name, batch, dev, stream, local_rank, peak):
     torch.cuda.synchronize(dev)
     if step.device_errors():
         raise RuntimeError(f"{name}: device bounds error during warm-up")
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     steps = args.other_steps
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -544,7 +563,7 @@ def run_ours(args):
 
     # ---- device-timed steps: L2 flushed between steps (default), then the
     # same steps back to back ----
-    flush = None if args.no_flush else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = None if args.no_flush else L2Flush(dev)
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
@@ -705,8 +724,7 @@ def main(argv=None):
                     help="decode a workload whose sequences share prefix blocks through "
                          "pa_decode_shared_prefix (auto) or plain pa_decode (off)")
     ap.add_argument("--no-flush", action="store_true",
-                    help="time the steps back to back without writing the L2 flush buffer "
-                         "between them")
+                    help="time the steps back to back, without the L2 flush between them")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="measure the headline workload only (at one GPU the line otherwise "
                          "adds the other benchmark families)")
