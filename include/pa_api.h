@@ -235,16 +235,14 @@ size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads
  * PA_DEVERR_PREFIX (its output is then not meaningful).
  * 16-bit caches with blocks of at least 8 tokens, at most 128 query heads
  * per KV head and fewer than 2^31 slots: the prefix part runs on tcgen05
- * tensor cores, on a stream the library owns (one per device, created at the
- * first call): the call
- * records an event on `stream`, makes its stream wait for it, launches the
- * prefix kernel there, and makes `stream` wait for that kernel before the
- * merge. Work enqueued on `stream` after the call therefore sees the
- * complete result, and the call can be captured into a CUDA graph from
- * `stream`. Calls from several host threads are serialised around the
- * fork and join. A tensor-core wait that gives up (1 s) sets
- * PA_DEVERR_TIMEOUT. Other caches (E4M3, smaller blocks, larger groups) run
- * the prefix on mma.sync in the same launch as the suffixes.
+ * tensor cores. The call enqueues three kernels on `stream`: the prefix
+ * kernel, the suffix decode launched as its programmatic dependent (it runs
+ * beside the prefix kernel and completes only after it), and the split-K
+ * merge as the suffix decode's dependent. Work enqueued on `stream` after
+ * the call therefore sees the complete result, and the call can be captured
+ * into a CUDA graph from `stream`. A tensor-core wait that gives up (1 s)
+ * sets PA_DEVERR_TIMEOUT. Other caches (E4M3, smaller blocks, larger groups)
+ * run the prefix on mma.sync in the same launch as the suffixes.
  *   prefix_blocks  number of shared leading blocks (0: plain pa_decode);
  *                  prefix_blocks * block_size must not exceed max_context.
  *   workspace      at least pa_decode_shared_prefix_workspace_size(...) bytes,
@@ -292,7 +290,12 @@ void pa_testing_withhold_prefix_scores(int32_t on);
 
 /* Synchronise `stream`, then read and clear the current device's error
  * word into *flags (PA_DEVERR_* bits). Returns PA_ERR_DEVICE_BOUNDS when
- * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure. */
+ * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure.
+ * The word is one per device, shared by every stream: only `stream` is
+ * synchronised, so a bit set by a kernel on another stream is reported by
+ * whichever call reads the word next (and a kernel on another stream still
+ * running may set one after the read). To attribute errors to calls, read
+ * the word with no other stream of the library's calls in flight. */
 pa_status pa_get_device_error(void* stream, uint32_t* flags);
 
 /* pa_decode without a caller-supplied workspace and without allocating any.
