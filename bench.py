@@ -401,7 +401,8 @@ def decode_plan(args, w, step, spb):
         pt = args.partition_tokens or B.pa_decode_shared_prefix_partition_tokens(
             w.batch, w.num_q_heads, w.max_context, spb, step.cache)
         n = max(1, math.ceil((w.max_context - spb * w.block_size) / pt))
-        return pt, n, 3, "pa_decode_shared_prefix (prefix + suffix + merge kernels)"
+        return pt, n, 3 if w.cache_dtype != "e4m3" else 2, \
+            "pa_decode_shared_prefix (prefix + suffix + merge kernels)"
     pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, w.max_context, step.cache)
     n = max(1, math.ceil(w.max_context / pt))
     name = ("pa_append_decode (append fused into decode; main + split-K reduce)" if args.fused

@@ -182,6 +182,7 @@ cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, siz
 template <typename TQ, int D>
 pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
+  const int n = p.num_partitions;
   auto go = [&](auto kern, int warps, int rows_per_cta) {
     const int64_t ctas = (rows + rows_per_cta - 1) / rows_per_cta;
     return launch_dependent(kern, dim3(static_cast<unsigned>(ctas)), dim3(warps * 32), 0, st, p) ==
@@ -191,11 +192,11 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   };
   // one warp per row: 32 rows per CTA, so that a large batch's merge is a few
   // hundred CTAs that all start at once
-  if (p.num_partitions <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32>, 32, 32);
-  if (p.num_partitions <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32>, 32, 32);
-  if (p.num_partitions <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2, 16, 8>, 8, 4);
-  if (p.num_partitions <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 16, 8>, 8, 2);
-  if (p.num_partitions <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16>, 16, 1);
+  if (n <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32>, 32, 32);
+  if (n <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32>, 32, 32);
+  if (n <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2, 16, 8>, 8, 4);
+  if (n <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 16, 8>, 8, 2);
+  if (n <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16>, 16, 1);
   return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 16, 32>, 32, 1);
 }
 
@@ -207,6 +208,8 @@ pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
   auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
                       : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
+  if constexpr (CK == pa::kE4M3 && NH == 1)
+    if (!p.k_new) kern = pa::pa_decode_e4m3_kernel<TQ, D, kDecodeWarps, kDecodeStages>;
   const int bt_entries = pa::staged_block_ids(p.partition_tokens, p.bs_log2);
   const int smem = (p.k_new && CK == pa::kE4M3)
                        ? S::new_rows_offset(bt_entries) + S::kNewRowBytes

@@ -1,8 +1,8 @@
 // Device helpers shared by the paged-attention kernels (sm_100a).
 //
 // Thin wrappers over PTX instructions: asynchronous global->shared copies,
-// ldmatrix, the m16n8k16 (16-bit) and m16n8k32 (E4M3) tensor-core MMAs, the
-// hardware base-2 exponential and the E4M3 <-> f16/f32 conversions.
+// ldmatrix, the m16n8k16 tensor-core MMA, the hardware base-2 exponential
+// and the E4M3 <-> f16/f32 conversions.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -91,17 +91,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
   }
-}
-
-// D(16x8, f32) += A(16x32, row) * B(32x8, col), A and B E4M3 (four codes per
-// register, the lowest k in the lowest byte).
-__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // 2^x on the SFU (ex2.approx; 2^-inf = 0).

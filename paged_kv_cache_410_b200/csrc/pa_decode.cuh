@@ -10,10 +10,10 @@
 // `partition_tokens` tokens): every query head of the KV head's group
 // (grouped-query attention, KV cache article section "显存账本") is served
 // from one read of the partition's K and V, so KV bytes cross HBM once per
-// KV head. Warps of the CTA take tiles of 16 tokens (32 for an E4M3 cache)
-// round-robin, each with its own NSTAGE-deep cp.async pipeline into shared
-// memory (no CTA-wide barrier in the main loop), and keep their own running
-// max / sum / output (online softmax). At the end the warps merge through shared memory; a sequence
+// KV head. Warps of the CTA take 16-token tiles round-robin, each with its
+// own NSTAGE-deep cp.async pipeline into shared memory (no CTA-wide barrier
+// in the main loop), and keep their own running max / sum / output (online
+// softmax). At the end the warps merge through shared memory; a sequence
 // that spans one partition writes its output directly, longer ones write
 // (max, sum, normalised output) partials that the reduce kernel combines.
 //
@@ -28,14 +28,13 @@
 // tokens or channels, so no accumulator row is padding; groups of 9..16
 // query heads use two column blocks.
 //
-// E4M3 caches. A tile is 32 tokens (8 KB of K and V at head_dim 128, as a
-// 16-token tile of a 16-bit cache), and S^T = K Q^T runs on E4M3 operands
-// (m16n8k32): K tiles enter the MMA as stored, and the query, with the K
-// scale folded in (q' = q * k_scale), is three E4M3 terms after a power-of-
-// two scaling of its row, so that their sum carries about as many bits as
-// f16. The V codes are widened to f16 (exactly) in registers for
-// O^T += V^T P^T with P in f16, and the V scale is applied to the merged
-// output.
+// E4M3 caches. K and V codes are widened to f16 in registers (exactly:
+// every E4M3 value is an f16 value) and both products run on f16 MMAs. The
+// K scale is folded into the query (q' = q * k_scale), which is scaled per
+// row by a power of two (max |q'| 2^e in [2^14, 2^15), so that no channel
+// of it falls into f16's subnormals) and rounded to f16 once; the
+// softmax's per-column log2 scale carries 2^-e, and the V scale multiplies
+// the merged output.
 #pragma once
 
 #include "pa_common.cuh"
@@ -153,6 +152,7 @@ __device__ __forceinline__ int suffix_partitions(const DecodeParams& p, int L) {
 
 enum CacheKind { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
 
+
 // Block ids of one partition staged in shared memory (longer slices are read
 // from global memory row by row).
 constexpr int kBlockIdsInSmem = 1024;
@@ -164,13 +164,13 @@ constexpr int kBlockIdsInSmem = 1024;
 // cancels in the final normalisation.
 constexpr float kRescaleLog2 = 8.f;
 
-template <int CK, int D, int TOK = 16>
+template <int CK, int D>
 struct TileGeom {
   static constexpr int ES = (CK == kE4M3) ? 1 : 2;  // bytes per cache element
   static constexpr int RB = D * ES;                  // bytes per token row (one head)
   static constexpr int CPR = RB / 16;                // 16-byte chunks per row
-  static constexpr int TOKENS = TOK;                 // rows of a tile
-  static constexpr int TB = TOK * RB;                // one tile of K (or V)
+  static constexpr int TOKENS = 16;                  // rows of a tile
+  static constexpr int TB = TOKENS * RB;             // one tile of K (or V)
   static_assert(CPR == 4 || CPR == 8 || CPR == 16, "unsupported row size");
   // Byte offset of 16-byte chunk `c` of row `r` inside a tile. Rows of 128 B
   // or more XOR the low three chunk bits with the row, so that 8 rows read
@@ -187,16 +187,9 @@ struct TileGeom {
   }
 };
 
-// Tokens of a decode tile: 16 for 16-bit caches, 32 for E4M3 (the same
-// bytes per tile).
-template <int CK>
-__host__ __device__ constexpr int decode_tile_tokens() {
-  return CK == kE4M3 ? 32 : 16;
-}
-
 template <int CK, int D, int NW, int NSTAGE>
 struct DecodeSmem {
-  using G = TileGeom<CK, D, decode_tile_tokens<CK>()>;
+  using G = TileGeom<CK, D>;
   static constexpr int kStageBytes = 2 * G::TB;  // K tile + V tile
   static constexpr int kPipeBytes = NW * NSTAGE * kStageBytes;
   static constexpr int kMergeBytes = NW * 16 * D * 4 + NW * 16 * 3 * 4 + 32 * 4;
@@ -241,28 +234,18 @@ __device__ __forceinline__ void load_query_fragments(const TQ* const (&rows)[NH]
   }
 }
 
-// E4M3 codes of two floats and the floats they decode to.
-__device__ __forceinline__ uint32_t e4m3x2_round(float lo, float hi, float& rlo, float& rhi) {
-  const uint32_t code = f32x2_to_e4m3x2(lo, hi);
-  uint32_t h, unused;
-  e4m3x4_to_f16x2x2(code, h, unused);
-  const __half2 v = *reinterpret_cast<const __half2*>(&h);
-  rlo = __low2float(v);
-  rhi = __high2float(v);
-  return code;
-}
-
-// Q^T fragments for an E4M3 cache (B operand of m16n8k32). Thread (g, t)
-// holds query row rows[nh] (column g of block nh; nullptr: zeros) times the K
-// scale, q' = q * k_scale, scaled by 2^e with e chosen per row so that
-// max |q'| 2^e lies in [128, 256), as three E4M3 terms: term 1 = e4m3(q' 2^e),
-// term 2 = e4m3 of what term 1 leaves, term 3 = e4m3 of what both leave.
-// qf[j][kk][nh] = {channels 32kk + 4t .. 32kk + 4t + 3 ; 32kk + 16 + 4t ..
-// + 3} of term j. sl2[nh][e] = scale_log2 * 2^-e of the row in accumulator
-// column 2t + e, which undoes the scaling in the softmax.
+// Q^T fragments for an E4M3 cache (B operand of the f16 MMA on widened K).
+// Thread (g, t) holds query row rows[nh] (column g of block nh; nullptr:
+// zeros) times the K scale, q' = q * k_scale (fp32), scaled by 2^e with e
+// chosen per row so that max |q'| 2^e lies in [2^14, 2^15), rounded to f16
+// once. Channel order (shared with attend_tile_e4m3's K fragments): within
+// each 32-channel group gq, k-step 2gq + h holds channels 8t + 4h + {0,1} in
+// slots 2t, 2t+1 and 8t + 4h + {2,3} in slots 2t+8, 2t+9, so that a thread's
+// K codes are 8 contiguous bytes. sl2[nh][e] = scale_log2 * 2^-e of the row
+// in accumulator column 2t + e.
 template <typename TQ, int D, int NH>
 __device__ __forceinline__ void load_query_e4m3(const TQ* const (&rows)[NH], const float* ks,
-                                                float scale_log2, uint32_t (&qf)[3][D / 32][NH][2],
+                                                float scale_log2, uint32_t (&qb)[D / 16][NH][2],
                                                 float (&sl2)[NH][2]) {
   const int t = threadIdx.x & 3;
 #pragma unroll
@@ -272,42 +255,32 @@ __device__ __forceinline__ void load_query_e4m3(const TQ* const (&rows)[NH], con
     float x[D / 32][2][4];
     float mx = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < D / 32; ++kk)
+    for (int gq = 0; gq < D / 32; ++gq)
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int c = 32 * kk + 16 * h + 4 * t + i;
-          x[kk][h][i] = ok ? to_f32<TQ>(qr[c]) * ks[c] : 0.f;
-          mx = fmaxf(mx, fabsf(x[kk][h][i]));
+          const int c = 32 * gq + 8 * t + 4 * h + i;
+          x[gq][h][i] = ok ? to_f32<TQ>(qr[c]) * ks[c] : 0.f;
+          mx = fmaxf(mx, fabsf(x[gq][h][i]));
         }
     // the four threads of the group hold the row's channels between them
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    // e = 7 - floor(log2 mx) (from the exponent field; kept within a range
+    // e = 14 - floor(log2 mx) (from the exponent field; kept within a range
     // where 2^e and 2^-e are normal floats)
     int e = 0;
     if (mx > 0.f) {
       const int ex = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
-      e = min(max(7 - ex, -100), 100);
+      e = min(max(14 - ex, -100), 100);
     }
     const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);  // 2^e
 #pragma unroll
-    for (int kk = 0; kk < D / 32; ++kk)
+    for (int gq = 0; gq < D / 32; ++gq)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        float y[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) y[i] = x[kk][h][i] * up;  // exact
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          float r[4];
-          const uint32_t c01 = e4m3x2_round(y[0], y[1], r[0], r[1]);
-          const uint32_t c23 = e4m3x2_round(y[2], y[3], r[2], r[3]);
-          qf[j][kk][nh][h] = c01 | (c23 << 16);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) y[i] -= r[i];  // exact: what the terms so far leave
-        }
+        qb[2 * gq + h][nh][0] = pack2<false>(x[gq][h][0] * up, x[gq][h][1] * up);
+        qb[2 * gq + h][nh][1] = pack2<false>(x[gq][h][2] * up, x[gq][h][3] * up);
       }
     // the accumulator's columns 2t, 2t + 1 are the rows of threads (2t, *) and
     // (2t + 1, *)
@@ -423,73 +396,57 @@ __device__ __forceinline__ void attend_tile(uint32_t sk_a, uint32_t sv_a, int nv
   }
 }
 
-// One tile of K and V of an E4M3 cache (rows < nskip or >= nvalid are zero
-// and masked; FULL: all rows count). S^T for each 16-token row block mt on
-// E4M3 MMAs, s[mt][nh] = {(token 16mt + g, columns 2t, 2t+1), (token
-// 16mt + g + 8, same)}, summed over the query's three terms; one online-
-// softmax update over the tile (sl2: the per-column log2 scale that also
-// undoes the query's power-of-two scaling); then O^T += V^T P^T per 16-token
-// block with V widened to f16.
+// One 16-token tile of K and V of an E4M3 cache (rows < nskip or >= nvalid
+// are zero and masked; FULL: all 16 rows count): S^T = K Q^T with K widened
+// to f16 in registers, s[nh] = {(token g, columns 2t, 2t+1), (token g + 8,
+// same)}; online softmax as attend_tile, with the per-column log2 scale sl2;
+// O^T += V^T P^T with V widened to f16.
 template <int D, int NH, bool FULL>
 __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, int nvalid,
                                                  int nskip, const float (&sl2)[NH][2],
-                                                 const uint32_t (&qf)[3][D / 32][NH][2],
+                                                 const uint32_t (&qb)[D / 16][NH][2],
                                                  float (&o)[D / 16][NH][4], float (&m_run)[NH][2],
                                                  float (&l_run)[NH][2]) {
-  using G = TileGeom<kE4M3, D, decode_tile_tokens<kE4M3>()>;
-  constexpr int MB = G::TOKENS / 16;  // 16-token row blocks of the tile
+  using G = TileGeom<kE4M3, D>;
   constexpr int MT = D / 16;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
   const int t = lane & 3;
 
-  float s[MB][NH][4];
+  float s[NH][4];
 #pragma unroll
-  for (int mt = 0; mt < MB; ++mt)
+  for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
+  // thread (g, t) reads 8 contiguous channel bytes of tokens g and g + 8 in
+  // each 32-channel group gq (the query's channel order)
 #pragma unroll
-    for (int nh = 0; nh < NH; ++nh) s[mt][nh][0] = s[mt][nh][1] = s[mt][nh][2] = s[mt][nh][3] = 0.f;
-  {
-    // A fragments of 16 tokens x 32 channels straight from the tile (bytes
-    // 4t.. of rows g, g + 8, then bytes 16 + 4t..): ldmatrix's b16 layout
-    const int mi = lane >> 3;
-    const int tok = (lane & 7) + 8 * (mi & 1);
-    const int chk = mi >> 1;
+  for (int gq = 0; gq < D / 32; ++gq) {
+    const int c = 2 * gq + (t >> 1);
+    const int bo = (t & 1) * 8;
+    const uint2 wl = lds64(sk_a + G::off(g, c) + bo);      // token g
+    const uint2 wh = lds64(sk_a + G::off(g + 8, c) + bo);  // token g + 8
+    uint32_t a0[4], a1[4];
+    e4m3x4_to_f16x2x2(wl.x, a0[0], a0[2]);
+    e4m3x4_to_f16x2x2(wh.x, a0[1], a0[3]);
+    e4m3x4_to_f16x2x2(wl.y, a1[0], a1[2]);
+    e4m3x4_to_f16x2x2(wh.y, a1[1], a1[3]);
 #pragma unroll
-    for (int kk = 0; kk < D / 32; ++kk)
-#pragma unroll
-      for (int mt = 0; mt < MB; ++mt) {
-        uint32_t a[4];
-        ldmatrix_x4(a[0], a[1], a[2], a[3], sk_a + G::off(16 * mt + tok, 2 * kk + chk));
-#pragma unroll
-        for (int nh = 0; nh < NH; ++nh)
-#pragma unroll
-          for (int j = 2; j >= 0; --j)  // smallest term first
-            mma_16832_e4m3(s[mt][nh], a, qf[j][kk][nh][0], qf[j][kk][nh][1]);
-      }
+    for (int nh = 0; nh < NH; ++nh) {
+      mma_16816<false>(s[nh], a0, qb[2 * gq][nh][0], qb[2 * gq][nh][1]);
+      mma_16816<false>(s[nh], a1, qb[2 * gq + 1][nh][0], qb[2 * gq + 1][nh][1]);
+    }
   }
 
-  // rows g, g + 8 (, g + 16, g + 24) of the tile
-  bool v[MB][2];
-#pragma unroll
-  for (int mt = 0; mt < MB; ++mt)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int r = 16 * mt + 8 * hh + g;
-      v[mt][hh] = FULL || (r < nvalid && r >= nskip);
-    }
-  uint32_t pb[MB][NH][2];
+  const bool va = FULL || (g < nvalid && g >= nskip);
+  const bool vb = FULL || (g + 8 < nvalid && g + 8 >= nskip);
+  uint32_t pb[NH][2];
   bool grew = false;
   float alpha[NH][2];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) {
-    float pr[MB][2][2];  // [mt][row half][column e]
+    float pr[2][2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int mt = 0; mt < MB; ++mt)
-        mx = fmaxf(mx, fmaxf(v[mt][0] ? s[mt][nh][e] : -INFINITY,
-                             v[mt][1] ? s[mt][nh][2 + e] : -INFINITY));
+      float mx = fmaxf(va ? s[nh][e] : -INFINITY, vb ? s[nh][2 + e] : -INFINITY);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -501,23 +458,15 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
       grew |= up;
       const float m_ref = up ? mx : m_run[nh][e];
       alpha[nh][e] = up ? ex2(m_run[nh][e] - m_ref) : 1.f;
-      float sum = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < MB; ++mt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float pv = ex2(fmaf(s[mt][nh][2 * hh + e], sc, -m_ref));
-          pr[mt][hh][e] = v[mt][hh] ? pv : 0.f;
-          sum += pr[mt][hh][e];
-        }
-      l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + sum;
+      const float p0 = ex2(fmaf(s[nh][e], sc, -m_ref));
+      const float p1 = ex2(fmaf(s[nh][2 + e], sc, -m_ref));
+      pr[0][e] = va ? p0 : 0.f;
+      pr[1][e] = vb ? p1 : 0.f;
+      l_run[nh][e] = l_run[nh][e] * alpha[nh][e] + (pr[0][e] + pr[1][e]);
       m_run[nh][e] = m_ref;
     }
-#pragma unroll
-    for (int mt = 0; mt < MB; ++mt) {
-      pb[mt][nh][0] = movmatrix_trans(pack2<false>(pr[mt][0][0], pr[mt][0][1]));
-      pb[mt][nh][1] = movmatrix_trans(pack2<false>(pr[mt][1][0], pr[mt][1][1]));
-    }
+    pb[nh][0] = movmatrix_trans(pack2<false>(pr[0][0], pr[0][1]));
+    pb[nh][1] = movmatrix_trans(pack2<false>(pr[1][0], pr[1][1]));
   }
   if (__any_sync(0xffffffffu, grew)) {
 #pragma unroll
@@ -531,46 +480,42 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
       }
   }
 
-  // O^T += V^T P^T, one 16-token block at a time. Row m of O^T block mt is
-  // channel DPT*g + 2*mt (m = g) or that + 1 (m = g + 8): this thread reads
-  // channels [DPT*g, DPT*g + DPT) of token rows 2t, 2t+1, 2t+8, 2t+9 of the
-  // block and pairs tokens with byte permutes.
+  // O^T += V^T P^T. Row m of O^T block mt is channel DPT*g + 2*mt (m = g) or
+  // that + 1 (m = g + 8): this thread reads channels [DPT*g, DPT*g + DPT) of
+  // token rows 2t, 2t+1, 2t+8, 2t+9 and pairs tokens with byte permutes.
   constexpr int DPT = D / 8;
   constexpr int WORDS = DPT / 4;
+  uint32_t ra[4][WORDS];
 #pragma unroll
-  for (int kb = 0; kb < MB; ++kb) {
-    uint32_t ra[4][WORDS];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int r = 16 * kb + 2 * t + (q4 & 1) + 8 * (q4 >> 1);
-      const int byte0 = DPT * g;
-      const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
-      if constexpr (WORDS == 4) {
-        const uint4 w = lds128(addr);
-        ra[q4][0] = w.x;
-        ra[q4][1] = w.y;
-        ra[q4][2] = w.z;
-        ra[q4][3] = w.w;
-      } else {
-        const uint2 w = lds64(addr);
-        ra[q4][0] = w.x;
-        ra[q4][1] = w.y;
-      }
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int r = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
+    const int byte0 = DPT * g;
+    const uint32_t addr = sv_a + G::off(r, byte0 >> 4) + (byte0 & 15);
+    if constexpr (WORDS == 4) {
+      const uint4 w = lds128(addr);
+      ra[q4][0] = w.x;
+      ra[q4][1] = w.y;
+      ra[q4][2] = w.z;
+      ra[q4][3] = w.w;
+    } else {
+      const uint2 w = lds64(addr);
+      ra[q4][0] = w.x;
+      ra[q4][1] = w.y;
     }
+  }
 #pragma unroll
-    for (int w = 0; w < WORDS; ++w) {
-      uint32_t f[4], e[4];
-      e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x5140), f[0], f[1]);
-      e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x7362), f[2], f[3]);
-      e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x5140), e[0], e[1]);
-      e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x7362), e[2], e[3]);
-      const uint32_t a0[4] = {f[0], f[1], e[0], e[1]};  // channel block 2w
-      const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
+  for (int w = 0; w < WORDS; ++w) {
+    uint32_t f[4], e[4];
+    e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x5140), f[0], f[1]);
+    e4m3x4_to_f16x2x2(__byte_perm(ra[0][w], ra[1][w], 0x7362), f[2], f[3]);
+    e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x5140), e[0], e[1]);
+    e4m3x4_to_f16x2x2(__byte_perm(ra[2][w], ra[3][w], 0x7362), e[2], e[3]);
+    const uint32_t a0[4] = {f[0], f[1], e[0], e[1]};  // channel block 2w
+    const uint32_t a1[4] = {f[2], f[3], e[2], e[3]};  // channel block 2w+1
 #pragma unroll
-      for (int nh = 0; nh < NH; ++nh) {
-        mma_16816<false>(o[2 * w][nh], a0, pb[kb][nh][0], pb[kb][nh][1]);
-        mma_16816<false>(o[2 * w + 1][nh], a1, pb[kb][nh][0], pb[kb][nh][1]);
-      }
+    for (int nh = 0; nh < NH; ++nh) {
+      mma_16816<false>(o[2 * w][nh], a0, pb[nh][0], pb[nh][1]);
+      mma_16816<false>(o[2 * w + 1][nh], a1, pb[nh][0], pb[nh][1]);
     }
   }
 }
@@ -587,7 +532,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   using S = DecodeSmem<CK, D, NW, NSTAGE>;
   using G = typename S::G;
   constexpr bool kE4 = (CK == kE4M3);
-  constexpr int TOK = G::TOKENS;            // tokens per tile (16, or 32 for E4M3)
+  constexpr int TOK = G::TOKENS;            // tokens per tile
   constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T (16-bit)
   constexpr int MT = D / 16;                // 16-channel row blocks of O^T
   constexpr int RPI = 32 / G::CPR;          // tile rows one load instruction covers
@@ -659,9 +604,8 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   // ---- Q^T fragments (B operand: k = channel, n = query head) -------------
   const TQ* qbase = reinterpret_cast<const TQ*>(p.q) +
                     (static_cast<int64_t>(b) * p.num_q_heads + hq0) * D;
-  uint32_t qb[kE4 ? 1 : KSTEPS][NH][2];         // 16-bit caches
-  uint32_t qf[kE4 ? 3 : 1][kE4 ? D / 32 : 1][NH][2];  // E4M3: three query terms
-  float sl2[NH][2];                              // E4M3: per-column log2 scale
+  uint32_t qb[KSTEPS][NH][2];
+  float sl2[NH][2];  // E4M3: per-column log2 scale
   {
     const TQ* rows[NH];
 #pragma unroll
@@ -669,7 +613,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
       rows[nh] = 8 * nh + g < nrows ? qbase + (8 * nh + g) * D : nullptr;
     if constexpr (kE4)
       load_query_e4m3<TQ, D, NH>(rows, p.k_scale + static_cast<int64_t>(hk) * D, p.scale_log2,
-                                 qf, sl2);
+                                 qb, sl2);
     else
       load_query_fragments<TQ, D, NH>(rows, qb);
   }
@@ -681,9 +625,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const uint8_t* vc = reinterpret_cast<const uint8_t*>(p.v_cache);
   const int64_t slot_stride = static_cast<int64_t>(p.num_kv_heads) * G::RB;
   const int bs_mask = (1 << p.bs_log2) - 1;
-  // blocks of >= 16 tokens: each 16-row half of a tile lies inside one block
-  // (tiles start 16-aligned)
-  const bool block_aligned = p.bs_log2 >= 4;
+  const bool block_aligned = p.bs_log2 >= 4;  // a 16-token tile lies inside one block
   // this lane's load slots: rows lrow + i*RPI, 16-byte chunk lch
   const int lrow = lane / G::CPR;
   const int lch = lane % G::CPR;
@@ -783,23 +725,16 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const uint32_t sv_a = sk_a + G::TB;
     const int tb = t0 + tile * TOK;
     if (block_aligned) {
-      constexpr int IPH = LITERS / (TOK / 16);  // load instructions per 16-row half
+      const int blk = block_id((tb >> p.bs_log2) - bt0);
+      const int64_t base =
+          ((static_cast<int64_t>(blk) << p.bs_log2) + (tb & bs_mask) + lrow) * slot_stride +
+          lane_goff;
 #pragma unroll
-      for (int h = 0; h < TOK / 16; ++h) {
-        // a half that starts past the partition's end is not looked up (its
-        // block id need not be staged)
-        const int th = tb + 16 * h;
-        const int blk = th < t1 ? block_id((th >> p.bs_log2) - bt0) : -1;
-        const int64_t base =
-            ((static_cast<int64_t>(blk) << p.bs_log2) + (th & bs_mask) + lrow) * slot_stride +
-            lane_goff;
-#pragma unroll
-        for (int ii = 0; ii < IPH; ++ii) {
-          const int r = 16 * h + lrow + ii * RPI;
-          const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
-          const int64_t off = ok ? base + static_cast<int64_t>(ii * RPI) * slot_stride : 0;
-          load_chunk(sk_a, sv_a, r, tb + r, ok, off);
-        }
+      for (int i = 0; i < LITERS; ++i) {
+        const int r = lrow + i * RPI;
+        const bool ok = blk >= 0 && tb + r < t1 && tb + r >= lo;
+        const int64_t off = ok ? base + static_cast<int64_t>(i * RPI) * slot_stride : 0;
+        load_chunk(sk_a, sv_a, r, tb + r, ok, off);
       }
     } else {
 #pragma unroll
@@ -854,9 +789,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const int nskip = max(lo - ts, 0);         // rows before the window (first tile only)
     if constexpr (kE4) {
       if (nvalid >= TOK && nskip == 0)
-        attend_tile_e4m3<D, NH, true>(sk_a, sv_a, nvalid, 0, sl2, qf, o, m_run, l_run);
+        attend_tile_e4m3<D, NH, true>(sk_a, sv_a, nvalid, 0, sl2, qb, o, m_run, l_run);
       else
-        attend_tile_e4m3<D, NH, false>(sk_a, sv_a, nvalid, nskip, sl2, qf, o, m_run, l_run);
+        attend_tile_e4m3<D, NH, false>(sk_a, sv_a, nvalid, nskip, sl2, qb, o, m_run, l_run);
     } else {
       if (nvalid >= TOK && nskip == 0)
         attend_tile<CK, D, NH, true>(sk_a, sv_a, nvalid, 0, p.scale_log2, qb, o, m_run, l_run);
@@ -943,9 +878,10 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   if constexpr (FUSED && CK == kE4M3) store_new_token();
 }
 
-// grid: (partitions, num_kv_heads * head_groups, batch)
+// One decode CTA of the launch: the sequence (longest first, when asked),
+// the CTA itself, and in cascade mode the wait for the prefix grid.
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
-__global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
+__device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
   // a kernel launched after this one as its programmatic dependent (the
   // split-K merge) may start as soon as every CTA here has started; it waits
   // for this grid's completion before reading anything
@@ -973,6 +909,20 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p
   // early; it completes only after the prefix grid has, so that the merge,
   // which waits for this grid, also sees the prefix partials
   if (p.prefix_blocks > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// grid: (partitions, num_kv_heads * head_groups, batch)
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
+__global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
+  decode_launch_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p);
+}
+
+// The same for an E4M3 cache and up to 8 query heads per KV head (no fused
+// append), held to 5 CTAs per SM (102 registers): that decode is bound by
+// instruction latency, and the extra warps pay (measured).
+template <typename TQ, int D, int NW, int NSTAGE>
+__global__ void __launch_bounds__(NW * 32, 5) pa_decode_e4m3_kernel(const DecodeParams p) {
+  decode_launch_cta<TQ, kE4M3, D, NW, NSTAGE, 1, false>(p);
 }
 
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
