@@ -389,14 +389,18 @@ def make_step(args, w, dev, spb):
 
 
 def decode_plan(args, w, step, spb):
-    """(partition tokens, partitions, decode launches, kernel description)."""
+    """(partition tokens, partitions, decode launches, kernel description).
+    A split decode of more than one sequence launches the work-list plan
+    kernel, the decode and the split-K merge; one partition, the decode
+    alone."""
     from paged_kv_cache_410_b200 import binding as B
+    split = lambda n: (n > 1) * (2 + (w.batch > 1)) or 1  # noqa: E731
     if args.window:
         span = min(w.max_context, args.window + 15)
         pt = args.partition_tokens or B.pa_decode_partition_tokens(w.batch, span, step.cache)
         n = max(1, math.ceil(span / pt))
-        return pt, n, 1 + (n > 1), (f"pa_decode_sliding_window (window {args.window}; "
-                                    "main + split-K reduce)")
+        return pt, n, split(n), (f"pa_decode_sliding_window (window {args.window}; "
+                                 "main + split-K reduce)")
     if spb:
         pt = args.partition_tokens or B.pa_decode_shared_prefix_partition_tokens(
             w.batch, w.num_q_heads, w.max_context, spb, step.cache)
@@ -407,7 +411,7 @@ def decode_plan(args, w, step, spb):
     n = max(1, math.ceil(w.max_context / pt))
     name = ("pa_append_decode (append fused into decode; main + split-K reduce)" if args.fused
             else "pa_decode (main + split-K reduce)")
-    return pt, n, 1 + (n > 1), name
+    return pt, n, split(n), name
 
 
 class L2Flush:

@@ -116,6 +116,12 @@ pa_status pa_append_kv(const void* k, const void* v, int32_t in_dtype, int64_t n
 
 /* Bytes of workspace pa_decode needs for these sizes and this partition
  * choice (0 when one partition covers max_context). Pure host function.
+ * The workspace holds the split-K partials (head_dim + 2 floats per query
+ * head and partition) and the call's work list (one 8-byte entry per
+ * partition a sequence can have, plus 256 bytes): a split decode of more than
+ * one sequence first lists its (sequence, partition) items, longest first,
+ * in one small kernel, then runs them on as many decode CTAs as the GPU holds
+ * at once. Nothing in the workspace needs a starting value.
  * Sizes whose workspace would pass 2^60 bytes are refused: this returns 0
  * and every decode entry point returns PA_ERR_UNSUPPORTED for them (the same
  * rule holds for the sliding-window and shared-prefix sizes below). */

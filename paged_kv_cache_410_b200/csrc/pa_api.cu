@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <type_traits>
 #include <mutex>
 #include <unordered_map>
@@ -93,7 +94,8 @@ int auto_partition(int64_t batch, int64_t max_context, const pa_cache_desc* cd) 
 struct Plan {
   int partition_tokens;
   int num_partitions;
-  size_t ws_o_bytes;
+  size_t ws_o_bytes;     // partial outputs, then (max, sum) pairs
+  size_t ws_list_offset;  // work-list counter (256 bytes), then the items
   size_t ws_bytes;
   bool fits;  // false: the workspace would not be addressable (sizes refused)
 };
@@ -124,11 +126,25 @@ Plan make_plan(int64_t batch, int64_t num_q_heads, int64_t max_context, int part
     pl.ws_o_bytes = round_up(static_cast<size_t>(batch * num_q_heads) * pl.num_partitions *
                                  cd->head_dim * sizeof(float),
                              256);
-    pl.ws_bytes = pl.ws_o_bytes + round_up(static_cast<size_t>(batch * num_q_heads) *
-                                               pl.num_partitions * sizeof(float2),
-                                           256);
+    pl.ws_list_offset = pl.ws_o_bytes + round_up(static_cast<size_t>(batch * num_q_heads) *
+                                                     pl.num_partitions * sizeof(float2),
+                                                 256);
+    // the work list: a counter section, then one (sequence, partition) item
+    // per partition a sequence can have
+    pl.ws_bytes = pl.ws_list_offset + 256 +
+                  round_up(static_cast<size_t>(batch) * pl.num_partitions * sizeof(int2), 256);
   }
   return pl;
+}
+
+// Partials and (plain decode) work list of a split plan in `ws`.
+void bind_workspace(pa::DecodeParams& p, const Plan& pl, void* ws) {
+  if (!pl.ws_bytes) return;
+  char* base = static_cast<char*>(ws);
+  p.ws_o = reinterpret_cast<float*>(base);
+  p.ws_ml = reinterpret_cast<float2*>(base + pl.ws_o_bytes);
+  p.work_count = reinterpret_cast<int*>(base + pl.ws_list_offset);
+  p.work_items = reinterpret_cast<int2*>(base + pl.ws_list_offset + 256);
 }
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device),
@@ -200,22 +216,108 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 16, 32>, 32, 1);
 }
 
-// Decode kernel over `grid_x` partition columns, then the split-K merge when
-// the plan has more than one partial per sequence (or always, in cascade mode).
+// Work-list mode (plain, fused and sliding-window decodes of a batch split
+// into partitions): the workspace holds the list, and the units (items x KV
+// head groups) stay below 2^31. The plan kernel may lengthen the partitions
+// by up to 2^kListGrowLog2 (fewer units and partials when the batch's
+// tokens allow; the workspace, sized for the host's length, holds fewer).
+// The suffix decode of a cascade keeps its grid (its sequences have one
+// partition or few, visited longest first).
+constexpr int kListGrowLog2 = 2;
+
+bool use_work_list(const pa::DecodeParams& p, bool dependent) {
+  return !dependent && p.prefix_blocks == 0 && p.work_items && p.batch > 1 &&
+         p.num_partitions > 1 &&
+         static_cast<int64_t>(p.batch) * p.num_partitions * p.num_kv_heads * p.head_groups <
+             (int64_t{1} << 31);
+}
+
+// CTAs of `kern` resident per SM at this block and shared-memory size, and
+// the device's SM count (cached per kernel, size and device).
+cudaError_t resident_ctas(const void* kern, int threads, int smem, int* per_sm, int* sms) {
+  struct Key {
+    const void* kern;
+    int threads, smem, dev;
+    bool operator==(const Key& o) const {
+      return kern == o.kern && threads == o.threads && smem == o.smem && dev == o.dev;
+    }
+  };
+  struct KeyHash {
+    size_t operator()(const Key& k) const {
+      return std::hash<const void*>()(k.kern) ^
+             (static_cast<size_t>(k.smem) * 131 + static_cast<size_t>(k.threads) * 7 +
+              static_cast<size_t>(k.dev));
+    }
+  };
+  static std::mutex mu;
+  static std::unordered_map<Key, std::pair<int, int>, KeyHash> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const Key key{kern, threads, smem, dev};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    int n = 0, m = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    it = cache.emplace(key, std::make_pair(n, m)).first;
+  }
+  *per_sm = it->second.first;
+  *sms = it->second.second;
+  return cudaSuccess;
+}
+
+// Decode kernel over `grid_x` partition columns (or, in work-list mode, the
+// plan kernel and a persistent grid), then the split-K merge when the plan
+// has more than one partial per sequence (or always, in cascade mode).
 template <typename TQ, int CK, int D, int NH>
-pa_status launch_decode_t(const pa::DecodeParams& p, int grid_x, cudaStream_t st,
+pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t st,
                           bool with_reduce = true, bool dependent = false) {
   using S = pa::DecodeSmem<CK, D, kDecodeWarps, kDecodeStages>;
-  auto kern = p.k_new ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
-                      : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
+  auto kern = p_in.k_new
+                  ? pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, true>
+                  : pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false>;
   if constexpr (CK == pa::kE4M3 && NH == 1)
-    if (!p.k_new) kern = pa::pa_decode_e4m3_kernel<TQ, D, kDecodeWarps, kDecodeStages>;
-  const int bt_entries = pa::staged_block_ids(p.partition_tokens, p.bs_log2);
+    kern = p_in.k_new ? pa::pa_decode_e4m3_kernel<TQ, D, kDecodeWarps, kDecodeStages, true>
+                      : pa::pa_decode_e4m3_kernel<TQ, D, kDecodeWarps, kDecodeStages, false>;
+  pa::DecodeParams p = p_in;
+  const bool list = use_work_list(p, dependent);
+  if (list) {
+    // the plan kernel may lengthen the partitions up to this
+    p.max_partition_tokens = static_cast<int>(
+        std::min<int64_t>(int64_t{p.partition_tokens} << kListGrowLog2, int64_t{1} << 20));
+  } else {
+    p.work_items = nullptr;
+    p.work_count = nullptr;
+    p.max_partition_tokens = 0;
+  }
+  const int bt_entries = pa::staged_block_ids(p);
   const int smem = (p.k_new && CK == pa::kE4M3)
                        ? S::new_rows_offset(bt_entries) + S::kNewRowBytes
                        : S::kMainBytes + bt_entries * 4;
   if (smem > 227 * 1024) return PA_ERR_UNSUPPORTED;
   if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return PA_ERR_CUDA;
+  if (list) {
+    // the plan kernel, then a persistent grid (one CTA per resident slot, at
+    // most one per unit) as its programmatic dependent
+    int per_sm = 0, sms = 0;
+    if (resident_ctas(reinterpret_cast<const void*>(kern), kDecodeWarps * 32, smem, &per_sm,
+                      &sms) != cudaSuccess)
+      return PA_ERR_CUDA;
+    const int64_t hb = static_cast<int64_t>(p.num_kv_heads) * p.head_groups;
+    const int64_t units = static_cast<int64_t>(p.batch) * p.num_partitions * hb;
+    const int64_t ctas = std::min<int64_t>(std::max(per_sm, 1) * int64_t{sms}, units);
+    p.list_slots = static_cast<int>(ctas);
+    pa::pa_decode_plan_kernel<<<1, pa::kPlanThreads, 0, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    if (launch_dependent(kern, dim3(static_cast<unsigned>(ctas)), dim3(kDecodeWarps * 32), smem,
+                         st, p) != cudaSuccess)
+      return PA_ERR_CUDA;
+    return with_reduce ? launch_reduce<TQ, D>(p, st) : PA_OK;
+  }
   dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
   if (dependent) {
     if (launch_dependent(kern, grid, dim3(kDecodeWarps * 32), smem, st, p) != cudaSuccess)
@@ -677,10 +779,7 @@ pa_status pa_decode(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q
   pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
                                      block_tables, max_blocks_per_seq, context_lens, max_context,
                                      scale, out, bs_log2);
-  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
-  p.ws_ml = pl.ws_bytes
-                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
-                : nullptr;
+  bind_workspace(p, pl, workspace);
   p.partition_tokens = pl.partition_tokens;
   p.num_partitions = pl.num_partitions;
   return launch_decode(p, q_dtype, cache, as_stream(stream));
@@ -713,10 +812,7 @@ pa_status pa_append_decode(const void* q, const void* k, const void* v, int32_t 
   pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
                                      block_tables, max_blocks_per_seq, context_lens, max_context,
                                      scale, out, bs_log2);
-  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
-  p.ws_ml = pl.ws_bytes
-                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
-                : nullptr;
+  bind_workspace(p, pl, workspace);
   p.partition_tokens = pl.partition_tokens;
   p.num_partitions = pl.num_partitions;
   p.k_new = k;
@@ -762,10 +858,7 @@ pa_status pa_decode_sliding_window(const void* q, int32_t q_dtype, int32_t batch
   pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
                                      block_tables, max_blocks_per_seq, context_lens, max_context,
                                      scale, out, bs_log2);
-  p.ws_o = pl.ws_bytes ? reinterpret_cast<float*>(workspace) : nullptr;
-  p.ws_ml = pl.ws_bytes
-                ? reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + pl.ws_o_bytes)
-                : nullptr;
+  bind_workspace(p, pl, workspace);
   p.partition_tokens = pl.partition_tokens;
   p.num_partitions = pl.num_partitions;
   p.window = window;

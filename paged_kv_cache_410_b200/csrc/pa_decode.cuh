@@ -91,9 +91,49 @@ struct DecodeParams {
   // of the launch's tail. Each CTA ranks the batch itself (batch <=
   // kOrderMaxBatch).
   int longest_first;
+  // Work-list mode (null: a grid of partitions x head groups x sequences):
+  // pa_decode_plan_kernel writes the launch's (sequence, partition) items to
+  // work_items, largest first, their count to work_count[1] and zero to
+  // work_count[0]; a persistent grid then takes (item, KV head group) units
+  // by atomicAdd on work_count[0].
+  int2* work_items;
+  int* work_count;
+  // Work-list mode: the persistent grid's CTAs (the plan kernel sizes the
+  // partitions by them), and the longest partition a CTA may be given (the
+  // launch's shared memory stages that many tokens' block ids; 0: as
+  // partition_tokens).
+  int list_slots;
+  int max_partition_tokens;
 };
 
 constexpr int kOrderMaxBatch = 256;
+
+// Work-list mode: where a persistent CTA stands in the list (shared memory,
+// written by thread 0): the ticket of its current unit and that unit's item.
+// The next ticket is taken only once the current unit's main loop is done
+// (a ticket reserved earlier would tie a unit to a CTA still busy), and its
+// item is loaded during the epilogue, so that both latencies hide there.
+struct WorkCursor {
+  int u;        // current unit: item u / hb, KV head group u % hb
+  int n_units;  // items x hb
+  int pt;       // the launch's partition length (the plan kernel's choice)
+  int2 item;    // item of u: (sequence, partition)
+};
+
+__device__ __forceinline__ int units_per_item(const DecodeParams& p) {
+  return p.num_kv_heads * p.head_groups;
+}
+
+__device__ __forceinline__ int2 cursor_item(const DecodeParams& p, const WorkCursor& c, int u) {
+  return u < c.n_units ? p.work_items[u / units_per_item(p)] : make_int2(-1, -1);
+}
+
+// thread 0: move the cursor to a new ticket at once
+__device__ __forceinline__ void cursor_next(const DecodeParams& p, WorkCursor& c) {
+  const int u = atomicAdd(p.work_count, 1);
+  c.item = cursor_item(p, c, u);
+  c.u = u;
+}
 
 // 16 consecutive channels of a 16-bit input row -> 16 E4M3 codes, each
 // e4m3_rn_satfinite(fp32(x) * inv_scale) (the append kernel's rounding).
@@ -143,11 +183,18 @@ __device__ __forceinline__ SeqSpan seq_span(const DecodeParams& p, int L) {
 }
 
 // Number of split-K partials of a sequence of length L after the prefix's
-// (cascade mode) ones, shared by the decode and reduce kernels.
-__device__ __forceinline__ int suffix_partitions(const DecodeParams& p, int L) {
+// (cascade mode) ones with partitions of pt tokens, shared by the decode and
+// reduce kernels.
+__device__ __forceinline__ int partitions_of(const DecodeParams& p, int L, int pt) {
   const SeqSpan s = seq_span(p, L);
   const int n = L - s.base;
-  return L > s.lo ? (n + p.partition_tokens - 1) / p.partition_tokens : 0;
+  return L > s.lo ? (n + pt - 1) / pt : 0;
+}
+
+// Partition length of this launch's CTAs: the host's, or in work-list mode
+// the plan kernel's choice (published in work_count[2]).
+__device__ __forceinline__ int launch_partition_tokens(const DecodeParams& p) {
+  return p.work_count ? p.work_count[2] : p.partition_tokens;
 }
 
 enum CacheKind { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
@@ -172,17 +219,29 @@ struct TileGeom {
   static constexpr int TOKENS = 16;                  // rows of a tile
   static constexpr int TB = TOKENS * RB;             // one tile of K (or V)
   static_assert(CPR == 4 || CPR == 8 || CPR == 16, "unsupported row size");
-  // Byte offset of 16-byte chunk `c` of row `r` inside a tile. Rows of 128 B
-  // or more XOR the low three chunk bits with the row, so that 8 rows read
-  // at one chunk column hit 8 distinct bank groups; 64-byte rows are
-  // swizzled per 128-byte line instead.
+  // Byte offset of 16-byte chunk `c` of row `r` inside a tile: the low three
+  // chunk bits are XORed with a function of the row (a permutation within
+  // each 128-byte line), chosen so that every read pattern of the kernels is
+  // free of bank conflicts.
+  //  * 16-bit rows (ldmatrix: 8 rows at one chunk column): r & 7.
+  //  * E4M3, 128-byte rows: a warp reads 8 contiguous bytes per lane of
+  //    rows g = 0..7 at chunk pair {2gq, 2gq + 1} (K), and 16 bytes of
+  //    chunk g of rows 2t + c (V). XORing with r & 7 sends rows r and r ^ 1
+  //    of the K read to the same pair (two-way conflicts); instead the pair
+  //    index takes bit 1 of r and bit 2 XOR bit 0, which is distinct over
+  //    rows 0..3, rows 4..7 (the two half-warps of the K read) and over
+  //    rows {c, c + 2, c + 4, c + 6} (the V read).
+  //  * E4M3, 64-byte rows (two rows per line): the same two reads are free
+  //    of conflicts with 2 * ((r >> 1) & 3).
   __device__ __forceinline__ static uint32_t off(int r, int c) {
-    if constexpr (CPR >= 8) {
+    if constexpr (ES == 2) {
       return static_cast<uint32_t>(r * RB + ((c ^ (r & 7)) << 4));
+    } else if constexpr (CPR >= 8) {
+      const int pair = (r & 2) | (((r >> 2) ^ r) & 1);
+      return static_cast<uint32_t>(r * RB + ((c ^ ((pair << 1) | (r & 1))) << 4));
     } else {
       const int u = r * CPR + c;
-      const int line = r >> 1;
-      return static_cast<uint32_t>(((u & ~7) | ((u & 7) ^ (line & 7))) << 4);
+      return static_cast<uint32_t>(((u & ~7) | ((u & 7) ^ (r & 6))) << 4);
     }
   }
 };
@@ -208,6 +267,10 @@ struct DecodeSmem {
 __host__ __device__ inline int staged_block_ids(int partition_tokens, int bs_log2) {
   const int n = (partition_tokens >> bs_log2) + 2;
   return n < kBlockIdsInSmem ? n : kBlockIdsInSmem;
+}
+// ... for the longest partition a CTA of the launch may be given
+__host__ __device__ inline int staged_block_ids(const DecodeParams& p) {
+  return staged_block_ids(max(p.partition_tokens, p.max_partition_tokens), p.bs_log2);
 }
 
 // ---- per-warp attention math shared by the decode and prefix kernels -------
@@ -297,6 +360,27 @@ template <int CK, int D>
 __device__ __forceinline__ int2 accumulator_channels(int mt, int g) {
   if constexpr (CK != kE4M3) return make_int2(16 * mt + g, 16 * mt + 8 + g);
   return make_int2((D / 8) * g + 2 * mt, (D / 8) * g + 2 * mt + 1);
+}
+
+// Position of channel c of query head `head` inside its row of the warps'
+// merge buffer: c XOR a value that depends on the head and on c / 32 only,
+// so that each aligned run of 32 channels stays in place as a set (the
+// merge reads it with consecutive threads, conflict-free) while the stores
+// of the accumulators, one channel per lane from 8 lanes g x 4 heads 2t + e,
+// land in 32 distinct banks: for 16-bit caches lane g holds channel
+// 16 mt + g (+ 8), so the head goes to bits 3-4; for E4M3 lane g holds
+// channel (D / 8) g + 2 mt (+ 1), so bits 0 .. log2(D / 32) - 1 take c / 32
+// and the next two the head.
+template <int CK, int D>
+__device__ __forceinline__ int merge_pos(int head, int c) {
+  const int h2 = (head >> 1) & 3;
+  if constexpr (CK != kE4M3) {
+    return c ^ (h2 << 3);
+  } else {
+    constexpr int kBlk = D / 32;  // 2 or 4
+    constexpr int kShift = kBlk == 4 ? 2 : 1;
+    return c ^ (((c >> 5) & (kBlk - 1)) | (h2 << kShift));
+  }
 }
 
 // One 16-token tile of K and V of a 16-bit cache in shared memory (rows <
@@ -526,9 +610,14 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
 // One decode CTA: partition `part` of sequence `b`, for KV head / head group
 // `by` (= kv_head * head_groups + head_group).
 // FUSED: the launch also appends each sequence's new token (pa_append_decode).
+// PT: the launch's partition length (p.partition_tokens, or in work-list
+// mode the plan kernel's). cursor (work-list mode, else null): thread 0 takes
+// the next ticket once the main loop is done, loads its item during the
+// epilogue and moves the cursor before returning.
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED = false>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part, const int by,
-                                           const int b) {
+                                           const int b, const int PT,
+                                           WorkCursor* cursor = nullptr) {
   using S = DecodeSmem<CK, D, NW, NSTAGE>;
   using G = typename S::G;
   constexpr bool kE4 = (CK == kE4M3);
@@ -565,15 +654,19 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
       bad |= row[i] != p.block_tables[i];
     if (bad) flag_error(PA_DEVERR_PREFIX);
   }
-  const int PT = p.partition_tokens;
-  const int nparts = suffix_partitions(p, L);
-  if (part >= (nparts > 0 || p.force_partials ? nparts : 1)) return;
+  const int nparts = partitions_of(p, L, PT);
+  const bool steer = cursor != nullptr && threadIdx.x == 0;  // this thread moves the cursor
+  if (part >= (nparts > 0 || p.force_partials ? nparts : 1)) {
+    if (steer) cursor_next(p, *cursor);
+    return;
+  }
 
   TQ* out = reinterpret_cast<TQ*>(p.out);
   if (L == 0) {  // (plain mode only: a cascade launch has no partition here)
     for (int i = threadIdx.x; i < nrows * D; i += NW * 32)
       out[(static_cast<int64_t>(b) * p.num_q_heads + hq0 + i / D) * D + (i % D)] =
           from_f32<TQ>(0.f);
+    if (steer) cursor_next(p, *cursor);
     return;
   }
   const SeqSpan span = seq_span(p, L);
@@ -583,12 +676,12 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const int ntiles = (t1 - t0 + TOK - 1) / TOK;
 
   // ---- block ids of this partition -> shared memory ----------------------
-  // (up to kBlockIdsInSmem of them; a longer slice is read from global
-  // memory per row instead). Blocks before `lo` are never looked up: a
-  // sliding-window caller may have freed them.
+  // (as many as the launch staged room for, at most kBlockIdsInSmem; a
+  // longer slice is read from global memory per row instead). Blocks before
+  // `lo` are never looked up: a sliding-window caller may have freed them.
   const int bt0 = max(t0, lo) >> p.bs_log2;
   const int nbt = ((t1 - 1) >> p.bs_log2) - bt0 + 1;
-  const bool bt_in_smem = nbt <= kBlockIdsInSmem;
+  const bool bt_in_smem = nbt <= staged_block_ids(p);
   const int32_t* gbt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + bt0;
   if (bt_in_smem) {
     for (int i = threadIdx.x; i < nbt; i += NW * 32) {
@@ -651,7 +744,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   // inv_scale), as pa_append_kv does) into shared memory, for the tile that
   // holds the token and for the store at the end
   const uint32_t s_new =
-      smem_addr(smem) + S::new_rows_offset(staged_block_ids(p.partition_tokens, p.bs_log2));
+      smem_addr(smem) + S::new_rows_offset(staged_block_ids(p));
   if constexpr (FUSED && kE4) {
     if (has_new && jnew >= max(t0, lo) && jnew < t1 && threadIdx.x < 2 * G::CPR) {
       const bool is_v = threadIdx.x >= G::CPR;
@@ -802,6 +895,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     __syncwarp();  // this stage is reloaded by the next iteration
   }
   cp_async_wait<0>();
+  const int ticket = steer ? atomicAdd(p.work_count, 1) : 0;
 
   // ---- merge the warps ------------------------------------------------------
 #pragma unroll
@@ -828,8 +922,8 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           const int2 ch = accumulator_channels<CK, D>(mt, g);
-          dst[ch.x] = o[mt][nh][e];
-          dst[ch.y] = o[mt][nh][2 + e];
+          dst[merge_pos<CK, D>(head, ch.x)] = o[mt][nh][e];
+          dst[merge_pos<CK, D>(head, ch.y)] = o[mt][nh][2 + e];
         }
         if (g == 0) {
           w_m[warp * 16 + head] = m_run[nh][e];
@@ -854,6 +948,8 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   }
   __syncthreads();
 
+  // (the ticket has arrived by now; its item loads while the output is written)
+  const int2 next_item = steer ? cursor_item(p, *cursor, ticket) : make_int2(-1, -1);
   const bool direct = nparts == 1 && !p.force_partials;
   const int slot = p.part_offset + part;
   const float* vs = (CK == kE4M3) ? p.v_scale + static_cast<int64_t>(hk) * D : nullptr;
@@ -861,8 +957,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const int row = i / D;
     const int c = i - row * D;
     float acc = 0.f;
+    const int pc = merge_pos<CK, D>(row, c);
 #pragma unroll
-    for (int w = 0; w < NW; ++w) acc += r_w[w * 16 + row] * w_o[(w * 16 + row) * D + c];
+    for (int w = 0; w < NW; ++w) acc += r_w[w * 16 + row] * w_o[(w * 16 + row) * D + pc];
     float val = acc / r_stat[2 * row + 1];
     if constexpr (CK == kE4M3) val *= vs[c];
     const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + row;
@@ -876,18 +973,40 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     }
   }
   if constexpr (FUSED && CK == kE4M3) store_new_token();
+  if (steer) {
+    cursor->u = ticket;
+    cursor->item = next_item;
+  }
 }
 
-// One decode CTA of the launch: the sequence (longest first, when asked),
-// the CTA itself, and in cascade mode the wait for the prefix grid.
+// One decode CTA of the launch. Grid mode: the CTA (part, by, b) of the
+// grid, with the sequence taken longest first when asked. Work-list mode:
+// units (item u / hb, KV head group u % hb) taken from the ticket counter
+// until the list is exhausted; each computes exactly what the CTA (part, by,
+// b) of a full grid would. In cascade mode the CTA ends with the wait for the
+// prefix grid.
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
 __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
   // a kernel launched after this one as its programmatic dependent (the
   // split-K merge) may start as soon as every CTA here has started; it waits
   // for this grid's completion before reading anything
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ WorkCursor cur;
+  const bool list = p.work_items != nullptr;
+  int part = static_cast<int>(blockIdx.x);
+  int by = static_cast<int>(blockIdx.y);
   int b = static_cast<int>(blockIdx.z);
-  if (p.longest_first) {
+  if (list) {
+    // the plan kernel, this launch's programmatic predecessor, wrote the list
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) {
+      // (batch x partitions x hb < 2^31: the host checks the bound)
+      cur.n_units = min(p.work_count[1], p.batch * p.num_partitions) * units_per_item(p);
+      cur.pt = launch_partition_tokens(p);
+      cursor_next(p, cur);
+    }
+    __syncthreads();
+  } else if (p.longest_first) {
     // the sequence of rank z in decreasing attended length
     __shared__ int s_key[kOrderMaxBatch];
     __shared__ int s_pick;
@@ -903,7 +1022,30 @@ __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
     __syncthreads();
     b = s_pick;
   }
-  decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, blockIdx.x, blockIdx.y, b);
+  while (true) {
+    if (list) {
+      const int u = cur.u;
+      if (u >= cur.n_units) break;
+      b = cur.item.x;
+      part = cur.item.y;
+      by = u % units_per_item(p);
+      __syncthreads();  // every thread has read the cursor before it moves
+      if (b < 0 || b >= p.batch || part < 0 || part >= p.num_partitions ||
+          cur.pt < p.partition_tokens || cur.pt > max(p.partition_tokens, p.max_partition_tokens) ||
+          (cur.pt & 15) != 0) {
+        // not what the plan kernel wrote (the workspace was changed under the
+        // launch): nothing is read through it
+        if (threadIdx.x == 0) cursor_next(p, cur);
+        __syncthreads();
+        continue;
+      }
+    }
+    decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, part, by, b,
+                                                 list ? cur.pt : p.partition_tokens,
+                                                 list ? &cur : nullptr);
+    if (!list) break;
+    __syncthreads();  // the cursor has moved; shared memory is free again
+  }
   // cascade mode: the shared-prefix kernel runs before this one in the stream
   // with this launch as its programmatic dependent, so this grid started
   // early; it completes only after the prefix grid has, so that the merge,
@@ -911,18 +1053,130 @@ __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
   if (p.prefix_blocks > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// grid: (partitions, num_kv_heads * head_groups, batch)
+// Minimum resident CTAs per SM asked of the compiler (0: none). The
+// two-column-block decode at head_dim 128 is held to 3 CTAs per SM (at most
+// 170 registers; left alone the compiler takes up to 255 and the SM holds
+// two); the others are left to the compiler's choice, which keeps them at
+// <= 128 registers (an explicit minimum of one CTA made it take 173 for the
+// one-block 16-bit decode and cost the SM its third CTA).
+template <int CK, int D, int NH>
+constexpr int decode_min_ctas() {
+  return (D == 128 && NH == 2) ? 3 : 0;
+}
+
+// grid: (partitions, num_kv_heads * head_groups, batch), or work-list mode
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
-__global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(NW * 32, (decode_min_ctas<CK, D, NH>()))
+    pa_decode_kernel(const DecodeParams p) {
   decode_launch_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p);
 }
 
-// The same for an E4M3 cache and up to 8 query heads per KV head (no fused
-// append), held to 5 CTAs per SM (102 registers): that decode is bound by
+// The same for an E4M3 cache and up to 8 query heads per KV head, held to 5
+// CTAs per SM (at most 102 registers a thread): that decode is bound by
 // instruction latency, and the extra warps pay (measured).
-template <typename TQ, int D, int NW, int NSTAGE>
+template <typename TQ, int D, int NW, int NSTAGE, bool FUSED>
 __global__ void __launch_bounds__(NW * 32, 5) pa_decode_e4m3_kernel(const DecodeParams p) {
-  decode_launch_cta<TQ, kE4M3, D, NW, NSTAGE, 1, false>(p);
+  decode_launch_cta<TQ, kE4M3, D, NW, NSTAGE, 1, FUSED>(p);
+}
+
+// ---- work list for batches of mixed lengths --------------------------------
+//
+// In a (partitions x head groups x sequences) grid every sequence gets as
+// many partition CTAs as the longest one needs; the CTAs past a shorter
+// sequence's end exit at once but still take a slot and a dispatch each, and
+// the CTAs are dispatched in index order whatever their size, so the longest
+// may start last. One CTA of this kernel lists the (sequence, partition)
+// items instead, sorted by size (tokens of the partition) into
+// kPlanBuckets classes, largest first, so that a persistent grid taking
+// units from a counter starts the long ones first and ends on the short ones.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 64;
+
+// Size class of an item of `tiles` 16-token tiles: kPlanBuckets for a full
+// partition down to 1; 0 for an empty sequence (its item writes a zero row).
+__device__ __forceinline__ int plan_bucket(int tiles, int full_tiles) {
+  if (tiles <= 0) return 0;
+  return 1 + min(kPlanBuckets - 1, static_cast<int>(static_cast<int64_t>(tiles - 1) *
+                                                    kPlanBuckets / full_tiles));
+}
+
+__global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const DecodeParams p) {
+  __shared__ int s_hist[kPlanBuckets + 1];
+  __shared__ int s_start[kPlanBuckets + 1];
+  __shared__ unsigned long long s_work;
+  __shared__ int s_pt;
+  // the decode grid may be placed now; it waits for this grid to complete
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  for (int i = threadIdx.x; i <= kPlanBuckets; i += kPlanThreads) s_hist[i] = 0;
+  if (threadIdx.x == 0) s_work = 0;
+  __syncthreads();
+  // The partition length: the host's times 1, 2 or 4 (within the room the
+  // launch staged for block ids), the longest whose item is at most 3/4 of a
+  // slot's share of the batch's tokens x head groups. Longer partitions
+  // mean fewer units and partials; the largest items still start first.
+  {
+    unsigned long long mine = 0;
+    for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
+      const int L = clamp_context(p, p.context_lens[b]);
+      if (L > 0) mine += static_cast<unsigned long long>(L - seq_span(p, L).base);
+    }
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&s_work, mine);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned long long share =
+        s_work * static_cast<unsigned long long>(units_per_item(p)) * 3 /
+        (4ull * static_cast<unsigned long long>(max(p.list_slots, 1)));
+    int pt = p.partition_tokens;
+    const int cap = max(p.partition_tokens, p.max_partition_tokens);
+    while (2 * pt <= cap && static_cast<unsigned long long>(2 * pt) <= share) pt *= 2;
+    s_pt = pt;
+  }
+  __syncthreads();
+  const int pt = s_pt;
+  const int full_tiles = max(pt / 16, 1);
+  // items of sequence b: np partitions, all full but the last (class bk)
+  auto shape = [&](int b, int& np, int& bk) {
+    const int L = clamp_context(p, p.context_lens[b]);
+    np = partitions_of(p, L, pt);
+    if (np == 0) {  // L == 0: one item, the zero row
+      np = 1;
+      bk = 0;
+      return;
+    }
+    const int last = (L - seq_span(p, L).base) - (np - 1) * pt;
+    bk = plan_bucket((last + 15) / 16, full_tiles);
+  };
+  for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
+    int np, bk;
+    shape(b, np, bk);
+    if (np > 1) atomicAdd(&s_hist[kPlanBuckets], np - 1);
+    atomicAdd(&s_hist[bk], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int at = 0;
+    for (int k = kPlanBuckets; k >= 0; --k) {
+      s_start[k] = at;
+      at += s_hist[k];
+    }
+    p.work_count[0] = 0;   // the decode's ticket counter
+    p.work_count[1] = at;  // items
+    p.work_count[2] = pt;  // partition length
+  }
+  __syncthreads();
+  // (the order within a class is whatever the atomics give: every item is
+  // computed the same wherever it lands)
+  for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
+    int np, bk;
+    shape(b, np, bk);
+    if (np > 1) {
+      const int at = atomicAdd(&s_start[kPlanBuckets], np - 1);
+      for (int j = 0; j < np - 1; ++j) p.work_items[at + j] = make_int2(b, j);
+    }
+    p.work_items[atomicAdd(&s_start[bk], 1)] = make_int2(b, np - 1);
+  }
 }
 
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
@@ -959,7 +1213,8 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
   int nparts = 0;
   if (row < rows) {
     const int b = static_cast<int>(row / p.num_q_heads);
-    nparts = p.part_offset + suffix_partitions(p, clamp_context(p, p.context_lens[b]));
+    nparts = p.part_offset +
+             partitions_of(p, clamp_context(p, p.context_lens[b]), launch_partition_tokens(p));
   }
   const bool work = nparts > 1 || (nparts == 1 && p.force_partials);
   const bool active = lane < D / 4;

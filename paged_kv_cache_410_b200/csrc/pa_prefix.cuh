@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(NW * 32, CK == kE4M3 ? 2 : 3)
     const int part = sid % cg.n_suffix_parts;
     const int r = sid / cg.n_suffix_parts;
     const int ny = p.num_kv_heads * p.head_groups;
-    decode_cta<TQ, CK, D, NW, NSTAGE, NH>(p, part, r % ny, r / ny);
+    decode_cta<TQ, CK, D, NW, NSTAGE, NH>(p, part, r % ny, r / ny, p.partition_tokens);
   }
 }
 

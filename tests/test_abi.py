@@ -158,12 +158,15 @@ def test_workspace_plan(lib):
     d = _desc(num_kv_heads=8, head_dim=128)
     # one partition covers the context: no workspace
     assert lib.pa_decode_workspace_size(4, 64, 100, 512, ctypes.byref(d)) == 0
-    # split: partial outputs (fp32, head_dim) + (max, sum) per partition, 256-byte sections
+    # split: partial outputs (fp32, head_dim) + (max, sum) per partition, then
+    # the work list (a 256-byte counter section and one 8-byte item per
+    # partition a sequence can have), 256-byte sections
     ws = lib.pa_decode_workspace_size(4, 64, 131072, 512, ctypes.byref(d))
     parts = 131072 // 512
     o = 4 * 64 * parts * 128 * 4
     ml = 4 * 64 * parts * 8
-    assert ws == -(-o // 256) * 256 + -(-ml // 256) * 256
+    items = 4 * parts * 8
+    assert ws == -(-o // 256) * 256 + -(-ml // 256) * 256 + 256 + -(-items // 256) * 256
     # automatic partition: 128 KB of K rows per KV head (512 tokens at fp16 and
     # head_dim 128, 1024 at head_dim 64 or E4M3), halved while the grid is
     # under two CTAs per SM
@@ -369,6 +372,9 @@ def test_workspace_sizes_cover_every_partition_plan(lib):
         o, ml = batch * hq * parts * d * 4, batch * hq * parts * 8
         return -(-o // 256) * 256 + -(-ml // 256) * 256
 
+    def need_list(batch, hq, parts, d):  # plain and window decodes: + the work list
+        return need(batch, hq, parts, d) + 256 + -(-(batch * parts * 8) // 256) * 256
+
     for _ in range(400):
         hkv = int(rng.choice([1, 2, 8, 32]))
         hq = hkv * int(rng.choice([1, 2, 4, 8, 16]))
@@ -383,14 +389,14 @@ def test_workspace_sizes_cover_every_partition_plan(lib):
         assert pt >= 64 and pt % 16 == 0
         parts = max(1, -(-maxc // pt))
         ws = lib.pa_decode_workspace_size(batch, hq, maxc, 0, desc)
-        assert ws == (need(batch, hq, parts, d) if parts > 1 else 0)
+        assert ws == (need_list(batch, hq, parts, d) if parts > 1 else 0)
         # sliding window: the plan spans at most window + 15 tokens
         window = int(rng.integers(1, 10000))
         span = min(maxc, window + 15)
         ptw = lib.pa_decode_partition_tokens(batch, span, desc)
         partsw = max(1, -(-span // ptw))
         wsw = lib.pa_decode_sliding_window_workspace_size(batch, hq, maxc, window, 0, desc)
-        assert wsw == (need(batch, hq, partsw, d) if partsw > 1 else 0)
+        assert wsw == (need_list(batch, hq, partsw, d) if partsw > 1 else 0)
         # shared prefix: prefix chunks plus the suffix partitions
         pb = int(rng.integers(1, maxc // bs + 2))
         if pb * bs > maxc:
