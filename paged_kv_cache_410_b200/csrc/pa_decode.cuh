@@ -1263,8 +1263,11 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
   if (work) {
     const float2* ml = p.ws_ml + row * p.num_partitions;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
-    // global max over the row's partials (every warp of the row computes it)
+    // global max over the row's partials (every warp of the row computes it;
+    // unrolled so that a lane's loads are all in flight together rather than
+    // one L2 round trip each)
     float M = -INFINITY;
+#pragma unroll 8
     for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
