@@ -92,7 +92,7 @@ typedef struct pa_cache_desc {
   int32_t head_dim;      /* 64 or 128 */
   int32_t cache_dtype;   /* pa_dtype */
   /* E4M3 caches only (NULL otherwise): device fp32 arrays [num_kv_heads *
-   * head_dim]. A stored code c of head h, channel d stands for
+   * head_dim], 16-byte aligned (checked). A stored code c of head h, channel d stands for
    * e4m3(c) * scale[h*head_dim + d]; append stores
    * e4m3_rn_satfinite(fp32(x) * inv_scale[h*head_dim + d]). */
   const float* k_scale;

@@ -386,7 +386,8 @@ pa_status check_decode_args(const void* q, int32_t q_dtype, int32_t batch, int32
     return PA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return PA_ERR_INVALID_ARG;
-  if (cache->cache_dtype == PA_E4M3 && (!cache->k_scale || !cache->v_scale))
+  if (cache->cache_dtype == PA_E4M3 && (!cache->k_scale || !cache->v_scale ||
+                                         !aligned16(cache->k_scale) || !aligned16(cache->v_scale)))
     return PA_ERR_INVALID_ARG;
   const int group = num_q_heads / cache->num_kv_heads;
   if (static_cast<int64_t>(cache->num_kv_heads) * ((group + 15) / 16) > 65535)

@@ -93,6 +93,44 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
   }
 }
 
+// L2 eviction-priority policies, and global stores / loads that carry one:
+// data written now and read once by a later kernel (split-K partials) is
+// stored evict-last, so that a stream of other data through L2 in between
+// does not push it out, and loaded evict-first by its one reader.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_hint(float* a, float v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(a), "f"(v), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void st_hint(float2* a, float2 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;\n" ::"l"(a), "f"(v.x),
+               "f"(v.y), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ float2 ld_hint(const float2* a, uint64_t pol) {
+  float2 v;
+  asm volatile("ld.global.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;\n"
+               : "=f"(v.x), "=f"(v.y)
+               : "l"(a), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ float4 ld_hint(const float4* a, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(a), "l"(pol));
+  return v;
+}
+
 // 2^x on the SFU (ex2.approx; 2^-inf = 0).
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -320,13 +320,24 @@ __device__ __forceinline__ void load_query_e4m3(const TQ* const (&rows)[NH], con
 #pragma unroll
     for (int gq = 0; gq < D / 32; ++gq)
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = 32 * gq + 8 * t + 4 * h + i;
-          x[gq][h][i] = ok ? to_f32<TQ>(qr[c]) * ks[c] : 0.f;
-          mx = fmaxf(mx, fabsf(x[gq][h][i]));
+      for (int h = 0; h < 2; ++h) {
+        // channels c .. c + 3: one 8-byte load of q, one 16-byte load of the
+        // scales (rows and scale arrays are 16-byte aligned)
+        const int c = 32 * gq + 8 * t + 4 * h;
+        uint2 qv = make_uint2(0u, 0u);
+        float4 sv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ok) {
+          qv = *reinterpret_cast<const uint2*>(qr + c);
+          sv = *reinterpret_cast<const float4*>(ks + c);
         }
+        const TQ* qe = reinterpret_cast<const TQ*>(&qv);
+        x[gq][h][0] = to_f32<TQ>(qe[0]) * sv.x;
+        x[gq][h][1] = to_f32<TQ>(qe[1]) * sv.y;
+        x[gq][h][2] = to_f32<TQ>(qe[2]) * sv.z;
+        x[gq][h][3] = to_f32<TQ>(qe[3]) * sv.w;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fabsf(x[gq][h][i]));
+      }
     // the four threads of the group hold the row's channels between them
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -952,6 +963,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   const int2 next_item = steer ? cursor_item(p, *cursor, ticket) : make_int2(-1, -1);
   const bool direct = nparts == 1 && !p.force_partials;
   const int slot = p.part_offset + part;
+  const uint64_t keep = direct ? 0 : l2_evict_last_policy();  // partials: kept for the merge
   const float* vs = (CK == kE4M3) ? p.v_scale + static_cast<int64_t>(hk) * D : nullptr;
   for (int i = threadIdx.x; i < nrows * D; i += NW * 32) {
     const int row = i / D;
@@ -966,10 +978,10 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     if (direct) {
       out[bh * D + c] = from_f32<TQ>(val);
     } else {
-      p.ws_o[(bh * p.num_partitions + slot) * D + c] = val;
+      st_hint(p.ws_o + (bh * p.num_partitions + slot) * D + c, val, keep);
       if (c == 0)
-        p.ws_ml[bh * p.num_partitions + slot] =
-            make_float2(r_stat[2 * row], r_stat[2 * row + 1]);
+        st_hint(p.ws_ml + bh * p.num_partitions + slot,
+                make_float2(r_stat[2 * row], r_stat[2 * row + 1]), keep);
     }
   }
   if constexpr (FUSED && CK == kE4M3) store_new_token();
@@ -1225,7 +1237,8 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
     if (work) {
       const float2* ml = p.ws_ml + row * p.num_partitions;
       const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
-      const float2 mine = lane < nparts ? ml[lane] : make_float2(-INFINITY, 0.f);
+      const uint64_t once = l2_evict_first_policy();  // the partials' one reader
+      const float2 mine = lane < nparts ? ld_hint(ml + lane, once) : make_float2(-INFINITY, 0.f);
       // unconditional loads (indexes clamped to the row's partials and to
       // the row's D / 4 lanes; the clamped copies get weight 0 or are not
       // stored), so that they are all issued together
@@ -1233,7 +1246,7 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
       float4 x[NL];
 #pragma unroll
       for (int i = 0; i < NL; ++i)
-        x[i] = po[static_cast<int64_t>(min(i, nparts - 1)) * (D / 4) + lc];
+        x[i] = ld_hint(po + static_cast<int64_t>(min(i, nparts - 1)) * (D / 4) + lc, once);
       float M = mine.x;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -1263,6 +1276,7 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
   if (work) {
     const float2* ml = p.ws_ml + row * p.num_partitions;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
+    const uint64_t once = l2_evict_first_policy();  // the partials' last reads
     // global max over the row's partials (every warp of the row computes it;
     // unrolled so that a lane's loads are all in flight together rather than
     // one L2 round trip each)
@@ -1278,7 +1292,7 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
       const float w = v.y * ex2(v.x - M);
       wsum += w;
       if (active) {
-        const float4 x = po[static_cast<int64_t>(i) * (D / 4) + lane];
+        const float4 x = ld_hint(po + static_cast<int64_t>(i) * (D / 4) + lane, once);
         acc.x += w * x.x;
         acc.y += w * x.y;
         acc.z += w * x.z;
