@@ -69,11 +69,17 @@ int64_t elem_bytes(int dtype) { return dtype == PA_E4M3 ? 1 : 2; }
 // or head_dim 64), halved (down to 64) while the launch would have fewer
 // than two CTAs per SM. When the sequences alone are fewer than one wave of
 // CTAs (batch x KV heads below kWaveCtas, so the split is what fills the
-// GPU: long contexts at small batch), the partition is then lengthened to
-// the shortest multiple of 16 tokens whose CTAs make whole waves: of equal
-// CTAs, a last partial wave costs as long as a full one.
+// GPU: long contexts at small batch), the partition is then lengthened so
+// that the CTAs make whole waves: of equal CTAs, a last partial wave costs
+// as long as a full one. Several sequences (a work-list launch, whose plan
+// may lengthen the partitions further) take the shortest such length; a
+// single sequence (a grid launch) takes the fewest waves whose partitions
+// stay within kMaxWavePartition tokens -- one wave where it can: measured
+// on the 131072-token context at batch 1, one wave of 440 CTAs read 0.834
+// of the copy bandwidth, two waves 0.814, four waves 0.792.
 constexpr int kDecodeCtasPerSm = 3;  // decode CTAs resident per SM at head_dim 128
 constexpr int64_t kWaveCtas = int64_t{kDecodeCtasPerSm} * kNumSMs;
+constexpr int64_t kMaxWavePartition = 8192;
 
 int auto_partition(int64_t batch, int64_t max_context, const pa_cache_desc* cd) {
   int pt = kPartitionRowBytes / static_cast<int>(cd->head_dim * elem_bytes(cd->cache_dtype));
@@ -83,9 +89,13 @@ int auto_partition(int64_t batch, int64_t max_context, const pa_cache_desc* cd) 
   if (cd->head_dim == 128 && rows > 0 && rows < kWaveCtas) {
     const int64_t waves = ctas(pt) / kWaveCtas;
     if (waves >= 1 && ctas(pt) % kWaveCtas != 0) {
-      const int64_t parts = waves * kWaveCtas / rows;  // partitions per row in whole waves
-      const int64_t pt2 = ((max_context + parts - 1) / parts + 15) / 16 * 16;
-      if (pt2 <= (int64_t{1} << 20) && ctas(pt2) <= waves * kWaveCtas) pt = static_cast<int>(pt2);
+      for (int64_t w = batch == 1 ? 1 : waves; w <= waves; ++w) {
+        const int64_t parts = w * kWaveCtas / rows;  // partitions per row in w whole waves
+        const int64_t pt2 = ((max_context + parts - 1) / parts + 15) / 16 * 16;
+        if (w < waves && pt2 > kMaxWavePartition) continue;
+        if (pt2 <= (int64_t{1} << 20) && ctas(pt2) <= w * kWaveCtas) pt = static_cast<int>(pt2);
+        break;
+      }
     }
   }
   return pt;

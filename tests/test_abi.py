@@ -183,11 +183,13 @@ def test_workspace_plan(lib):
 
 def test_small_batches_split_into_whole_waves(lib):
     """With fewer (sequence, KV head) pairs than one wave of decode CTAs (3 per
-    SM on 148 SMs), the automatic partition is lengthened to the shortest
-    multiple of 16 tokens whose CTAs fill whole waves."""
+    SM on 148 SMs), the automatic partition is lengthened so that the CTAs
+    fill whole waves: for several sequences the shortest multiple of 16
+    tokens that keeps the 512-token plan's whole waves, for a single sequence
+    the fewest waves whose partitions stay within 8192 tokens."""
     waves_of = 3 * 148
     d = _desc(num_kv_heads=8, head_dim=128, cache_dtype=B.PA_BF16)
-    for batch, ctx, want in ((1, 131072, 592), (4, 131072, 528), (2, 20000, 752)):
+    for batch, ctx, want in ((4, 131072, 528), (2, 20000, 752)):
         pt = lib.pa_decode_partition_tokens(batch, ctx, ctypes.byref(d))
         assert pt == want, (batch, ctx, pt)
         ctas = batch * 8 * -(-ctx // pt)
@@ -195,6 +197,19 @@ def test_small_batches_split_into_whole_waves(lib):
         assert ctas <= full * waves_of and pt % 16 == 0
         # 16 tokens shorter would need one more (partial) wave
         assert batch * 8 * -(-ctx // (pt - 16)) > full * waves_of
+    # one sequence: a single wave of 440 CTAs (55 partitions of 2384 tokens)...
+    pt = lib.pa_decode_partition_tokens(1, 131072, ctypes.byref(d))
+    assert pt == 2384 and 8 * -(-131072 // pt) <= waves_of
+    assert 8 * -(-131072 // (pt - 16)) > waves_of
+    # ... or, when one wave would need partitions over 8192 tokens, the fewest
+    # whole waves that do not (2^20 tokens: 3 waves of 166 partitions)
+    ctx = 1 << 20
+    pt = lib.pa_decode_partition_tokens(1, ctx, ctypes.byref(d))
+    def within(w):  # the partition that fills w whole waves, rounded up to 16 tokens
+        per = -(-ctx // (w * waves_of // 8))
+        return (per + 15) // 16 * 16
+    assert within(1) > 8192 and within(2) > 8192 and pt == within(3) <= 8192
+    assert 8 * -(-ctx // pt) <= 3 * waves_of
     # a batch that fills the GPU by itself keeps the byte rule
     d32 = _desc(num_kv_heads=32, head_dim=128)
     assert lib.pa_decode_partition_tokens(64, 4096, ctypes.byref(d32)) == 512
