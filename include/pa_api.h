@@ -336,6 +336,22 @@ pa_status pa_decode_static_workspace(const void* q, int32_t q_dtype, int32_t bat
                                      float scale, void* out, int32_t partition_tokens,
                                      void* stream);
 
+/* Reproducible results (process-wide, any thread; 0 at load). With 0, a
+ * pa_decode, pa_decode_static_workspace or pa_decode_sliding_window call on
+ * one sequence (batch == 1) over a 16-bit cache with blocks of 16 tokens or
+ * more, whose plan splits it into partitions of 1024 tokens or more, runs in
+ * steal mode: the CTAs of each KV head group take the sequence's tiles in
+ * chunks from a counter in the workspace instead of each reading a fixed
+ * partition, so that no CTA on a slower SM holds up the call. Which CTA
+ * combines which tiles then varies from call to call, and so may the last
+ * bits of the output (every result is within the same rounding of the
+ * split-K merge). With 1, no call uses steal mode, and a call repeated with
+ * the same inputs, sizes and partition length gives the same bits; every
+ * other decode is reproducible in either setting. The switch is read when a
+ * call is made (a captured launch keeps its mode). Returns the previous
+ * setting. */
+int32_t pa_set_deterministic(int32_t on);
+
 /* Static text for a status code. */
 const char* pa_status_string(int32_t status);
 

@@ -32,7 +32,8 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
             "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
             "pa_append_decode", "pa_copy_blocks_layers",
-            "pa_decode_shared_prefix_partition_tokens", "pa_testing_withhold_prefix_scores"]
+            "pa_decode_shared_prefix_partition_tokens", "pa_testing_withhold_prefix_scores",
+            "pa_set_deterministic"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -80,6 +81,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
     lib.pa_version.restype = i32
+    lib.pa_set_deterministic.argtypes = [i32]
+    lib.pa_set_deterministic.restype = i32
     lib.pa_decode_static_workspace.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32,
                                                ctypes.c_float, P, i32, P]
     lib.pa_decode_static_workspace.restype = ctypes.c_int
@@ -408,3 +411,22 @@ def pa_status_string(status: int) -> str:
 
 def pa_version() -> int:
     return int(load_library().pa_version())
+
+
+def pa_set_deterministic(on: bool) -> bool:
+    """Reproducible results on (no steal mode for single-sequence split
+    decodes) or off (the default); returns the previous setting."""
+    return bool(load_library().pa_set_deterministic(1 if on else 0))
+
+
+class deterministic:
+    """``with deterministic():`` runs its body with reproducible results on
+    and puts the previous setting back after."""
+
+    def __enter__(self):
+        self.prev = pa_set_deterministic(True)
+        return self
+
+    def __exit__(self, *exc):
+        pa_set_deterministic(self.prev)
+        return False

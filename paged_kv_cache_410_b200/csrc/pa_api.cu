@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <array>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -242,6 +243,42 @@ bool use_work_list(const pa::DecodeParams& p, bool dependent) {
              (int64_t{1} << 31);
 }
 
+// Steal mode (a single sequence's split decode over a 16-bit cache with
+// blocks of 16 tokens or more and partitions of kStealMinPartition tokens or
+// more, unless the caller asked for reproducible results): the CTAs of each
+// KV head group share the sequence's tiles through a counter per group, so
+// that CTAs on slower SMs take fewer tiles instead of setting the launch's
+// end. Shorter partitions keep their fixed split: the claims' latency would
+// cost more than the balance gains. The counters sit in the work list's
+// section of the workspace (256 bytes, then 8 per partition; 8 bytes a
+// counter), and a counter's claimed-tile field (kStealCountBits wide) must
+// hold the tiles plus one overshooting chunk per warp.
+constexpr int kStealMinPartition = 1024;
+std::atomic<int> g_deterministic{0};
+
+bool use_steal(const pa::DecodeParams& p, int grid_x, bool dependent) {
+  const int64_t hb = static_cast<int64_t>(p.num_kv_heads) * p.head_groups;
+  const int64_t list_bytes = 256 + (static_cast<int64_t>(p.num_partitions) * 8 + 255) / 256 * 256;
+  const int64_t most_claimed = static_cast<int64_t>(p.max_context) / 16 + 1 +
+                               static_cast<int64_t>(p.num_partitions) * kDecodeWarps *
+                                   pa::kStealChunk + pa::kStealChunk;
+  return g_deterministic.load(std::memory_order_relaxed) == 0 && !dependent &&
+         p.prefix_blocks == 0 && !p.k_new && p.work_count && p.batch == 1 &&
+         p.num_partitions > 1 && p.partition_tokens >= kStealMinPartition &&
+         grid_x == p.num_partitions && p.part_offset == 0 &&
+         !p.force_partials && p.bs_log2 >= 4 && hb * 8 <= list_bytes &&
+         most_claimed < (int64_t{1} << pa::kStealCountBits);
+}
+
+// A fresh steal epoch per launch (bit 62 set, the call count above the
+// claimed-tile field).
+unsigned long long next_steal_epoch() {
+  static std::atomic<unsigned long long> calls{0};
+  const unsigned long long n = (calls.fetch_add(1, std::memory_order_relaxed) + 1) &
+                               ((1ull << (62 - pa::kStealCountBits)) - 1);
+  return (1ull << 62) | (n << pa::kStealCountBits);
+}
+
 // CTAs of `kern` resident per SM at this block and shared-memory size, and
 // the device's SM count (cached per kernel, size and device).
 cudaError_t resident_ctas(const void* kern, int threads, int smem, int* per_sm, int* sms) {
@@ -295,6 +332,15 @@ pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t
                       : pa::pa_decode_e4m3_kernel<TQ, D, kDecodeWarps, kDecodeStages, false>;
   pa::DecodeParams p = p_in;
   const bool list = use_work_list(p, dependent);
+  p.steal_ctr = nullptr;
+  p.steal_epoch = 0;
+  if constexpr (CK != pa::kE4M3) {
+    if (!list && use_steal(p, grid_x, dependent)) {
+      kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false, true>;
+      p.steal_ctr = reinterpret_cast<unsigned long long*>(p.work_count);
+      p.steal_epoch = next_steal_epoch();
+    }
+  }
   if (list) {
     // the plan kernel may lengthen the partitions up to this
     p.max_partition_tokens = static_cast<int>(
@@ -707,6 +753,10 @@ const char* pa_status_string(int32_t s) {
 }
 
 int32_t pa_version(void) { return 100; }
+
+int32_t pa_set_deterministic(int32_t on) {
+  return g_deterministic.exchange(on != 0 ? 1 : 0);
+}
 
 void pa_testing_withhold_prefix_scores(int32_t on) {
   std::lock_guard<std::mutex> lock(g_hook_mu);

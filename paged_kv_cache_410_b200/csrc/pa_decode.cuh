@@ -104,7 +104,48 @@ struct DecodeParams {
   // partition_tokens).
   int list_slots;
   int max_partition_tokens;
+  // Steal mode (null: none; a single sequence's split decode): the CTAs of a
+  // (sequence, KV head group) row share its tiles instead of each taking one
+  // partition. Their warps claim chunks of kStealChunk tiles from
+  // steal_ctr[row], a 64-bit counter whose bits from kStealCountBits up hold
+  // the call's epoch (steal_epoch, already shifted; bit 62 always set, which
+  // a work-list item, two non-negative ints, never has) and the low bits the
+  // tiles claimed so far; each CTA still writes the one partial of its
+  // partition column, and the merge zeroes the counters.
+  unsigned long long* steal_ctr;
+  unsigned long long steal_epoch;
 };
+
+constexpr int kStealChunk = 4;
+constexpr int kStealCountBits = 24;
+
+// The first of n tiles newly claimed from a steal counter (one thread; n = 0
+// only installs this launch's epoch). A counter of another epoch (an earlier
+// call's, or bytes a workspace held before) is replaced by (epoch, n) with a
+// compare-and-swap from the exact value last seen; a swap fails only when
+// another claimant changed the counter in between, by its own first add of
+// the launch (at most one per warp) or by installing the epoch, after which
+// the counter only grows. The retries are bounded all the same: after
+// kStealMaxRounds the claim gives up (claims nothing, flags
+// PA_DEVERR_TIMEOUT).
+constexpr int kStealMaxRounds = 1 << 20;
+__device__ __forceinline__ int steal_claim(unsigned long long* ctr, unsigned long long epoch,
+                                           int n) {
+  const unsigned long long mask = (1ull << kStealCountBits) - 1;
+  const unsigned long long add = static_cast<unsigned long long>(n);
+  unsigned long long v = atomicAdd(ctr, add);
+  if ((v & ~mask) == epoch) return static_cast<int>(v & mask);
+  v += add;  // what this add left behind
+  for (int round = 0; round < kStealMaxRounds; ++round) {
+    const unsigned long long seen = atomicCAS(ctr, v, epoch | add);
+    if (seen == v) return 0;
+    if ((seen & ~mask) == epoch)  // installed by another claimant
+      return static_cast<int>(atomicAdd(ctr, add) & mask);
+    v = seen;
+  }
+  flag_error(PA_DEVERR_TIMEOUT);
+  return 1 << 30;
+}
 
 constexpr int kOrderMaxBatch = 256;
 
@@ -625,7 +666,10 @@ __device__ __forceinline__ void attend_tile_e4m3(uint32_t sk_a, uint32_t sv_a, i
 // mode the plan kernel's). cursor (work-list mode, else null): thread 0 takes
 // the next ticket once the main loop is done, loads its item during the
 // epilogue and moves the cursor before returning.
-template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED = false>
+// STEAL: steal mode (p.steal_ctr set; 16-bit caches with blocks of 16 tokens
+// or more, one head group per KV head, no fused append, grid mode).
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED = false,
+          bool STEAL = false>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part, const int by,
                                            const int b, const int PT,
                                            WorkCursor* cursor = nullptr) {
@@ -682,8 +726,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   }
   const SeqSpan span = seq_span(p, L);
   const int lo = span.lo;  // first attended token
-  const int t0 = span.base + part * PT;
-  const int t1 = min(t0 + PT, L);
+  // the partition; in steal mode the row's whole attended range
+  const int t0 = STEAL ? span.base : span.base + part * PT;
+  const int t1 = STEAL ? L : min(t0 + PT, L);
   const int ntiles = (t1 - t0 + TOK - 1) / TOK;
 
   // ---- block ids of this partition -> shared memory ----------------------
@@ -692,7 +737,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
   // `lo` are never looked up: a sliding-window caller may have freed them.
   const int bt0 = max(t0, lo) >> p.bs_log2;
   const int nbt = ((t1 - 1) >> p.bs_log2) - bt0 + 1;
-  const bool bt_in_smem = nbt <= staged_block_ids(p);
+  const bool bt_in_smem = !STEAL && nbt <= staged_block_ids(p);
   const int32_t* gbt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq + bt0;
   if (bt_in_smem) {
     for (int i = threadIdx.x; i < nbt; i += NW * 32) {
@@ -824,12 +869,15 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     cp_async_16(sk_a + so, kc + off, ok ? 16u : 0u);
     cp_async_16(sv_a + so, vc + off, ok ? 16u : 0u);
   };
-  auto load_tile = [&](int tile, int stage) {
+  // (blk_given: the tile's block id where the caller has it already, as in
+  // steal mode; kLookUp: look it up here)
+  constexpr int kLookUp = -2;
+  auto load_tile = [&](int tile, int stage, int blk_given) {
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
     const int tb = t0 + tile * TOK;
     if (block_aligned) {
-      const int blk = block_id((tb >> p.bs_log2) - bt0);
+      const int blk = blk_given != kLookUp ? blk_given : block_id((tb >> p.bs_log2) - bt0);
       const int64_t base =
           ((static_cast<int64_t>(blk) << p.bs_log2) + (tb & bs_mask) + lrow) * slot_stride +
           lane_goff;
@@ -868,29 +916,13 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     l_run[nh][0] = l_run[nh][1] = 0.f;
   }
 
-  const int my_tiles = warp < ntiles ? (ntiles - warp + NW - 1) / NW : 0;
-#pragma unroll
-  for (int s = 0; s < NSTAGE - 1; ++s) {
-    if (s < my_tiles) load_tile(warp + s * NW, s);
-    cp_async_commit();
-  }
-
-  for (int it = 0; it < my_tiles; ++it) {
-    {
-      const int nxt = it + NSTAGE - 1;
-      if (nxt < my_tiles) load_tile(warp + nxt * NW, nxt % NSTAGE);
-      cp_async_commit();
-    }
-    cp_async_wait<NSTAGE - 1>();
-    __syncwarp();
-
-    const int stage = it % NSTAGE;
+  // One tile from pipeline stage `stage` into the warp's running state.
+  auto attend = [&](int tile, int stage) {
     const uint32_t sk_a = smem_addr(wbuf + stage * S::kStageBytes);
     const uint32_t sv_a = sk_a + G::TB;
-    const int tile = warp + it * NW;
     const int ts = t0 + tile * TOK;
-    const int nvalid = t1 - ts;                // rows of the tile below the end (>= 1)
-    const int nskip = max(lo - ts, 0);         // rows before the window (first tile only)
+    const int nvalid = t1 - ts;         // rows of the tile below the end (>= 1)
+    const int nskip = max(lo - ts, 0);  // rows before the window (first tile only)
     if constexpr (kE4) {
       if (nvalid >= TOK && nskip == 0)
         attend_tile_e4m3<D, NH, true>(sk_a, sv_a, nvalid, 0, sl2, qb, o, m_run, l_run);
@@ -903,7 +935,105 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
         attend_tile<CK, D, NH, false>(sk_a, sv_a, nvalid, nskip, p.scale_log2, qb, o, m_run,
                                       l_run);
     }
-    __syncwarp();  // this stage is reloaded by the next iteration
+  };
+
+  if constexpr (!STEAL) {
+    // the warp's tiles: warp, warp + NW, ... of the partition
+    const int my_tiles = warp < ntiles ? (ntiles - warp + NW - 1) / NW : 0;
+#pragma unroll
+    for (int s = 0; s < NSTAGE - 1; ++s) {
+      if (s < my_tiles) load_tile(warp + s * NW, s, kLookUp);
+      cp_async_commit();
+    }
+    for (int it = 0; it < my_tiles; ++it) {
+      {
+        const int nxt = it + NSTAGE - 1;
+        if (nxt < my_tiles) load_tile(warp + nxt * NW, nxt % NSTAGE, kLookUp);
+        cp_async_commit();
+      }
+      cp_async_wait<NSTAGE - 1>();
+      __syncwarp();
+      attend(warp + it * NW, it % NSTAGE);
+      __syncwarp();  // this stage is reloaded by the next iteration
+    }
+  } else {
+    // The row's tiles in chunks of kStealChunk: first each CTA's own share
+    // (about half the row split evenly, its chunks round robin over the
+    // warps), then a pool of the rest that the warps of all the row's CTAs
+    // claim chunk by chunk from the counter, so that CTAs which finish their
+    // share early take more of it. The shares keep the claims away from the
+    // launch's first microseconds, when every warp of the row would contend
+    // on the counter, and the row's first CTA installs the launch's epoch
+    // meanwhile. A warp works one chunk while the next one's block ids load
+    // (its first lanes read them when the chunk is chosen).
+    unsigned long long* ctr =
+        p.steal_ctr + (static_cast<int64_t>(b) * p.num_kv_heads * p.head_groups + by);
+    const int share = ((ntiles / 2) / nparts) & ~(kStealChunk * NW - 1);
+    const int share_chunks = share / (kStealChunk * NW);  // per warp
+    const int pool = nparts * share;                       // first tile of the pool
+    if (part == 0 && threadIdx.x == 0) steal_claim(ctr, p.steal_epoch, 0);
+    int k_share = 0;
+    // first tile of the warp's next chunk (>= ntiles: none left), and the
+    // chunk's block ids in lanes 0 .. kStealChunk - 1
+    auto next_chunk = [&](int& id) -> int {
+      int c;
+      if (k_share < share_chunks) {
+        c = part * share + (k_share++ * NW + warp) * kStealChunk;
+      } else {
+        int off = 0;
+        if (lane == 0) off = steal_claim(ctr, p.steal_epoch, kStealChunk);
+        c = pool + __shfl_sync(0xffffffffu, off, 0);
+      }
+      id = -1;
+      if (lane < kStealChunk && c + lane < ntiles)
+        id = block_id(((t0 + (c + lane) * TOK) >> p.bs_log2) - bt0);
+      return c;
+    };
+    int id_cur = -1, id_nxt = -1;  // block id of tile (chunk + lane), lanes < kStealChunk
+    int c_cur = next_chunk(id_cur);                           // current chunk
+    int c_nxt = c_cur < ntiles ? next_chunk(id_nxt) : c_cur;  // next chunk
+    int c_k = 0;  // tiles of the current chunk handed out
+    // the warp's next tile (-1: none left) and its block id
+    auto next_tile = [&](int& blk) -> int {
+      while (c_cur < ntiles) {
+        if (c_k < kStealChunk && c_cur + c_k < ntiles) {
+          blk = __shfl_sync(0xffffffffu, id_cur, c_k);
+          return c_cur + c_k++;
+        }
+        c_cur = c_nxt;
+        id_cur = id_nxt;
+        c_k = 0;
+        if (c_cur < ntiles) c_nxt = next_chunk(id_nxt);
+      }
+      blk = -1;
+      return -1;
+    };
+    // tiles loaded ahead, in order (pend[0]: the next iteration's)
+    int pend[NSTAGE - 1], pblk[NSTAGE - 1];
+#pragma unroll
+    for (int s = 0; s < NSTAGE - 1; ++s) {
+      pend[s] = next_tile(pblk[s]);
+      if (pend[s] >= 0) load_tile(pend[s], s, pblk[s]);
+      cp_async_commit();
+    }
+    for (int it = 0; pend[0] >= 0; ++it) {
+      const int tile = pend[0];
+#pragma unroll
+      for (int s = 0; s + 1 < NSTAGE - 1; ++s) {
+        pend[s] = pend[s + 1];
+        pblk[s] = pblk[s + 1];
+      }
+      {
+        int& nt = pend[NSTAGE - 2];
+        nt = next_tile(pblk[NSTAGE - 2]);
+        if (nt >= 0) load_tile(nt, (it + NSTAGE - 1) % NSTAGE, pblk[NSTAGE - 2]);
+        cp_async_commit();
+      }
+      cp_async_wait<NSTAGE - 1>();
+      __syncwarp();
+      attend(tile, it % NSTAGE);
+      __syncwarp();  // this stage is reloaded by the next iteration
+    }
   }
   cp_async_wait<0>();
   const int ticket = steer ? atomicAdd(p.work_count, 1) : 0;
@@ -972,7 +1102,8 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const int pc = merge_pos<CK, D>(row, c);
 #pragma unroll
     for (int w = 0; w < NW; ++w) acc += r_w[w * 16 + row] * w_o[(w * 16 + row) * D + pc];
-    float val = acc / r_stat[2 * row + 1];
+    const float lsum_row = r_stat[2 * row + 1];  // 0: a steal-mode CTA that got no tile
+    float val = lsum_row > 0.f ? acc / lsum_row : 0.f;
     if constexpr (CK == kE4M3) val *= vs[c];
     const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + row;
     if (direct) {
@@ -997,7 +1128,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 // until the list is exhausted; each computes exactly what the CTA (part, by,
 // b) of a full grid would. In cascade mode the CTA ends with the wait for the
 // prefix grid.
-template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED, bool STEAL = false>
 __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
   // a kernel launched after this one as its programmatic dependent (the
   // split-K merge) may start as soon as every CTA here has started; it waits
@@ -1052,7 +1183,7 @@ __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
         continue;
       }
     }
-    decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p, part, by, b,
+    decode_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED, STEAL>(p, part, by, b,
                                                  list ? cur.pt : p.partition_tokens,
                                                  list ? &cur : nullptr);
     if (!list) break;
@@ -1077,10 +1208,11 @@ constexpr int decode_min_ctas() {
 }
 
 // grid: (partitions, num_kv_heads * head_groups, batch), or work-list mode
-template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED>
+// (STEAL: steal mode, a grid over one sequence)
+template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED, bool STEAL = false>
 __global__ void __launch_bounds__(NW * 32, (decode_min_ctas<CK, D, NH>()))
     pa_decode_kernel(const DecodeParams p) {
-  decode_launch_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED>(p);
+  decode_launch_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED, STEAL>(p);
 }
 
 // The same for an E4M3 cache and up to 8 query heads per KV head, held to 5
@@ -1212,6 +1344,12 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
   static_assert(NWARPS % WPR == 0, "whole rows per CTA");
   constexpr int RPC = NWARPS / WPR;  // rows per CTA
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (p.steal_ctr && blockIdx.x == 0) {
+    // the decode grid has completed: its steal counters go back to zero, so
+    // that a replay of the same launch (same epoch) starts afresh
+    const int n = p.batch * p.num_kv_heads * p.head_groups;
+    for (int i = threadIdx.x; i < n; i += NWARPS * 32) p.steal_ctr[i] = 0ull;
+  }
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int rloc = warp / WPR;

@@ -421,3 +421,14 @@ def test_workspace_sizes_cover_every_partition_plan(lib):
         sparts = -(-(maxc - pb * bs) // pts)
         wss = lib.pa_decode_shared_prefix_workspace_size(batch, hq, maxc, pb, 0, desc)
         assert wss >= need(batch, hq, 1 + sparts, d)
+
+
+def test_reproducible_results_switch(lib):
+    # a process-wide host setting, read by each decode call; off at load
+    prev = B.pa_set_deterministic(True)
+    assert prev is False
+    assert B.pa_set_deterministic(True) is True
+    assert B.pa_set_deterministic(False) is True
+    with B.deterministic():
+        assert lib.pa_set_deterministic(1) == 1
+    assert B.pa_set_deterministic(False) is False

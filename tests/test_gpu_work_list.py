@@ -8,7 +8,8 @@ with the same sequence decoded alone (a batch of one keeps the full grid)
 with the partition length the plan kernel chose (read back from the
 workspace, where the plan publishes it: 1, 2 or 4 times the host's) and a
 plan of as many partitions as the batch's launch had, so that the merge
-runs the same code."""
+runs the same code. The decodes alone ask for reproducible results, which
+keeps each CTA on its own partition (no steal mode)."""
 import numpy as np
 import pytest
 import torch
@@ -66,6 +67,8 @@ def listed_vs_alone(w, pt, window=0, fused=False, repeats=2):
               B.pa_decode_workspace_size(1, w.num_q_heads, maxc_one, step.cache, pt_used))
     wsb = torch.empty(max(ws_one, 1), dtype=torch.uint8, device="cuda")
     one = torch.empty_like(step.out[:1])
+    det = B.deterministic()
+    det.__enter__()
     for b in range(w.batch):
         one.fill_(float("nan"))
         args = (step.q[b:b + 1], step.k_cache, step.v_cache, step.block_tables[b:b + 1],
@@ -76,7 +79,10 @@ def listed_vs_alone(w, pt, window=0, fused=False, repeats=2):
         else:
             B.pa_decode(*args, pt_used, wsb if ws_one else None, step.stream)
         torch.cuda.synchronize()
-        assert np.array_equal(to_bits(one)[0], bits[b]), f"sequence {b} differs from its decode alone"
+        if not np.array_equal(to_bits(one)[0], bits[b]):
+            det.__exit__(None, None, None)
+            raise AssertionError(f"sequence {b} differs from its decode alone")
+    det.__exit__(None, None, None)
     assert step.device_errors() == 0
     return step, pt_used
 
