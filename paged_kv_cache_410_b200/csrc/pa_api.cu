@@ -221,10 +221,14 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   // hundred CTAs that all start at once
   if (n <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32>, 32, 32);
   if (n <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32>, 32, 32);
-  if (n <= 48) return go(pa::pa_decode_reduce_kernel<TQ, D, 2, 16, 8>, 8, 4);
-  if (n <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 16, 8>, 8, 2);
+  // several warps per row: at most 8 partials a warp up to 128 partials, 16
+  // up to 256; beyond, 32 warps take batches of 8 each (1024 threads leave a
+  // thread 64 registers)
+  if (n <= 32) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 8, 16>, 16, 4);
+  if (n <= 64) return go(pa::pa_decode_reduce_kernel<TQ, D, 8, 8, 16>, 16, 2);
+  if (n <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 8, 16>, 16, 1);
   if (n <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16>, 16, 1);
-  return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 16, 32>, 32, 1);
+  return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 8, 32>, 32, 1);
 }
 
 // Work-list mode (plain, fused and sliding-window decodes of a batch split

@@ -1329,12 +1329,13 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 //
 // A CTA has NWARPS warps; WPR warps merge one (sequence, query head) row, so
 // a CTA covers NWARPS / WPR rows (the host picks WPR from the number of
-// partials: few partials, several rows per CTA; many partials, up to 32
-// warps per row). Within a warp, lanes read 32 partials' (max, sum) at a
-// time for the global max, then the warp walks its share of the partials:
-// lane l owns channels 4l .. 4l+3 (float4 loads of the partial outputs); the
-// WPR warps' sums are added in shared memory. With one warp per row (at most
-// NL partials) every load is issued before any is used.
+// partials so that a warp has at most NL of them, up to 32 warps per row).
+// Lane l owns channels 4l .. 4l+3 (float4 loads of the partial outputs).
+// With one warp per row, the lanes hold the row's (max, sum) pairs and every
+// load is issued before any is used. With several, each warp loads its
+// partials' pairs and outputs together, weights them by its own max, and the
+// WPR warps' sums are rescaled to the row's max and added in shared memory:
+// the partials arrive in one round trip either way.
 //
 // The kernel is launched as the programmatic dependent of the kernels that
 // write the partials: it waits for them to complete before reading.
@@ -1359,6 +1360,7 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
 
   __shared__ float4 s_acc[NWARPS][D / 4];
   __shared__ float s_wsum[NWARPS];
+  __shared__ float s_max[NWARPS];
 
   int nparts = 0;
   if (row < rows) {
@@ -1411,47 +1413,77 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
     }
     return;
   }
+  float mw = -INFINITY;  // this warp's max over its partials
   if (work) {
     const float2* ml = p.ws_ml + row * p.num_partitions;
     const float4* po = reinterpret_cast<const float4*>(p.ws_o + row * p.num_partitions * D);
     const uint64_t once = l2_evict_first_policy();  // the partials' last reads
-    // global max over the row's partials (every warp of the row computes it;
-    // unrolled so that a lane's loads are all in flight together rather than
-    // one L2 round trip each)
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
+    const int lc = active ? lane : D / 4 - 1;
+    // this warp's partials wsub, wsub + WPR, ..., NL of them at a time: all
+    // loads of a batch are issued before any is used (the row may have fewer
+    // partials than the launch's plan: those past its count are not read and
+    // get weight 0), and the batch is weighted by the warp's own running max,
+    // so that the partials' (max, sum) pairs and outputs arrive in one round
+    // trip
+    for (int i0 = wsub; i0 < nparts; i0 += NL * WPR) {
+      float2 mk[NL];
+      float4 xk[NL];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    // this warp's partials: wsub, wsub + WPR, ...
-#pragma unroll 8
-    for (int i = wsub; i < nparts; i += WPR) {
-      const float2 v = ml[i];  // the same address in every lane: one broadcast load
-      const float w = v.y * ex2(v.x - M);
-      wsum += w;
-      if (active) {
-        const float4 x = ld_hint(po + static_cast<int64_t>(i) * (D / 4) + lane, once);
-        acc.x += w * x.x;
-        acc.y += w * x.y;
-        acc.z += w * x.z;
-        acc.w += w * x.w;
+      for (int k = 0; k < NL; ++k) {
+        const int i = i0 + k * WPR;
+        mk[k] = make_float2(-INFINITY, 0.f);
+        xk[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < nparts) {
+          mk[k] = ld_hint(ml + i, once);
+          xk[k] = ld_hint(po + static_cast<int64_t>(i) * (D / 4) + lc, once);
+        }
+      }
+      float mb = mw;
+#pragma unroll
+      for (int k = 0; k < NL; ++k) mb = fmaxf(mb, mk[k].x);
+      // rescale what the earlier batches summed to the new max
+      const float r = (mw == -INFINITY) ? 0.f : ex2(mw - mb);
+      acc.x *= r;
+      acc.y *= r;
+      acc.z *= r;
+      acc.w *= r;
+      wsum *= r;
+      mw = mb;
+#pragma unroll
+      for (int k = 0; k < NL; ++k) {
+        // (an empty partial has max -inf and sum 0: weight 0)
+        const float w = mk[k].x != -INFINITY ? mk[k].y * ex2(mk[k].x - mb) : 0.f;
+        wsum += w;
+        acc.x += w * xk[k].x;
+        acc.y += w * xk[k].y;
+        acc.z += w * xk[k].z;
+        acc.w += w * xk[k].w;
       }
     }
   }
   if (active) s_acc[warp][lane] = acc;
-  if (lane == 0) s_wsum[warp] = wsum;
+  if (lane == 0) {
+    s_wsum[warp] = wsum;
+    s_max[warp] = mw;
+  }
   __syncthreads();
   if (work && wsub == 0 && active) {
-    float4 a = s_acc[warp][lane];
-    float ws = s_wsum[warp];
+    // the row's WPR warps, each scaled from its own max to the row's
+    float M = s_max[warp];
 #pragma unroll
-    for (int k = 1; k < WPR; ++k) {
+    for (int k = 1; k < WPR; ++k) M = fmaxf(M, s_max[warp + k]);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ws = 0.f;
+#pragma unroll
+    for (int k = 0; k < WPR; ++k) {
+      const float mk = s_max[warp + k];
+      const float r = (mk == -INFINITY) ? 0.f : ex2(mk - M);
       const float4 b4 = s_acc[warp + k][lane];
-      a.x += b4.x;
-      a.y += b4.y;
-      a.z += b4.z;
-      a.w += b4.w;
-      ws += s_wsum[warp + k];
+      a.x += r * b4.x;
+      a.y += r * b4.y;
+      a.z += r * b4.z;
+      a.w += r * b4.w;
+      ws += r * s_wsum[warp + k];
     }
     TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
     const float inv = 1.f / ws;
