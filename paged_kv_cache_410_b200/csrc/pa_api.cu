@@ -338,6 +338,7 @@ pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t
   const bool list = use_work_list(p, dependent);
   p.steal_ctr = nullptr;
   p.steal_epoch = 0;
+  p.steal_merge = 0;
   if constexpr (CK != pa::kE4M3) {
     if (!list && use_steal(p, grid_x, dependent)) {
       kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false, true>;
@@ -379,6 +380,35 @@ pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t
     return with_reduce ? launch_reduce<TQ, D>(p, st) : PA_OK;
   }
   dim3 grid(grid_x, p.num_kv_heads * p.head_groups, p.batch);
+  if (p.steal_ctr) {
+    // Steal mode: when the whole grid fits on the GPU at once and the
+    // workspace section holds three counters per head group, the rows merge
+    // their own partials in the launch (a cooperative launch, so that the
+    // CTAs a row's merge waits for are resident) and no merge kernel follows
+    int per_sm = 0, sms = 0;
+    if (resident_ctas(reinterpret_cast<const void*>(kern), kDecodeWarps * 32, smem, &per_sm,
+                      &sms) != cudaSuccess)
+      return PA_ERR_CUDA;
+    const int64_t hb = static_cast<int64_t>(p.num_kv_heads) * p.head_groups;
+    const int64_t list_bytes =
+        256 + (static_cast<int64_t>(p.num_partitions) * 8 + 255) / 256 * 256;
+    const int64_t ctas = static_cast<int64_t>(grid_x) * hb * p.batch;
+    if (ctas <= static_cast<int64_t>(per_sm) * sms && 3 * hb * p.batch * 8 <= list_bytes) {
+      pa::DecodeParams pm = p;
+      pm.steal_merge = 1;
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(kDecodeWarps * 32);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      return cudaLaunchKernelEx(&cfg, kern, pm) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    }
+  }
   if (dependent) {
     if (launch_dependent(kern, grid, dim3(kDecodeWarps * 32), smem, st, p) != cudaSuccess)
       return PA_ERR_CUDA;

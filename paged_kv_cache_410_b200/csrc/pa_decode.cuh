@@ -114,6 +114,12 @@ struct DecodeParams {
   // partition column, and the merge zeroes the counters.
   unsigned long long* steal_ctr;
   unsigned long long steal_epoch;
+  // Steal mode, launched cooperatively (all CTAs resident at once): each
+  // row's CTAs merge the row's partials themselves once the last of them is
+  // written, counting on steal_ctr[rows + row] (partials written) and
+  // steal_ctr[2 rows + row] (CTAs done), and the row's last CTA zeroes its
+  // three counters; no merge kernel follows.
+  int steal_merge;
 };
 
 constexpr int kStealChunk = 4;
@@ -145,6 +151,138 @@ __device__ __forceinline__ int steal_claim(unsigned long long* ctr, unsigned lon
   }
   flag_error(PA_DEVERR_TIMEOUT);
   return 1 << 30;
+}
+
+// Steal mode with the merge in the launch: the partials of a (sequence, KV
+// head group) row -- nparts of them, one per CTA of the row -- combined by
+// those CTAs into `out` once all are written. CTA `part` takes an even slice
+// of the row's float4 output columns (query head x 4 channels); a warp
+// merges one column at a time, its lanes taking the partials lane, lane +
+// 32, ... with a running max each, then combined across the warp. The wait
+// for the row's last partial is bounded (1 s of %globaltimer; then
+// PA_DEVERR_TIMEOUT and no merge): the launch is cooperative, so the CTAs it
+// waits for are resident.
+constexpr unsigned long long kStealWaitNs = 1000000000ull;
+template <typename TQ, int D, int NW>
+__device__ __forceinline__ void steal_merge_row(const DecodeParams& p, int b, int by, int hq0,
+                                             int nrows, int nparts, int part) {
+  const int64_t rows = static_cast<int64_t>(p.batch) * p.num_kv_heads * p.head_groups;
+  const int64_t row = static_cast<int64_t>(b) * p.num_kv_heads * p.head_groups + by;
+  unsigned long long* done = p.steal_ctr + rows + row;
+  unsigned long long* gone = p.steal_ctr + 2 * rows + row;
+  const unsigned long long mask = (1ull << kStealCountBits) - 1;
+  __shared__ int s_ok;
+  __syncthreads();  // every partial of this CTA is stored
+  if (threadIdx.x == 0) {
+    __threadfence();
+    steal_claim(done, p.steal_epoch, 1);
+    unsigned long long t_start, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
+    int ok = 0;
+    while (true) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(done) : "memory");
+      if ((v & ~mask) == p.steal_epoch && static_cast<int>(v & mask) >= nparts) {
+        ok = 1;
+        break;
+      }
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t_start > kStealWaitNs) {
+        flag_error(PA_DEVERR_TIMEOUT);
+        break;
+      }
+      __nanosleep(128);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (s_ok) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    constexpr int C4 = D / 4;
+    const int total = nrows * C4;
+    const int per = (total + nparts - 1) / nparts;
+    const int hi = min(total, (part + 1) * per);
+    for (int col = part * per + warp; col < hi; col += NW) {
+      const int r = col / C4;
+      const int c4 = col - r * C4;
+      const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + r;
+      const float2* ml = p.ws_ml + bh * p.num_partitions;
+      const float4* po = reinterpret_cast<const float4*>(p.ws_o + bh * p.num_partitions * D) + c4;
+      float mx = -INFINITY, ws = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < nparts; j0 += 64) {
+        // two partials per lane, both loaded before either is used
+        float2 v[2];
+        float4 o[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int j = j0 + lane + 32 * k;
+          v[k] = make_float2(-INFINITY, 0.f);
+          o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (j < nparts) {
+            v[k] = __ldcg(ml + j);
+            o[k] = __ldcg(po + static_cast<int64_t>(j) * C4);
+          }
+        }
+        const float mn = fmaxf(mx, fmaxf(v[0].x, v[1].x));
+        if (mn == -INFINITY) continue;  // (CTAs that got no tile: sum 0)
+        const float sc = mx == -INFINITY ? 0.f : ex2(mx - mn);
+        ws *= sc;
+        acc.x *= sc;
+        acc.y *= sc;
+        acc.z *= sc;
+        acc.w *= sc;
+        mx = mn;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const float w = v[k].x == -INFINITY ? 0.f : v[k].y * ex2(v[k].x - mx);
+          ws += w;
+          acc.x += w * o[k].x;
+          acc.y += w * o[k].y;
+          acc.z += w * o[k].z;
+          acc.w += w * o[k].w;
+        }
+      }
+      float M = mx;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float sc = mx == -INFINITY ? 0.f : ex2(mx - M);
+      ws *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ws += __shfl_xor_sync(0xffffffffu, ws, o);
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+      }
+      if (lane == 0) {
+        TQ* out = reinterpret_cast<TQ*>(p.out) + bh * D + 4 * c4;
+        const float inv = 1.f / ws;
+        out[0] = from_f32<TQ>(acc.x * inv);
+        out[1] = from_f32<TQ>(acc.y * inv);
+        out[2] = from_f32<TQ>(acc.z * inv);
+        out[3] = from_f32<TQ>(acc.w * inv);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_ok) {
+    // the row's last CTA out puts its counters back to zero (every CTA of
+    // the row is past the wait by then), so that a replay of this launch
+    // with the same epoch starts afresh
+    if (steal_claim(gone, p.steal_epoch, 1) == nparts - 1) {
+      atomicExch(p.steal_ctr + row, 0ull);
+      atomicExch(done, 0ull);
+      atomicExch(gone, 0ull);
+    }
+  }
 }
 
 constexpr int kOrderMaxBatch = 256;
@@ -971,7 +1109,14 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     const int share = ((ntiles / 2) / nparts) & ~(kStealChunk * NW - 1);
     const int share_chunks = share / (kStealChunk * NW);  // per warp
     const int pool = nparts * share;                       // first tile of the pool
-    if (part == 0 && threadIdx.x == 0) steal_claim(ctr, p.steal_epoch, 0);
+    if (part == 0 && threadIdx.x == 0) {
+      steal_claim(ctr, p.steal_epoch, 0);
+      if (p.steal_merge) {  // and the in-launch merge's two counters
+        const int64_t rows = static_cast<int64_t>(p.batch) * p.num_kv_heads * p.head_groups;
+        steal_claim(ctr + rows, p.steal_epoch, 0);
+        steal_claim(ctr + 2 * rows, p.steal_epoch, 0);
+      }
+    }
     int k_share = 0;
     // first tile of the warp's next chunk (>= ntiles: none left), and the
     // chunk's block ids in lanes 0 .. kStealChunk - 1
@@ -1116,6 +1261,9 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     }
   }
   if constexpr (FUSED && CK == kE4M3) store_new_token();
+  if constexpr (STEAL) {
+    if (p.steal_merge && !direct) steal_merge_row<TQ, D, NW>(p, b, by, hq0, nrows, nparts, part);
+  }
   if (steer) {
     cursor->u = ticket;
     cursor->item = next_item;
@@ -1201,16 +1349,17 @@ __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
 // 170 registers; left alone the compiler takes up to 255 and the SM holds
 // two); the others are left to the compiler's choice, which keeps them at
 // <= 128 registers (an explicit minimum of one CTA made it take 173 for the
-// one-block 16-bit decode and cost the SM its third CTA).
-template <int CK, int D, int NH>
+// one-block 16-bit decode and cost the SM its third CTA). The steal-mode
+// decode at head_dim 128 is held to 3 as well.
+template <int CK, int D, int NH, bool STEAL = false>
 constexpr int decode_min_ctas() {
-  return (D == 128 && NH == 2) ? 3 : 0;
+  return (D == 128 && (NH == 2 || STEAL)) ? 3 : 0;
 }
 
 // grid: (partitions, num_kv_heads * head_groups, batch), or work-list mode
 // (STEAL: steal mode, a grid over one sequence)
 template <typename TQ, int CK, int D, int NW, int NSTAGE, int NH, bool FUSED, bool STEAL = false>
-__global__ void __launch_bounds__(NW * 32, (decode_min_ctas<CK, D, NH>()))
+__global__ void __launch_bounds__(NW * 32, (decode_min_ctas<CK, D, NH, STEAL>()))
     pa_decode_kernel(const DecodeParams p) {
   decode_launch_cta<TQ, CK, D, NW, NSTAGE, NH, FUSED, STEAL>(p);
 }

@@ -7,8 +7,12 @@ fixed partition; a CTA on a slower SM then takes fewer tiles. Which CTA
 takes which tiles changes from call to call, so the output is compared with
 the float64 oracle within the decode tolerance, call after call, with the
 workspace refilled with garbage before each call (counters of no epoch of
-this process). After each call the merge has put the counters back to zero,
-which also shows that steal mode ran; a launch outside steal mode (shorter
+this process). When the whole grid fits on the GPU at once, each row's CTAs
+merge the row's partials themselves inside the (cooperative) launch, with
+two more counters per row; otherwise the merge kernel runs after the grid.
+After each call the counters are back at zero (the merge kernel, or the
+row's last CTA, zeroes them), which also shows that steal mode ran; a
+launch outside steal mode (shorter
 partitions, blocks of 8 tokens, reproducible results asked for) leaves that
 section as it was."""
 import numpy as np
@@ -98,6 +102,14 @@ def test_sliding_window():
     # the plan
     w = W.custom([9000], num_q_heads=16, num_kv_heads=4, head_dim=128, seed=23)
     run_calls(w, 1024, window=5000)
+
+
+def test_grid_larger_than_the_gpu_holds():
+    # 20 partitions x 32 KV heads: more CTAs than fit at once, so the rows
+    # are merged by the merge kernel after the grid (smaller grids merge
+    # their rows inside the launch)
+    w = W.custom([20000], num_q_heads=32, num_kv_heads=32, head_dim=128, seed=29)
+    run_calls(w, 1024)
 
 
 def test_static_workspace():
