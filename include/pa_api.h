@@ -294,6 +294,15 @@ pa_status pa_copy_blocks_layers(const int32_t* pairs_host, int32_t num_pairs,
  * default; not for production calls. */
 void pa_testing_withhold_prefix_scores(int32_t on);
 
+/* Test hook for the failure path of a steal-mode decode that merges its rows
+ * inside the launch (see pa_set_deterministic: a single long sequence whose
+ * CTAs all fit on the GPU at once). While on (process-wide), the first CTA
+ * of each row does not count its partial, so every CTA's wait for the row
+ * runs out after its 1 s limit: no row is merged, the output is left as it
+ * was, the device error word gets PA_DEVERR_TIMEOUT and the context stays
+ * usable. Off by default; not for production calls. */
+void pa_testing_withhold_steal_counts(int32_t on);
+
 /* Synchronise `stream`, then read and clear the current device's error
  * word into *flags (PA_DEVERR_* bits). Returns PA_ERR_DEVICE_BOUNDS when
  * any bit was set, PA_OK when none, PA_ERR_CUDA on a runtime failure.

@@ -33,7 +33,7 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
             "pa_append_decode", "pa_copy_blocks_layers",
             "pa_decode_shared_prefix_partition_tokens", "pa_testing_withhold_prefix_scores",
-            "pa_set_deterministic"]
+            "pa_set_deterministic", "pa_testing_withhold_steal_counts"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_version.restype = i32
     lib.pa_set_deterministic.argtypes = [i32]
     lib.pa_set_deterministic.restype = i32
+    lib.pa_testing_withhold_steal_counts.argtypes = [i32]
+    lib.pa_testing_withhold_steal_counts.restype = None
     lib.pa_decode_static_workspace.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32,
                                                ctypes.c_float, P, i32, P]
     lib.pa_decode_static_workspace.restype = ctypes.c_int
@@ -387,6 +389,13 @@ def pa_copy_blocks_layers(pairs, k_caches, v_caches, cache: PagedCache, stream=N
     rc = lib.pa_copy_blocks_layers(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], kp, vp, n,
                                    ctypes.byref(d), _stream(stream))
     _check(rc, "pa_copy_blocks_layers")
+
+
+def pa_testing_withhold_steal_counts(on: bool):
+    """Test hook (process-wide): in a steal-mode decode that merges its rows
+    in the launch, each row's first CTA does not count its partial, so the
+    rows' bounded waits run out (PA_DEVERR_TIMEOUT)."""
+    load_library().pa_testing_withhold_steal_counts(1 if on else 0)
 
 
 def pa_testing_withhold_prefix_scores(on: bool):

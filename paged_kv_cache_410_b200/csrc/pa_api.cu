@@ -259,6 +259,7 @@ bool use_work_list(const pa::DecodeParams& p, bool dependent) {
 // hold the tiles plus one overshooting chunk per warp.
 constexpr int kStealMinPartition = 1024;
 std::atomic<int> g_deterministic{0};
+std::atomic<int> g_withhold_steal_counts{0};  // pa_testing_withhold_steal_counts
 
 bool use_steal(const pa::DecodeParams& p, int grid_x, bool dependent) {
   const int64_t hb = static_cast<int64_t>(p.num_kv_heads) * p.head_groups;
@@ -339,6 +340,7 @@ pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t
   p.steal_ctr = nullptr;
   p.steal_epoch = 0;
   p.steal_merge = 0;
+  p.steal_withhold = 0;
   if constexpr (CK != pa::kE4M3) {
     if (!list && use_steal(p, grid_x, dependent)) {
       kern = pa::pa_decode_kernel<TQ, CK, D, kDecodeWarps, kDecodeStages, NH, false, true>;
@@ -396,6 +398,7 @@ pa_status launch_decode_t(const pa::DecodeParams& p_in, int grid_x, cudaStream_t
     if (ctas <= static_cast<int64_t>(per_sm) * sms && 3 * hb * p.batch * 8 <= list_bytes) {
       pa::DecodeParams pm = p;
       pm.steal_merge = 1;
+      pm.steal_withhold = g_withhold_steal_counts.load(std::memory_order_relaxed);
       cudaLaunchConfig_t cfg{};
       cfg.gridDim = grid;
       cfg.blockDim = dim3(kDecodeWarps * 32);
@@ -787,6 +790,10 @@ const char* pa_status_string(int32_t s) {
 }
 
 int32_t pa_version(void) { return 100; }
+
+void pa_testing_withhold_steal_counts(int32_t on) {
+  g_withhold_steal_counts.store(on != 0 ? 1 : 0, std::memory_order_relaxed);
+}
 
 int32_t pa_set_deterministic(int32_t on) {
   return g_deterministic.exchange(on != 0 ? 1 : 0);

@@ -118,8 +118,10 @@ struct DecodeParams {
   // row's CTAs merge the row's partials themselves once the last of them is
   // written, counting on steal_ctr[rows + row] (partials written) and
   // steal_ctr[2 rows + row] (CTAs done), and the row's last CTA zeroes its
-  // three counters; no merge kernel follows.
+  // three counters; no merge kernel follows. steal_withhold (test hook):
+  // the row's first CTA does not count its partial, so every wait runs out.
   int steal_merge;
+  int steal_withhold;
 };
 
 constexpr int kStealChunk = 4;
@@ -175,7 +177,7 @@ __device__ __forceinline__ void steal_merge_row(const DecodeParams& p, int b, in
   __syncthreads();  // every partial of this CTA is stored
   if (threadIdx.x == 0) {
     __threadfence();
-    steal_claim(done, p.steal_epoch, 1);
+    if (!(p.steal_withhold && part == 0)) steal_claim(done, p.steal_epoch, 1);
     unsigned long long t_start, t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_start));
     int ok = 0;

@@ -143,3 +143,30 @@ def test_not_used(why):
         assert not B.pa_set_deterministic(False)  # the previous setting is back
     else:
         run_calls(w, pt, expect_steal=False)
+
+
+def test_merge_wait_timeout_is_reported_and_recoverable():
+    # the in-launch merge's wait for a row's partials is bounded: with one
+    # CTA per row not counting its partial, every wait runs out (1 s), the
+    # device error word reports PA_DEVERR_TIMEOUT and no row is merged;
+    # afterwards the context is usable and a normal call matches the oracle
+    w = W.custom([12000], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=31)
+    step = DecodeStep(w, "cuda", partition_tokens=1024)
+    step.copy()
+    step.append()
+    torch.cuda.synchronize()
+    step.out.fill_(float("nan"))
+    B.pa_testing_withhold_steal_counts(1)
+    try:
+        step.decode()
+        torch.cuda.synchronize()
+        assert step.device_errors() & B.DEVERR_TIMEOUT
+        assert torch.isnan(step.out).all()  # nothing was merged
+    finally:
+        B.pa_testing_withhold_steal_counts(0)
+    for _ in range(2):
+        step.decode()
+        torch.cuda.synchronize()
+        assert step.device_errors() == 0
+    _, _, want = oracle_step(w)
+    assert max_abs_err(step.out_f64(), want) <= TOL[w.io_dtype]
