@@ -12,7 +12,9 @@
  * Variants: pa_append_decode (append fused into the decode launch),
  * pa_decode_sliding_window, pa_decode_shared_prefix (a shared prefix attended
  * once for the whole batch), pa_copy_blocks_layers (every layer's caches in
- * one call) and pa_decode_static_workspace (no caller workspace).
+ * one call), pa_decode_static_workspace (no caller workspace), and
+ * pa_decode_partial + pa_merge_partials (a sequence's history split across
+ * calls or GPUs, merged after an exchange of the partial results).
  *
  * Sources of the definitions (page titles and sections):
  *  - "AI 陪读顶会论文（三）：KV Cache 显存占用计算与 PagedAttention 原理拆解",
@@ -344,6 +346,49 @@ pa_status pa_decode_static_workspace(const void* q, int32_t q_dtype, int32_t bat
                                      const int32_t* context_lens, int32_t max_context,
                                      float scale, void* out, int32_t partition_tokens,
                                      void* stream);
+
+/* Context parallelism, part 1: pa_decode over the tokens each sequence's
+ * table lists, stopping short of the final normalisation across calls, so
+ * that several calls over disjoint parts of every sequence's history (for
+ * example the block-aligned context slices that several GPUs hold) can be
+ * merged by pa_merge_partials into exactly what one pa_decode over the whole
+ * history gives, up to rounding. It is the decode's own split-K merge
+ * (softmax of the scores over partitions) carried across calls; the pages
+ * have no counterpart beyond that merge.
+ *   part_o   [batch][num_q_heads][head_dim] fp32: each row's attention
+ *            output over this call's tokens (normalised as pa_decode's);
+ *            16-byte aligned.
+ *   part_ml  [batch][num_q_heads][2] fp32: each row's (m, l) over the
+ *            same tokens, with s_j = scale * q.k_j * log2(e), m a reference
+ *            value at or below max_j s_j and within 8 of it (the decode moves
+ *            its running maximum only by steps of at least 8), and
+ *            l = sum_j 2^(s_j - m): the pair encodes the softmax
+ *            denominator, m + log2(l) = log2(sum_j 2^(s_j)). A row with no
+ *            tokens (context_lens[b] == 0) gives output 0, m = -inf, l = 0.
+ *            16-byte aligned.
+ * Other arguments, checks, statuses and the workspace (the
+ * pa_decode_workspace_size formula) as for pa_decode; `out` is not used.
+ * The call keeps the plain grid of partitions (no work list, no steal mode)
+ * and is reproducible. */
+pa_status pa_decode_partial(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                            const void* k_cache, const void* v_cache, const pa_cache_desc* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context, float scale,
+                            float* part_o, float* part_ml, int32_t partition_tokens,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Context parallelism, part 2: merge num_parts results of pa_decode_partial
+ * stacked part-major, part_o [num_parts][rows][head_dim] and part_ml
+ * [num_parts][rows][2] (rows = batch * num_q_heads; the layout an all-gather
+ * of each GPU's part_o / part_ml produces), into out [rows][head_dim] in
+ * out_dtype (PA_F16 or PA_BF16): out = sum_n w_n o_n / sum_n w_n with
+ * w_n = l_n * 2^(m_n - max over the parts of m). Parts with l = 0 weigh
+ * nothing; a row whose parts all have l = 0 gives 0. head_dim 64 or 128;
+ * every pointer 16-byte aligned device memory. Returns PA_ERR_INVALID_ARG /
+ * PA_ERR_UNSUPPORTED on bad sizes or pointers (nothing enqueued). */
+pa_status pa_merge_partials(const float* part_o, const float* part_ml, int32_t num_parts,
+                            int64_t rows, int32_t head_dim, void* out, int32_t out_dtype,
+                            void* stream);
 
 /* Reproducible results (process-wide, any thread; 0 at load). With 0, a
  * pa_decode, pa_decode_static_workspace or pa_decode_sliding_window call on

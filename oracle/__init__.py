@@ -184,3 +184,70 @@ def decode(q, q_dtype, k_cache, v_cache, cache_dtype, block_tables, context_lens
                            float(np.float32(scale)), int(window), _ptr(out))
     _check(rc, "oracle_decode")
     return out
+
+
+def _values(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Stored bit patterns as float64 values."""
+    if dtype == "f16":
+        return f16_to_double(a)
+    if dtype == "bf16":
+        return bf16_to_double(a)
+    return e4m3_to_double(a)
+
+
+def decode_partial(q, q_dtype, k_cache, v_cache, cache_dtype, block_tables, context_lens, scale,
+                   k_scale=None, v_scale=None):
+    """The pieces of the decode over the tokens each table lists, for merging
+    with other parts of the same histories (numpy, float64; small cases).
+    Returns (o [B, Hq, D], m [B, Hq], l [B, Hq]) with s_j = scale * q . k_j
+    over the row's tokens, m = max_j s_j, l = sum_j exp(s_j - m) and
+    o = sum_j exp(s_j - m) v_j / l: the softmax of the decode's attention
+    equation split at its normaliser. A row with no tokens gives o = 0,
+    m = -inf, l = 0. (The attention equation of "AI 陪读顶会论文（三）：KV
+    Cache 显存占用计算与 PagedAttention 原理拆解", section "为什么自回归解码
+    必须使用 KV Cache？", as ``decode`` computes it, with the softmax's sum
+    left unnormalised across parts.)"""
+    qv = _values(np.asarray(q), q_dtype)
+    kc = _values(np.asarray(k_cache), cache_dtype)
+    vc = _values(np.asarray(v_cache), cache_dtype)
+    if cache_dtype == "e4m3":
+        kc = kc * np.asarray(k_scale, np.float64)[None, None]
+        vc = vc * np.asarray(v_scale, np.float64)[None, None]
+    b_n, hq, d = qv.shape
+    _, bs, hkv, _ = kc.shape
+    group = hq // hkv
+    o = np.zeros((b_n, hq, d))
+    m = np.full((b_n, hq), -np.inf)
+    l = np.zeros((b_n, hq))
+    for b in range(b_n):
+        L = int(context_lens[b])
+        if L == 0:
+            continue
+        j = np.arange(L)
+        blk = np.asarray(block_tables[b])[j // bs]
+        K = kc[blk, j % bs]  # [L, Hkv, D]
+        V = vc[blk, j % bs]
+        for i in range(hq):
+            h = i // group
+            s = float(np.float32(scale)) * (K[:, h] @ qv[b, i])
+            m[b, i] = s.max()
+            e = np.exp(s - m[b, i])
+            l[b, i] = e.sum()
+            o[b, i] = (e @ V[:, h]) / l[b, i]
+    return o, m, l
+
+
+def merge_partials(o, m, l):
+    """Merge parts stacked part-major (o [N, ..., D], m and l [N, ...]) of the
+    same rows into the decode output: sum_n w_n o_n / sum_n w_n with
+    w_n = l_n exp(m_n - max_n m_n); parts with l = 0 weigh nothing and rows
+    without any token give 0."""
+    o = np.asarray(o, np.float64)
+    m = np.asarray(m, np.float64)
+    l = np.asarray(l, np.float64)
+    M = np.max(np.where(l > 0, m, -np.inf), axis=0)
+    M = np.where(np.isfinite(M), M, 0.0)  # (rows without tokens: every weight is 0)
+    w = np.where(l > 0, l * np.exp(np.where(l > 0, m, 0.0) - M[None]), 0.0)
+    den = w.sum(axis=0)
+    num = (w[..., None] * o).sum(axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)

@@ -33,7 +33,8 @@ EXPORTED = ["pa_append_kv", "pa_decode_workspace_size", "pa_decode_partition_tok
             "pa_decode_sliding_window_workspace_size", "pa_decode_sliding_window",
             "pa_append_decode", "pa_copy_blocks_layers",
             "pa_decode_shared_prefix_partition_tokens", "pa_testing_withhold_prefix_scores",
-            "pa_set_deterministic", "pa_testing_withhold_steal_counts"]
+            "pa_set_deterministic", "pa_testing_withhold_steal_counts",
+            "pa_decode_partial", "pa_merge_partials"]
 
 
 class PagedAttentionError(RuntimeError):
@@ -85,6 +86,11 @@ def load_library(path: str = LIB_PATH):
     lib.pa_set_deterministic.restype = i32
     lib.pa_testing_withhold_steal_counts.argtypes = [i32]
     lib.pa_testing_withhold_steal_counts.restype = None
+    lib.pa_decode_partial.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32, ctypes.c_float,
+                                      P, P, i32, P, ctypes.c_size_t, P]
+    lib.pa_decode_partial.restype = ctypes.c_int
+    lib.pa_merge_partials.argtypes = [P, P, i32, ctypes.c_int64, i32, P, i32, P]
+    lib.pa_merge_partials.restype = ctypes.c_int
     lib.pa_decode_static_workspace.argtypes = [P, i32, i32, i32, P, P, D, P, i32, P, i32,
                                                ctypes.c_float, P, i32, P]
     lib.pa_decode_static_workspace.restype = ctypes.c_int
@@ -262,6 +268,44 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, cache
                        float(scale), po, int(partition_tokens), _dev(workspace, "workspace"),
                        _nbytes(workspace), _stream(stream))
     _check(rc, "pa_decode")
+
+
+def pa_decode_partial(q, k_cache, v_cache, block_tables, context_lens, scale, part_o, part_ml,
+                      cache: PagedCache, max_context: int, partition_tokens: int = 0,
+                      workspace=None, stream=None):
+    """pa_decode over the tokens each table lists, left as the pieces a merge
+    of several such calls needs: part_o [B, Hq, D] float32 (each row's
+    normalised output) and part_ml [B, Hq, 2] float32 (max score in log2
+    units, sum of 2^(score - max)). Workspace as for pa_decode."""
+    lib = load_library()
+    d = cache.desc()
+    batch, hq = q.shape[0], q.shape[1]
+    pq, pt, pl, _ = _decode_io(q, block_tables, context_lens, q, cache)
+    po = _dev(part_o, "part_o", (torch.float32,), (batch, hq, cache.head_dim))
+    pm = _dev(part_ml, "part_ml", (torch.float32,), (batch, hq, 2))
+    kc, vc = cache.cache_ptrs(k_cache, v_cache)
+    rc = lib.pa_decode_partial(pq, _dtype_code(q.dtype), batch, hq, kc, vc, ctypes.byref(d), pt,
+                               block_tables.shape[1], pl, int(max_context), float(scale), po, pm,
+                               int(partition_tokens), _dev(workspace, "workspace"),
+                               _nbytes(workspace), _stream(stream))
+    _check(rc, "pa_decode_partial")
+
+
+def pa_merge_partials(part_o, part_ml, out, stream=None):
+    """out [rows..., D] (fp16 / bf16) from pa_decode_partial results stacked
+    part-major: part_o [N, rows..., D] float32, part_ml [N, rows..., 2]
+    float32 (an all-gather's layout)."""
+    lib = load_library()
+    if part_o.dim() < 2 or part_o.shape[1:] != out.shape:
+        raise ValueError("part_o: expected [num_parts, *out.shape]")
+    n, hd = part_o.shape[0], out.shape[-1]
+    rows = out.numel() // hd if hd else 0
+    po = _dev(part_o, "part_o", (torch.float32,))
+    pm = _dev(part_ml, "part_ml", (torch.float32,), tuple(part_o.shape[:-1]) + (2,))
+    pout = _dev(out, "out", _IO)
+    rc = lib.pa_merge_partials(po, pm, int(n), int(rows), int(hd), pout, _dtype_code(out.dtype),
+                               _stream(stream))
+    _check(rc, "pa_merge_partials")
 
 
 def pa_append_decode(q, k, v, slot_mapping, k_cache, v_cache, block_tables, context_lens,

@@ -206,8 +206,8 @@ cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, siz
 // Split-K merge, the decode kernel's programmatic dependent: 1, 2, 4, 8, 16
 // or 32 warps per (sequence, query head) row by the number of partials per
 // row (a row of 16 or 32 warps is a CTA of its own).
-template <typename TQ, int D>
-pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
+template <typename TQ, int D, bool PARTIAL>
+pa_status launch_reduce_t(const pa::DecodeParams& p, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.batch) * p.num_q_heads;
   const int n = p.num_partitions;
   auto go = [&](auto kern, int warps, int rows_per_cta) {
@@ -219,16 +219,22 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
   };
   // one warp per row: 32 rows per CTA, so that a large batch's merge is a few
   // hundred CTAs that all start at once
-  if (n <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32>, 32, 32);
-  if (n <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32>, 32, 32);
+  if (n <= 8) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 8, 32, PARTIAL>, 32, 32);
+  if (n <= 16) return go(pa::pa_decode_reduce_kernel<TQ, D, 1, 16, 32, PARTIAL>, 32, 32);
   // several warps per row: at most 8 partials a warp up to 128 partials, 16
   // up to 256; beyond, 32 warps take batches of 8 each (1024 threads leave a
   // thread 64 registers)
-  if (n <= 32) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 8, 16>, 16, 4);
-  if (n <= 64) return go(pa::pa_decode_reduce_kernel<TQ, D, 8, 8, 16>, 16, 2);
-  if (n <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 8, 16>, 16, 1);
-  if (n <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16>, 16, 1);
-  return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 8, 32>, 32, 1);
+  if (n <= 32) return go(pa::pa_decode_reduce_kernel<TQ, D, 4, 8, 16, PARTIAL>, 16, 4);
+  if (n <= 64) return go(pa::pa_decode_reduce_kernel<TQ, D, 8, 8, 16, PARTIAL>, 16, 2);
+  if (n <= 128) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 8, 16, PARTIAL>, 16, 1);
+  if (n <= 256) return go(pa::pa_decode_reduce_kernel<TQ, D, 16, 16, 16, PARTIAL>, 16, 1);
+  return go(pa::pa_decode_reduce_kernel<TQ, D, 32, 8, 32, PARTIAL>, 32, 1);
+}
+
+// (partial mode writes fp32 pieces instead of `out`: its own instantiations)
+template <typename TQ, int D>
+pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
+  return p.cp_o ? launch_reduce_t<TQ, D, true>(p, st) : launch_reduce_t<TQ, D, false>(p, st);
 }
 
 // Work-list mode (plain, fused and sliding-window decodes of a batch split
@@ -241,7 +247,7 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
 constexpr int kListGrowLog2 = 2;
 
 bool use_work_list(const pa::DecodeParams& p, bool dependent) {
-  return !dependent && p.prefix_blocks == 0 && p.work_items && p.batch > 1 &&
+  return !dependent && p.prefix_blocks == 0 && p.work_items && !p.cp_o && p.batch > 1 &&
          p.num_partitions > 1 &&
          static_cast<int64_t>(p.batch) * p.num_partitions * p.num_kv_heads * p.head_groups <
              (int64_t{1} << 31);
@@ -267,7 +273,7 @@ bool use_steal(const pa::DecodeParams& p, int grid_x, bool dependent) {
   const int64_t most_claimed = static_cast<int64_t>(p.max_context) / 16 + 1 +
                                static_cast<int64_t>(p.num_partitions) * kDecodeWarps *
                                    pa::kStealChunk + pa::kStealChunk;
-  return g_deterministic.load(std::memory_order_relaxed) == 0 && !dependent &&
+  return g_deterministic.load(std::memory_order_relaxed) == 0 && !dependent && !p.cp_o &&
          p.prefix_blocks == 0 && !p.k_new && p.work_count && p.batch == 1 &&
          p.num_partitions > 1 && p.partition_tokens >= kStealMinPartition &&
          grid_x == p.num_partitions && p.part_offset == 0 &&
@@ -790,6 +796,70 @@ const char* pa_status_string(int32_t s) {
 }
 
 int32_t pa_version(void) { return 100; }
+
+pa_status pa_decode_partial(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                            const void* k_cache, const void* v_cache, const pa_cache_desc* cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context, float scale,
+                            float* part_o, float* part_ml, int32_t partition_tokens,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!part_o || !part_ml || !aligned16(part_ml)) return PA_ERR_INVALID_ARG;
+  int bs_log2 = 0;
+  bool nothing = false;
+  // (part_o stands in for `out` in the shared checks: same rows, never read)
+  pa_status st = check_decode_args(q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                                   block_tables, max_blocks_per_seq, context_lens, max_context,
+                                   scale, part_o, partition_tokens, &bs_log2, &nothing);
+  if (st != PA_OK || nothing) return st;
+  const Plan pl = make_plan(batch, num_q_heads, max_context, partition_tokens, cache);
+  if (!pl.fits) return PA_ERR_UNSUPPORTED;
+  if (pl.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < pl.ws_bytes) return PA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PA_ERR_WORKSPACE;
+  }
+  pa::DecodeParams p = decode_params(q, batch, num_q_heads, k_cache, v_cache, cache,
+                                     block_tables, max_blocks_per_seq, context_lens, max_context,
+                                     scale, part_o, bs_log2);
+  bind_workspace(p, pl, workspace);
+  p.partition_tokens = pl.partition_tokens;
+  p.num_partitions = pl.num_partitions;
+  p.cp_o = part_o;
+  p.cp_ml = reinterpret_cast<float2*>(part_ml);
+  return launch_decode(p, q_dtype, cache, as_stream(stream));
+}
+
+pa_status pa_merge_partials(const float* part_o, const float* part_ml, int32_t num_parts,
+                            int64_t rows, int32_t head_dim, void* out, int32_t out_dtype,
+                            void* stream) {
+  if (num_parts < 1 || rows < 0 || (head_dim != 64 && head_dim != 128)) return PA_ERR_INVALID_ARG;
+  if (out_dtype != PA_F16 && out_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (rows == 0) return PA_OK;
+  if (!part_o || !part_ml || !out || !aligned16(part_o) || !aligned16(part_ml) ||
+      !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if (rows > (int64_t{1} << 40) / num_parts) return PA_ERR_UNSUPPORTED;
+  const int64_t ctas = (rows + 7) / 8;
+  if (ctas > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  const cudaStream_t st = as_stream(stream);
+  const float2* ml = reinterpret_cast<const float2*>(part_ml);
+  const dim3 grid(static_cast<unsigned>(ctas));
+  if (out_dtype == PA_F16) {
+    if (head_dim == 64)
+      pa::pa_merge_partials_kernel<__half, 64><<<grid, 256, 0, st>>>(part_o, ml, num_parts, rows,
+                                                                   static_cast<__half*>(out));
+    else
+      pa::pa_merge_partials_kernel<__half, 128><<<grid, 256, 0, st>>>(
+          part_o, ml, num_parts, rows, static_cast<__half*>(out));
+  } else {
+    if (head_dim == 64)
+      pa::pa_merge_partials_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(
+          part_o, ml, num_parts, rows, static_cast<__nv_bfloat16*>(out));
+    else
+      pa::pa_merge_partials_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(
+          part_o, ml, num_parts, rows, static_cast<__nv_bfloat16*>(out));
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 void pa_testing_withhold_steal_counts(int32_t on) {
   g_withhold_steal_counts.store(on != 0 ? 1 : 0, std::memory_order_relaxed);

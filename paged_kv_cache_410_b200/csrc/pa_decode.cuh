@@ -122,6 +122,14 @@ struct DecodeParams {
   // the row's first CTA does not count its partial, so every wait runs out.
   int steal_merge;
   int steal_withhold;
+  // Partial mode (pa_decode_partial; null: off): instead of `out`, each
+  // (sequence, query head) row's attention over the tokens its table lists
+  // goes to cp_o[row][D] (fp32, normalised as `out` would be) and
+  // cp_ml[row] = (max score in log2 units, sum of 2^(score - max)), the
+  // pieces a later merge of several such calls (pa_merge_partials) needs;
+  // an empty row gives (0, (-inf, 0)). The launch keeps the plain grid.
+  float* cp_o;
+  float2* cp_ml;
 };
 
 constexpr int kStealChunk = 4;
@@ -858,9 +866,15 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
 
   TQ* out = reinterpret_cast<TQ*>(p.out);
   if (L == 0) {  // (plain mode only: a cascade launch has no partition here)
-    for (int i = threadIdx.x; i < nrows * D; i += NW * 32)
-      out[(static_cast<int64_t>(b) * p.num_q_heads + hq0 + i / D) * D + (i % D)] =
-          from_f32<TQ>(0.f);
+    for (int i = threadIdx.x; i < nrows * D; i += NW * 32) {
+      const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + i / D;
+      if (p.cp_o) {
+        p.cp_o[bh * D + (i % D)] = 0.f;
+        if (i % D == 0) p.cp_ml[bh] = make_float2(-INFINITY, 0.f);
+      } else {
+        out[bh * D + (i % D)] = from_f32<TQ>(0.f);
+      }
+    }
     if (steer) cursor_next(p, *cursor);
     return;
   }
@@ -1253,7 +1267,10 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, const int part
     float val = lsum_row > 0.f ? acc / lsum_row : 0.f;
     if constexpr (CK == kE4M3) val *= vs[c];
     const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + row;
-    if (direct) {
+    if (direct && p.cp_o) {
+      p.cp_o[bh * D + c] = val;
+      if (c == 0) p.cp_ml[bh] = make_float2(r_stat[2 * row], r_stat[2 * row + 1]);
+    } else if (direct) {
       out[bh * D + c] = from_f32<TQ>(val);
     } else {
       st_hint(p.ws_o + (bh * p.num_partitions + slot) * D + c, val, keep);
@@ -1474,6 +1491,25 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   }
 }
 
+// A merged row's four channels of lane `lane`: to `out` in TQ, or in partial
+// mode (PARTIAL) to cp_o / cp_ml as fp32 with the row's (max, sum).
+template <typename TQ, int D, bool PARTIAL>
+__device__ __forceinline__ void write_merged(const DecodeParams& p, int64_t row, int lane,
+                                             float4 a, float ws, float M) {
+  const float inv = 1.f / ws;
+  if constexpr (PARTIAL) {
+    reinterpret_cast<float4*>(p.cp_o + row * D)[lane] =
+        make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+    if (lane == 0) p.cp_ml[row] = make_float2(M, ws);
+    return;
+  }
+  TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
+  out[0] = from_f32<TQ>(a.x * inv);
+  out[1] = from_f32<TQ>(a.y * inv);
+  out[2] = from_f32<TQ>(a.z * inv);
+  out[3] = from_f32<TQ>(a.w * inv);
+}
+
 // Merge split-K partials: with per-partition max m_p (log2 units), sum l_p
 // and normalised output o_p, out = sum_p w_p o_p / sum_p w_p where
 // w_p = l_p * 2^(m_p - max_p m_p).
@@ -1490,7 +1526,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
 //
 // The kernel is launched as the programmatic dependent of the kernels that
 // write the partials: it waits for them to complete before reading.
-template <typename TQ, int D, int WPR, int NL, int NWARPS>
+template <typename TQ, int D, int WPR, int NL, int NWARPS, bool PARTIAL = false>
 __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const DecodeParams p) {
   static_assert(D % 4 == 0 && D <= 128, "one float4 per lane");
   static_assert(NWARPS % WPR == 0, "whole rows per CTA");
@@ -1554,12 +1590,16 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
         acc.w += w * x[i].w;
       }
       if (active) {
-        TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
-        const float inv = 1.f / wsum;
-        out[0] = from_f32<TQ>(acc.x * inv);
-        out[1] = from_f32<TQ>(acc.y * inv);
-        out[2] = from_f32<TQ>(acc.z * inv);
-        out[3] = from_f32<TQ>(acc.w * inv);
+        if constexpr (PARTIAL) {
+          write_merged<TQ, D, PARTIAL>(p, row, lane, acc, wsum, M);
+        } else {
+          TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
+          const float inv = 1.f / wsum;
+          out[0] = from_f32<TQ>(acc.x * inv);
+          out[1] = from_f32<TQ>(acc.y * inv);
+          out[2] = from_f32<TQ>(acc.z * inv);
+          out[3] = from_f32<TQ>(acc.w * inv);
+        }
       }
     }
     return;
@@ -1636,13 +1676,49 @@ __global__ void __launch_bounds__(NWARPS * 32) pa_decode_reduce_kernel(const Dec
       a.w += r * b4.w;
       ws += r * s_wsum[warp + k];
     }
-    TQ* out = reinterpret_cast<TQ*>(p.out) + row * D + 4 * lane;
-    const float inv = 1.f / ws;
-    out[0] = from_f32<TQ>(a.x * inv);
-    out[1] = from_f32<TQ>(a.y * inv);
-    out[2] = from_f32<TQ>(a.z * inv);
-    out[3] = from_f32<TQ>(a.w * inv);
+    write_merged<TQ, D, PARTIAL>(p, row, lane, a, ws, M);
   }
+}
+
+// Merge of several pa_decode_partial results (context parallelism: each
+// call covered a disjoint part of every sequence's tokens): part n of row r
+// is part_o[n][r][D] with (max, sum) part_ml[n][r], in the log2 units
+// pa_decode_partial writes; out[r] = sum_n w_n o_n / sum_n w_n with
+// w_n = sum_n 2^(max_n - max over n). A warp per row, lane l owning channels
+// 4l .. 4l+3; a part with sum 0 (no tokens) weighs nothing.
+template <typename TQ, int D>
+__global__ void __launch_bounds__(256) pa_merge_partials_kernel(const float* part_o,
+                                                               const float2* part_ml,
+                                                               int num_parts, int64_t rows,
+                                                               TQ* out) {
+  static_assert(D % 4 == 0 && D <= 128, "one float4 per lane");
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= rows || lane >= D / 4) return;
+  float M = -INFINITY;
+  for (int n = 0; n < num_parts; ++n) {
+    const float2 v = part_ml[n * rows + r];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
+  }
+  float ws = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int n = 0; n < num_parts; ++n) {
+    const float2 v = part_ml[n * rows + r];
+    if (!(v.y > 0.f)) continue;
+    const float w = v.y * ex2(v.x - M);
+    const float4 o = reinterpret_cast<const float4*>(part_o + (n * rows + r) * D)[lane];
+    ws += w;
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = ws > 0.f ? 1.f / ws : 0.f;  // no part with tokens: a zero row
+  TQ* o = out + r * D + 4 * lane;
+  o[0] = from_f32<TQ>(acc.x * inv);
+  o[1] = from_f32<TQ>(acc.y * inv);
+  o[2] = from_f32<TQ>(acc.z * inv);
+  o[3] = from_f32<TQ>(acc.w * inv);
 }
 
 }  // namespace pa
