@@ -411,6 +411,18 @@ def decode_plan(args, w, step, spb):
     n = max(1, math.ceil(w.max_context / pt))
     name = ("pa_append_decode (append fused into decode; main + split-K reduce)" if args.fused
             else "pa_decode (main + split-K reduce)")
+    if (not args.fused and w.batch == 1 and n > 1 and pt >= 1024 and w.cache_dtype != "e4m3"
+            and w.block_size >= 16):
+        # steal mode; the rows merge inside the (cooperative) launch when the
+        # grid fits on the GPU at once: 3 CTAs per SM at head_dim 128 (66 KB
+        # of shared memory, up to 168 registers), 4 at 64 (up to 128)
+        import torch
+        sms = torch.cuda.get_device_properties(step.q.device).multi_processor_count
+        groups = w.num_kv_heads * -(-(w.num_q_heads // w.num_kv_heads) // 16)
+        if n * groups <= sms * (3 if w.head_dim == 128 else 4) and 3 * groups * 8 <= (
+                256 + -(-n * 8 // 256) * 256):
+            return pt, n, 1, "pa_decode (steal mode, rows merged in the launch)"
+        return pt, n, 2, "pa_decode (steal mode + split-K reduce)"
     return pt, n, split(n), name
 
 
