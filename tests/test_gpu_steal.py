@@ -170,3 +170,32 @@ def test_merge_wait_timeout_is_reported_and_recoverable():
         assert step.device_errors() == 0
     _, _, want = oracle_step(w)
     assert max_abs_err(step.out_f64(), want) <= TOL[w.io_dtype]
+
+
+@pytest.mark.parametrize("L", [0, 3000, 9000])
+def test_launch_planned_for_longer_histories(L):
+    # max_context (what the launch and its plan are sized for) well above the
+    # sequence's length: the CTA columns past the sequence's partitions leave
+    # at once, and only its own partitions' CTAs share its tiles and merge
+    w = W.custom([max(L, 1)], num_q_heads=32, num_kv_heads=8, head_dim=128, seed=33 + L)
+    step = DecodeStep(w, "cuda")
+    step.copy()
+    step.append()
+    step.context_lens.fill_(L)
+    w.context_lens[:] = L
+    maxc = 40000
+    ws_n = B.pa_decode_workspace_size(1, w.num_q_heads, maxc, step.cache, 1024)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    for fill in (0xFF, 0x00):
+        ws.fill_(fill)
+        out = torch.full_like(step.out, float("nan"))
+        B.pa_decode(step.q, step.k_cache, step.v_cache, step.block_tables, step.context_lens,
+                    float(w.scale), out, step.cache, maxc, 1024, ws, step.stream)
+        torch.cuda.synchronize()
+        assert step.device_errors() == 0
+        got = out.double().cpu().numpy()
+        if L == 0:
+            assert np.all(got == 0)
+        else:
+            _, _, want = oracle_step(w)
+            assert max_abs_err(got, want) <= TOL[w.io_dtype]
