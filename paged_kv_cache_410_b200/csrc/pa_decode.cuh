@@ -93,9 +93,10 @@ struct DecodeParams {
   int longest_first;
   // Work-list mode (null: a grid of partitions x head groups x sequences):
   // pa_decode_plan_kernel writes the launch's (sequence, partition) items to
-  // work_items, largest first, their count to work_count[1] and zero to
-  // work_count[0]; a persistent grid then takes (item, KV head group) units
-  // by atomicAdd on work_count[0].
+  // work_items, largest first, their count to work_count[1] and the
+  // persistent grid's size (list_slots) to work_count[0]; CTA i of that grid
+  // starts with unit i, and every later unit is a ticket from atomicAdd on
+  // work_count[0].
   int2* work_items;
   int* work_count;
   // Work-list mode: the persistent grid's CTAs (the plan kernel sizes the
@@ -1313,7 +1314,10 @@ __device__ __forceinline__ void decode_launch_cta(const DecodeParams& p) {
       // (batch x partitions x hb < 2^31: the host checks the bound)
       cur.n_units = min(p.work_count[1], p.batch * p.num_partitions) * units_per_item(p);
       cur.pt = launch_partition_tokens(p);
-      cursor_next(p, cur);
+      // the first unit is the CTA's own index: no ticket to wait for
+      const int u = static_cast<int>(blockIdx.x);
+      cur.item = cursor_item(p, cur, u);
+      cur.u = u;
     }
     __syncthreads();
   } else if (p.longest_first) {
@@ -1426,10 +1430,16 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   // launch staged for block ids), the longest whose item is at most 3/4 of a
   // slot's share of the batch's tokens x head groups. Longer partitions
   // mean fewer units and partials; the largest items still start first.
+  // (each thread keeps the length of its first sequence: the passes below
+  // read it again, and a batch of up to kPlanThreads has no other)
+  const int my_len = threadIdx.x < p.batch ? clamp_context(p, p.context_lens[threadIdx.x]) : 0;
+  auto seq_len = [&](int b) {
+    return b == static_cast<int>(threadIdx.x) ? my_len : clamp_context(p, p.context_lens[b]);
+  };
   {
     unsigned long long mine = 0;
     for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
-      const int L = clamp_context(p, p.context_lens[b]);
+      const int L = seq_len(b);
       if (L > 0) mine += static_cast<unsigned long long>(L - seq_span(p, L).base);
     }
     for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
@@ -1450,7 +1460,7 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   const int full_tiles = max(pt / 16, 1);
   // items of sequence b: np partitions, all full but the last (class bk)
   auto shape = [&](int b, int& np, int& bk) {
-    const int L = clamp_context(p, p.context_lens[b]);
+    const int L = seq_len(b);
     np = partitions_of(p, L, pt);
     if (np == 0) {  // L == 0: one item, the zero row
       np = 1;
@@ -1467,15 +1477,38 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
     atomicAdd(&s_hist[bk], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int at = 0;
-    for (int k = kPlanBuckets; k >= 0; --k) {
-      s_start[k] = at;
-      at += s_hist[k];
+  if (threadIdx.x < 32) {
+    // each class's first slot, largest class first: an exclusive scan of the
+    // histogram taken from bucket kPlanBuckets down, by one warp (lane l
+    // holds positions PER*l .. PER*l + PER - 1 of that order)
+    constexpr int PER = (kPlanBuckets + 1 + 31) / 32;
+    const int lane = threadIdx.x;
+    int v[PER];
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int r = lane * PER + j;
+      v[j] = r <= kPlanBuckets ? s_hist[kPlanBuckets - r] : 0;
+      sum += v[j];
     }
-    p.work_count[0] = 0;   // the decode's ticket counter
-    p.work_count[1] = at;  // items
-    p.work_count[2] = pt;  // partition length
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int at = incl - sum;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int r = lane * PER + j;
+      if (r <= kPlanBuckets) s_start[kPlanBuckets - r] = at;
+      at += v[j];
+    }
+    if (lane == 31) {
+      p.work_count[0] = p.list_slots;  // the decode's ticket counter, past the first units
+      p.work_count[1] = incl;  // items
+      p.work_count[2] = pt;    // partition length
+    }
   }
   __syncthreads();
   // (the order within a class is whatever the atomics give: every item is
