@@ -68,7 +68,7 @@ extern "C" {
 typedef enum pa_status {
   PA_OK = 0,
   PA_ERR_INVALID_ARG = 1,   /* a host-side argument check failed */
-  PA_ERR_UNSUPPORTED = 2,   /* valid, but a dtype/shape this build has no kernel for */
+  PA_ERR_UNSUPPORTED = 2,   /* valid, but a dtype/shape the library has no kernel for */
   PA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
   PA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
   PA_ERR_DEVICE_BOUNDS = 5  /* pa_get_device_error: a kernel saw an out-of-range value */

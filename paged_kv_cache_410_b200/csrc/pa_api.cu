@@ -557,7 +557,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library).
+// against the CUDA driver library).
 EncodeTiledFn encode_tiled() {
   static const EncodeTiledFn fn = [] {
     void* f = nullptr;

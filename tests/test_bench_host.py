@@ -133,7 +133,7 @@ def test_small_fp8_batches_scale_the_beam_groups():
 
 def test_reference_arm_config_equals_the_gpu_arms():
     """Both arms describe the same workload with the same config object, the
-    decode path included (the driver compares them)."""
+    decode path included, so that their lines can be compared key for key."""
     env = dict(os.environ, PYTHONPATH=ROOT)
     for extra in ([], ["--no-flush"]):
         r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
