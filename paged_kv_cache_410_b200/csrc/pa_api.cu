@@ -241,10 +241,11 @@ pa_status launch_reduce(const pa::DecodeParams& p, cudaStream_t st) {
 // into partitions): the workspace holds the list, and the units (items x KV
 // head groups) stay below 2^31. The plan kernel may lengthen the partitions
 // by up to 2^kListGrowLog2 (fewer units and partials when the batch's
-// tokens allow; the workspace, sized for the host's length, holds fewer).
+// tokens allow; the workspace, sized for the host's length, holds fewer):
+// up to 4 times by doubling, up to 8 times to hold every sequence whole.
 // The suffix decode of a cascade keeps its grid (its sequences have one
 // partition or few, visited longest first).
-constexpr int kListGrowLog2 = 2;
+constexpr int kListGrowLog2 = 3;
 
 bool use_work_list(const pa::DecodeParams& p, bool dependent) {
   return !dependent && p.prefix_blocks == 0 && p.work_items && !p.cp_o && p.batch > 1 &&

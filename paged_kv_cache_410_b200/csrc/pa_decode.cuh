@@ -1420,16 +1420,24 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   __shared__ int s_hist[kPlanBuckets + 1];
   __shared__ int s_start[kPlanBuckets + 1];
   __shared__ unsigned long long s_work;
+  __shared__ int s_span;
   __shared__ int s_pt;
   // the decode grid may be placed now; it waits for this grid to complete
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int i = threadIdx.x; i <= kPlanBuckets; i += kPlanThreads) s_hist[i] = 0;
-  if (threadIdx.x == 0) s_work = 0;
+  if (threadIdx.x == 0) {
+    s_work = 0;
+    s_span = 0;
+  }
   __syncthreads();
-  // The partition length: the host's times 1, 2 or 4 (within the room the
-  // launch staged for block ids), the longest whose item is at most 3/4 of a
-  // slot's share of the batch's tokens x head groups. Longer partitions
-  // mean fewer units and partials; the largest items still start first.
+  // The partition length. When one partition can hold every sequence's
+  // attended span (within the room the launch staged for block ids, up to
+  // 8 times the host's length) and the batch still has 4 waves of units
+  // (sequences x head groups against the grid's CTAs), that: no sequence is
+  // split and there is nothing to merge. Otherwise the host's times 1, 2 or
+  // 4, the longest whose item is at most 3/2 of a slot's share of the
+  // batch's tokens x head groups. Longer partitions mean fewer units and
+  // partials; the largest items still start first.
   // (each thread keeps the length of its first sequence: the passes below
   // read it again, and a batch of up to kPlanThreads has no other)
   const int my_len = threadIdx.x < p.batch ? clamp_context(p, p.context_lens[threadIdx.x]) : 0;
@@ -1438,21 +1446,40 @@ __global__ void __launch_bounds__(kPlanThreads) pa_decode_plan_kernel(const Deco
   };
   {
     unsigned long long mine = 0;
+    int span = 0;
     for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
       const int L = seq_len(b);
-      if (L > 0) mine += static_cast<unsigned long long>(L - seq_span(p, L).base);
+      if (L > 0) {
+        const int n = L - seq_span(p, L).base;
+        mine += static_cast<unsigned long long>(n);
+        span = max(span, n);
+      }
     }
-    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
-    if ((threadIdx.x & 31) == 0) atomicAdd(&s_work, mine);
+    for (int o = 16; o > 0; o >>= 1) {
+      mine += __shfl_xor_sync(0xffffffffu, mine, o);
+      span = max(span, __shfl_xor_sync(0xffffffffu, span, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      atomicAdd(&s_work, mine);
+      atomicMax(&s_span, span);
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const unsigned long long share =
-        s_work * static_cast<unsigned long long>(units_per_item(p)) * 3 /
-        (4ull * static_cast<unsigned long long>(max(p.list_slots, 1)));
-    int pt = p.partition_tokens;
-    const int cap = max(p.partition_tokens, p.max_partition_tokens);
-    while (2 * pt <= cap && static_cast<unsigned long long>(2 * pt) <= share) pt *= 2;
+    const int host = p.partition_tokens;
+    const int cap = max(host, p.max_partition_tokens);
+    const int whole = (s_span + 15) & ~15;
+    int pt = host;
+    if (whole > host && whole <= cap &&
+        static_cast<int64_t>(p.batch) * units_per_item(p) >= 4ll * max(p.list_slots, 1)) {
+      pt = whole;
+    } else {
+      const unsigned long long share =
+          s_work * static_cast<unsigned long long>(units_per_item(p)) * 3 /
+          (2ull * static_cast<unsigned long long>(max(p.list_slots, 1)));
+      const int cap4 = min(cap, 4 * host);
+      while (2 * pt <= cap4 && static_cast<unsigned long long>(2 * pt) <= share) pt *= 2;
+    }
     s_pt = pt;
   }
   __syncthreads();

@@ -6,7 +6,8 @@ full grid would: the output of each sequence is compared with the float64
 oracle (outputs start as NaN, so a unit never taken shows), and bit for bit
 with the same sequence decoded alone (a batch of one keeps the full grid)
 with the partition length the plan kernel chose (read back from the
-workspace, where the plan publishes it: 1, 2 or 4 times the host's) and a
+workspace, where the plan publishes it: 1, 2 or 4 times the host's, or up to
+8 times it to hold the longest sequence whole) and a
 plan of as many partitions as the batch's launch had, so that the merge
 runs the same code. The decodes alone ask for reproducible results, which
 keeps each CTA on its own partition (no steal mode)."""
@@ -57,7 +58,12 @@ def listed_vs_alone(w, pt, window=0, fused=False, repeats=2):
     list_at = (-(-(rows * n_parts * w.head_dim * 4) // 256) * 256 +
                -(-(rows * n_parts * 8) // 256) * 256)
     pt_used = int(step.workspace[list_at + 8:list_at + 12].view(torch.int32).item())
-    assert pt_used in (pt, 2 * pt, 4 * pt), (pt, pt_used)
+    # the longest attended span (a window's starts at its 16-aligned base)
+    lens = step.context_lens.cpu().numpy().astype(int)
+    bases = [((L - window) & ~15) if window and L > window else 0 for L in lens]
+    longest = max([L - b for L, b in zip(lens, bases)] + [0])
+    assert pt_used % 16 == 0 and pt <= pt_used <= 8 * pt, (pt, pt_used)
+    assert pt_used in (pt, 2 * pt, 4 * pt) or pt_used >= longest, (pt, pt_used, longest)
     # each sequence alone: the full grid at that length, with a plan of as
     # many partitions (the merge picks its code by the plan's count; a
     # window's plan spans window + 15 tokens whatever max_context is)
